@@ -1,0 +1,375 @@
+"""Benchmark: effective weight bandwidth of the compressed Llama-3.1-8B MLP.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload (one "step"): one Llama-3.1-8B-shaped MLP layer -- gate and up
+[14336, 4096], down [4096, 14336], BF16 N(0, 0.02^2) with 0.05% N(0, 1)
+outliers (seeds 1, 2, 3; rank r adds 100 r) -- multiplied by activations X of
+M = 1, 4, 16 and 64 rows (12 matmuls, Y = X W^T, fp32 out).  Each
+(projection, M) runs the plan picked by libuw's autotuner (full decode +
+plain kernel, runtime transcode + fused kernel, or direct palette + fused
+kernel; FMA GEMV or tcgen05).  Matmuls are issued M-outer / projection-inner,
+so two other matrices (>= 160 MB) stream between two uses of one matrix and
+each read comes from HBM, not from the 126 MB L2.
+
+value  = sum over the step's matmuls of 2*N*K (uncompressed BF16 weight bytes)
+         / step time  [GB/s], inputs resident in HBM, CUDA events, max over ranks.
+e2e    = the same, with X copied from pinned host memory and Y read back to
+         pinned host memory inside the timed region, through the C ABI.
+roofline: the kernel group with the largest share of the step; achieved =
+         its algorithmic bytes (compressed planes + X + Y) / its event-timed
+         duration, against the measured HBM copy bandwidth.
+cpu_baseline: the CPU oracle (decode + float64 matmul) on a bounded sample.
+
+Multi-GPU: every rank owns an independent layer (weak scaling, no collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+MS = (1, 4, 16, 64)
+PROJ = (("gate", 14336, 4096), ("up", 14336, 4096), ("down", 4096, 14336))
+METRIC = "effective weight GB/s & fused matmul TFLOP/s at M=1..1024 vs HBM/tensor roofline"
+WORKLOAD = "llama-3.1-8b MLP layer (gate/up/down), M in {1,4,16,64}, autotuned plans"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(budget_s: float = 25.0):
+    """Oracle pipeline (bit-by-bit Huffman decode + float64 matmul) for the gate
+    projection at M = 1, 4, 16, 64, decoding once per M as the pipeline does.
+    Stops after the M whose cumulative time passes budget_s."""
+    from oracle import oracle as O
+    from decode_gemm_exponent_b200 import synth
+    n, k = PROJ[0][1], PROJ[0][2]
+    w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1)
+    enc = O.encode(w)                      # offline, untimed
+    done_bytes, t_total, done = 0, 0.0, []
+    for m in MS:
+        x = synth.activations_bf16(m, k, seed=1)
+        t0 = time.perf_counter()
+        wd = O.decode(enc)
+        O.gemm(x, wd)
+        t_total += time.perf_counter() - t0
+        done_bytes += 2 * n * k
+        done.append(m)
+        if t_total > budget_s:
+            break
+    return done_bytes / t_total / 1e9, "gate [14336,4096] at M in %s, decode + float64 matmul" % (done,), t_total
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    from oracle import oracle as O
+    from decode_gemm_exponent_b200 import synth
+    n, k = PROJ[0][1], PROJ[0][2]
+    w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1)
+    enc = O.encode(w)
+    x = synth.activations_bf16(1, k, seed=1)
+
+    def step():
+        wd = O.decode(enc)
+        O.gemm(x, wd)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2 * n * k / dt / 1e9
+    sample = "gate [14336,4096] at M=1 per step: bit-by-bit Huffman decode + float64 matmul"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "reference_sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+def alg_bytes(mat, m, plan):
+    """Algorithmic HBM bytes of the kernels one matmul call launches."""
+    info = mat.info
+    n, k = mat.n, mat.k
+    common = info.section_bytes[0] + info.section_bytes[1] + (n * k // 64) // 8 * 2   # sm + raw + flags/base
+    xy = m * k * 2 + m * n * 4
+    if plan.pipeline == 4:
+        return {"fused": common + n * k // 2 + xy}
+    huff_in = common + (info.stream_bits + 7) // 8 + (info.n_chunks + 1) * 4
+    if plan.pipeline == 1:
+        return {"decode": huff_in + 2 * n * k, "plain": 2 * n * k + xy}
+    return {"transcode": huff_in + n * k // 2, "fused": common + n * k // 2 + xy}
+
+
+def launches_per_call(plan):
+    n = 1 + (1 if plan.pipeline in (1, 3) else 0)
+    if plan.kernel == 2 and plan.split_k > 1:
+        n += 1
+    return n
+
+
+def kernel_group(plan):
+    kern = "fma_gemv" if plan.kernel == 1 else "tcgen05_bn%d" % plan.bn
+    pipe = {1: "decode+plain", 3: "transcode+fused", 4: "fused"}[plan.pipeline]
+    return "%s/%s" % (pipe, kern)
+
+
+def run_gpu(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from decode_gemm_exponent_b200 import synth, uw
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    # ---- inputs (host encode is the offline step, outside any timing)
+    mats = []
+    for i, (name, n, k) in enumerate(PROJ):
+        w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1 + i + 100 * rank)
+        mats.append(uw.Matrix(uw.encode(w), device=dev))
+    xs = {m: {k: torch.from_numpy(synth.activations_bf16(m, k, seed=m).view(np.int16)).to(dev)
+              for k in {p[2] for p in PROJ}} for m in MS}
+
+    plans, plan_json = uw.autotune(mats, list(MS), reps=10)
+    calls = []
+    for j, m in enumerate(MS):
+        for i, mat in enumerate(mats):
+            p = plans[i][j]
+            nb = mat.workspace_bytes(m, p)
+            ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+            y = torch.empty(m, mat.n, dtype=torch.float32, device=dev)
+            calls.append(dict(mat=mat, m=m, plan=p, ws=ws, y=y, x=xs[m][mat.k], name=PROJ[i][0]))
+    stream = torch.cuda.current_stream()
+
+    def issue(c):
+        c["mat"].matmul(c["x"], c["plan"], y=c["y"], ws=c["ws"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        for c in calls:
+            issue(c)
+    for mat in mats:
+        st = mat.device_status()
+        if st != 0:
+            raise RuntimeError("kernel status %d during warm-up" % st)
+
+    # ---- device-resident timing, one event pair per call
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            for c, (e0, e1) in zip(calls, ev[s]):
+                e0.record(stream)
+                issue(c)
+                e1.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    if world > 1:
+        t = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    weight_bytes = sum(2 * c["mat"].n * c["mat"].k for c in calls)
+    value = weight_bytes * world / (step_ms * 1e-3) / 1e9
+
+    # per-call durations -> kernel groups
+    per_call = [statistics.median(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps))
+                for i in range(len(calls))]
+    groups = {}
+    for c, ms_ in zip(calls, per_call):
+        g = groups.setdefault(kernel_group(c["plan"]), {"ms": 0.0, "bytes": 0, "calls": 0})
+        g["ms"] += ms_
+        g["bytes"] += sum(alg_bytes(c["mat"], c["m"], c["plan"]).values())
+        g["calls"] += 1
+    dom_name, dom = max(groups.items(), key=lambda kv: kv[1]["ms"])
+    achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+
+    # ---- end-to-end through the C ABI with pinned host buffers
+    hx = {(c["m"], c["mat"].k): c["x"].cpu().pin_memory() for c in calls}
+    hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
+    h2d = sum(t.numel() * 2 for t in hx.values())
+    d2h = sum(t.numel() * 4 for t in hy)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        for key, t in hx.items():
+            xs[key[0]][key[1]].copy_(t, non_blocking=True)
+        for c, h in zip(calls, hy):
+            issue(c)
+            h.copy_(c["y"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    for mat in mats:
+        st = mat.device_status()
+        if st != 0:
+            raise RuntimeError("kernel status %d after timing" % st)
+
+    if rank != 0:
+        return 0
+    clocks = clk.summary()
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, sample, secs = oracle_sample()
+        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+               "seconds": round(secs, 2)}
+    infos = [m.info for m in mats]
+    out = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD,
+            "l2": "no flush: each matrix is re-read after >= 160 MB of other matrices (inputs larger than L2)",
+            "compressed_fraction_huffman": round(sum(i.huffman_bytes for i in infos) /
+                                                 sum(2 * i.n * i.k for i in infos), 4),
+            "compressed_fraction_palette": round(sum(i.palette_bytes for i in infos) /
+                                                 sum(2 * i.n * i.k for i in infos), 4),
+            "plans": {"%s@M=%d" % (c["name"], c["m"]): kernel_group(c["plan"]) +
+                      ("/split%d" % c["plan"].split_k if c["plan"].kernel == 2 else "") for c in calls},
+            "per_call_us": {"%s@M=%d" % (c["name"], c["m"]): round(1e3 * t, 2) for c, t in zip(calls, per_call)},
+        },
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": peaks["_source"] + " hbm_gbs"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": weight_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": sum(launches_per_call(c["plan"]) for c in calls) * args.steps,
+        "clocks": clocks,
+    }
+    if args.plan_json:
+        with open(args.plan_json, "w") as f:
+            f.write(plan_json)
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plan-json", default=None, help="write the autotuner's plan file here")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_gpu(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,170 @@
+// autotune.cu -- measured plan selection (Unweight page §九: no single
+// pipeline wins everywhere, so an autotuner times the candidates on the target
+// GPU for every projection and batch size and writes a per-model plan file).
+//
+// For each matrix and each batch size m the candidates are the pipelines the
+// blob supports (decode + plain kernel, runtime transcode + fused kernel,
+// direct palette + fused kernel) crossed with the kernel variants: the FMA
+// GEMV (m <= 8, 1 or 2 rows per warp) and the tcgen05 kernel with token tiles
+// around m and split-K factors that fill the 148 SMs.  Each candidate is run
+// once to warm up (its status is checked) and then `reps` times between CUDA
+// events; the fastest average wins.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kernels.h"
+#include "uw_format.h"
+
+namespace {
+
+constexpr int kSMs = 148;
+
+std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
+    std::vector<int> pipes;
+    if (w.flags & UW_EMIT_HUFFMAN) {
+        pipes.push_back(UW_PIPE_DECODE_GEMM);
+        pipes.push_back(UW_PIPE_TRANSCODE_FUSED);
+    }
+    if ((w.flags & UW_EMIT_PALETTE) && w.pal) pipes.push_back(UW_PIPE_DIRECT_PALETTE);
+    std::vector<uw_plan> out;
+    for (int pipe : pipes) {
+        if (m <= 8)
+            for (int rows : {1, 2}) {
+                uw_plan p{};
+                p.pipeline = pipe;
+                p.kernel = UW_KERNEL_FMA;
+                p.bn = rows;
+                p.split_k = 1;
+                out.push_back(p);
+            }
+        int bn_hi = 16;
+        while (bn_hi < m && bn_hi < 256) bn_hi *= 2;
+        for (int bn : {bn_hi / 2, bn_hi}) {
+            if (bn < 16) continue;
+            const int64_t tiles = ((w.n + 127) / 128) * ((m + bn - 1) / bn);
+            const int ksteps = int(w.k / 64);
+            for (int split : {1, 2, 4, 8}) {
+                if (split > 1 && (tiles * split > 4 * kSMs || ksteps / split < 4)) continue;
+                if (split > 1 && tiles >= 2 * kSMs) continue;
+                uw_plan p{};
+                p.pipeline = pipe;
+                p.kernel = UW_KERNEL_TC;
+                p.bn = bn;
+                p.split_k = split;
+                out.push_back(p);
+            }
+        }
+    }
+    return out;
+}
+
+const char *pipe_name(int p) {
+    return p == UW_PIPE_DECODE_GEMM ? "decode_gemm" : p == UW_PIPE_TRANSCODE_FUSED ? "transcode_fused"
+                                                                                 : "direct_palette";
+}
+
+std::string plan_json(const uw_plan &p, double us) {
+    char buf[256];
+    std::snprintf(buf, sizeof buf,
+                  "{\"pipeline\": \"%s\", \"kernel\": \"%s\", \"bn\": %d, \"split_k\": %d, \"us\": %.3f}",
+                  pipe_name(p.pipeline), p.kernel == UW_KERNEL_FMA ? "fma" : "tc", p.bn, p.split_k, us);
+    return buf;
+}
+
+}  // namespace
+
+extern "C" uw_status uw_autotune_workspace_size(const uw_dmat *const *mats, int n_mats,
+                                                const int64_t *ms, int n_ms, size_t *bytes) {
+    if (!mats || !ms || !bytes || n_mats <= 0 || n_ms <= 0) return UW_ERR_INVALID_ARG;
+    size_t best = 0;
+    for (int i = 0; i < n_mats; i++) {
+        if (!mats[i]) return UW_ERR_INVALID_ARG;
+        for (int j = 0; j < n_ms; j++) {
+            if (ms[j] <= 0) return UW_ERR_INVALID_ARG;
+            for (const uw_plan &p : candidates(*mats[i], ms[j])) {
+                size_t b = 0;
+                uw_status st = uw_workspace_size(ms[j], mats[i]->n, mats[i]->k, &p, &b);
+                if (st != UW_OK) return st;
+                best = std::max(best, b);
+            }
+        }
+    }
+    *bytes = best;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_plan_autotune(const uw_dmat *const *mats, int n_mats, const int64_t *ms,
+                                      int n_ms, const uint16_t *x_dev, float *y_dev, void *ws,
+                                      size_t ws_bytes, int reps, uw_plan *plans_out, char *json_out,
+                                      size_t json_cap, void *stream) {
+    if (!mats || !ms || !x_dev || !y_dev || !plans_out || n_mats <= 0 || n_ms <= 0) return UW_ERR_INVALID_ARG;
+    if (reps <= 0) reps = 5;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t e0, e1;
+    if (cudaEventCreate(&e0) != cudaSuccess) return UW_ERR_CUDA;
+    if (cudaEventCreate(&e1) != cudaSuccess) {
+        cudaEventDestroy(e0);
+        return UW_ERR_CUDA;
+    }
+    std::string json = "{\"plans\": [";
+    uw_status result = UW_OK;
+    for (int i = 0; i < n_mats && result == UW_OK; i++) {
+        const uw_dmat &w = *mats[i];
+        for (int j = 0; j < n_ms && result == UW_OK; j++) {
+            const int64_t m = ms[j];
+            double best_us = 1e30;
+            uw_plan best{};
+            std::string cand_json;
+            for (const uw_plan &p : candidates(w, m)) {
+                uw_status st = uw_fused_matmul(x_dev, m, &w, nullptr, y_dev, &p, ws, ws_bytes, stream);
+                if (st == UW_OK) st = w.dev_status ? uw_device_status(&w, stream)
+                                                   : (cudaStreamSynchronize(s) == cudaSuccess ? UW_OK : UW_ERR_CUDA);
+                if (st != UW_OK) {
+                    if (st == UW_ERR_CUDA) {
+                        result = st;
+                        break;
+                    }
+                    continue;   // candidate not runnable here (e.g. workspace too small)
+                }
+                cudaEventRecord(e0, s);
+                for (int r = 0; r < reps; r++) uw_fused_matmul(x_dev, m, &w, nullptr, y_dev, &p, ws, ws_bytes, stream);
+                cudaEventRecord(e1, s);
+                if (cudaEventSynchronize(e1) != cudaSuccess) {
+                    result = UW_ERR_CUDA;
+                    break;
+                }
+                float ms_el = 0.f;
+                cudaEventElapsedTime(&ms_el, e0, e1);
+                const double us = 1000.0 * ms_el / reps;
+                if (!cand_json.empty()) cand_json += ", ";
+                cand_json += plan_json(p, us);
+                if (us < best_us) {
+                    best_us = us;
+                    best = p;
+                }
+            }
+            if (result != UW_OK) break;
+            if (best_us >= 1e30) {
+                result = UW_ERR_WORKSPACE;
+                break;
+            }
+            plans_out[i * n_ms + j] = best;
+            char head[160];
+            std::snprintf(head, sizeof head, "%s{\"matrix\": %d, \"n\": %lld, \"k\": %lld, \"m\": %lld, \"best\": ",
+                          (i == 0 && j == 0) ? "" : ", ", i, (long long)w.n, (long long)w.k, (long long)m);
+            json += head + plan_json(best, best_us) + ", \"candidates\": [" + cand_json + "]}";
+        }
+    }
+    json += "]}";
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (result != UW_OK) return result;
+    if (json_out) {
+        if (json.size() + 1 > json_cap) return UW_ERR_INVALID_ARG;
+        std::memcpy(json_out, json.c_str(), json.size() + 1);
+    }
+    return UW_OK;
+}

@@ -1,0 +1,250 @@
+// device_common.cuh -- sm_100a device helpers for libuw kernels:
+// bounded mbarrier waits, bulk/tensor TMA copies, tcgen05 (TMEM + MMA)
+// wrappers, and the BF16 rebuild arithmetic of the Unweight page (§四: the
+// sign/mantissa byte is raw, the exponent byte comes from a 16-entry palette
+// or from the raw plane).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/uw.h"
+
+namespace uw {
+namespace dev {
+
+// ---------------------------------------------------------------- misc
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void flag_error(uint32_t *status, uint32_t bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// byte permute (PTX prmt, default mode: selector bit 3 replicates the sign
+// bit of the selected byte)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }" ::"r"(
+            smem_addr(bar)),
+        "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait until the phase with the given parity has completed, or until
+// `timeout_ns` of wall time has passed.  Returns false on time-out.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > timeout_ns) return false;
+    }
+}
+
+// ---------------------------------------------------------------- TMA
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes and
+// both addresses must be multiples of 16).
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// 2-D tiled tensor copy global -> shared (x = innermost coordinate).
+__device__ __forceinline__ void tma_load_2d(void *dst_smem, const CUtensorMap *map, int32_t x,
+                                            int32_t y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// generic-proxy shared-memory writes -> visible to the async proxy (MMA, TMA)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (BF16 in, FP32 accumulate)
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// arrive on `bar` once all previously issued tcgen05.mma of this thread finish
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
+// 32 lanes x 32 bit, 16 consecutive columns per thread
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major tile whose rows are 128 bytes
+// (64 BF16), stored with the 128-byte swizzle in 1024-byte atoms of 8 rows.
+__device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr & 0x3FFFFu) >> 4);        // start address
+    d |= uint64_t(1) << 16;                         // leading byte offset (unused here)
+    d |= uint64_t(1024 >> 4) << 32;                 // stride byte offset: 8 rows * 128 B
+    d |= uint64_t(1) << 46;                         // descriptor version (sm_100)
+    d |= uint64_t(2) << 61;                         // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: kind::f16, A = B = BF16, D = F32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- rebuild
+
+struct Palette16 {
+    uint32_t p0, p1, p2, p3;   // palette[0..3], [4..7], [8..11], [12..15] as bytes
+};
+
+// One 4-bit-palette word (8 weights) -> their exponent bytes: e0 = weights
+// 0..3, e1 = weights 4..7 (one byte each, weight 0 lowest).  The low three
+// index bits are prmt selectors into the 8-byte half-palettes; bit 3 of each
+// index sits in a byte's top bit (of the word, or of the word shifted by 4),
+// so a sign-replicating prmt turns it into a whole-byte mask.
+__device__ __forceinline__ void pal_exponents(uint32_t x, const Palette16 &P, uint32_t &e0,
+                                              uint32_t &e1) {
+    const uint32_t s0 = x & 0x7777u;
+    const uint32_t s1 = (x >> 16) & 0x7777u;
+    const uint32_t m0 = prmt(x, 0u, 0xBA98u);
+    const uint32_t m1 = prmt(x << 4, 0u, 0xBA98u);
+    const uint32_t lo0 = prmt(P.p0, P.p1, s0), hi0 = prmt(P.p2, P.p3, s0);
+    const uint32_t lo1 = prmt(P.p0, P.p1, s1), hi1 = prmt(P.p2, P.p3, s1);
+    e0 = (hi0 & m0) | (lo0 & ~m0);
+    e1 = (hi1 & m1) | (lo1 & ~m1);
+}
+
+// t = [e1 sm1 e0 sm0] (bytes, low first) -> two BF16 patterns
+// s<<15 | e<<7 | m in the low and high halves.
+__device__ __forceinline__ uint32_t join2(uint32_t t) {
+    const uint32_t a = t >> 1;
+    const uint32_t c = t << 8;
+    const uint32_t sel = (t & 0x007F007Fu) | (c & ~0x007F007Fu);
+    return (a & 0x7F807F80u) | (sel & ~0x7F807F80u);
+}
+
+// 4 exponents (e) + 4 sign/mantissa bytes (s) -> 4 BF16 in two words
+__device__ __forceinline__ void join4(uint32_t e, uint32_t s, uint32_t &w01, uint32_t &w23) {
+    w01 = join2(prmt(s, e, 0x5140u));
+    w23 = join2(prmt(s, e, 0x7362u));
+}
+
+// 8 weights: exponents (e0,e1) + sm bytes (s0,s1) -> uint4 of 8 BF16
+__device__ __forceinline__ uint4 join8(uint32_t e0, uint32_t e1, uint32_t s0, uint32_t s1) {
+    uint4 r;
+    join4(e0, s0, r.x, r.y);
+    join4(e1, s1, r.z, r.w);
+    return r;
+}
+
+// 8 palette indices in natural order (index j in bits 4j..4j+3) -> the
+// stored 4-bit-palette word layout (index bit 3 moved to a byte top bit).
+__device__ __forceinline__ uint32_t natural_to_pal(uint32_t x) {
+    const uint32_t low3 = x & 0x77777777u;
+    const uint32_t b = (x >> 3) & 0x11111111u;                          // bit 3 of j at bit 4j
+    const uint32_t vlo = (((b & 0x1111u) * 0x1248u) >> 12) & 0xFu;      // j = 0..3 -> bits 0..3
+    const uint32_t vhi = ((((b >> 16) & 0x1111u) * 0x1248u) >> 12) & 0xFu;  // j = 4..7
+    return low3 | ((vlo * 0x10204080u) & 0x80808080u) | ((vhi * 0x01020408u) & 0x08080808u);
+}
+
+}  // namespace dev
+}  // namespace uw

@@ -1,0 +1,52 @@
+// kernels.h -- host-side launch interface of the libuw CUDA kernels (internal).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/uw.h"
+
+namespace uw {
+
+// Huffman decode of a whole matrix (Unweight page §六, pipelines 1 and 3).
+// out_bf16 != nullptr: write BF16 [n*k]; out_pal != nullptr: write the
+// 4-bit palette plane [n*k/2].  Exactly one must be non-null.
+cudaError_t launch_huff_decode(const uw_dmat &w, uint16_t *out_bf16, uint8_t *out_pal,
+                               cudaStream_t stream);
+
+// CUDA-core FMA GEMV, m <= 8 (Unweight page §七, small-batch case).
+// pal_plane == nullptr: plain BF16 weights `w_bf16`; otherwise the fused
+// palette path using `w` (sm/raw planes) and `pal_plane`.
+cudaError_t launch_gemv_fma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
+                            const uint8_t *pal_plane, int64_t n, int64_t k, float *y,
+                            int rows_per_warp, cudaStream_t stream);
+
+// tcgen05 GEMM (Unweight page §七, reconstructive matmul), token tile `bn`.
+struct TcLaunch {
+    const uint16_t *x;         // [m, k] BF16
+    int64_t m, n, k;
+    const uint16_t *w_bf16;    // plain path (nullptr for the fused path)
+    const uw_dmat *w;          // fused path: sm/raw/flag planes
+    const uint8_t *pal;        // fused path: palette plane
+    float *y;                  // [m, n]
+    float *partial;            // [split_k, m, n] when split_k > 1
+    int bn, split_k, stages;
+    uint32_t debug_flags;
+    uint64_t timeout_ns;
+    uint32_t *dev_status;
+};
+cudaError_t launch_gemm_tc(const TcLaunch &p, cudaStream_t stream);
+
+// Fixed-order sum of split-K partials: y[i] = sum_s partial[s][i], s ascending.
+cudaError_t launch_splitk_reduce(const float *partial, int split_k, int64_t count, float *y,
+                                 cudaStream_t stream);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once through the
+// runtime so that the library needs no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+}  // namespace uw

@@ -1,0 +1,251 @@
+/*
+ * uw.h -- C ABI of libuw: lossless BF16 exponent compression with fused
+ * decode-matmul kernels for NVIDIA B200 (sm_100a).
+ *
+ * The method follows the web page "Unweight：Cloudflare 如何在不损失精度的情况下
+ * 把大模型压缩 22%" (cited below as "the Unweight page", by section number):
+ *   §三  a BF16 weight is 1 sign, 8 exponent and 7 mantissa bits; only the
+ *        exponent is predictable (few values dominate, ~2.6 bits of entropy).
+ *   §四  the sign+mantissa byte stays raw, the exponent byte is Huffman coded;
+ *        any row of 64 weights holding an exponent outside the matrix's top-16
+ *        palette is stored raw, so the hot loop needs no per-element branch.
+ *   §五  decompress next to the compute, never back to HBM, to save bandwidth.
+ *   §六  four pipelines: full decode + GEMM, exponent-only decode, runtime
+ *        Huffman -> 4-bit palette transcode, and pre-transcoded palette.
+ *   §七  reconstructive matmul: compressed tiles are staged into shared memory,
+ *        rebuilt to BF16 there and fed straight to the tensor cores.
+ *   §九  an autotuner measures the pipelines and kernel variants per
+ *        projection and batch size and writes a per-model plan.
+ *
+ * Conventions for every entry point:
+ *   - Returns a uw_status; nothing throws across the ABI.
+ *   - Matrices are row-major.  W is [n, k] (one output feature per row), X is
+ *     [m, k] BF16, Y is [m, n] float32, Y = X * W^T.  BF16 values are passed
+ *     as their raw 16-bit patterns (uint16_t).
+ *   - n and k must be positive multiples of 64 (UW_ERR_UNSUPPORTED_SHAPE).
+ *     Null required pointers, m <= 0 and bad plans give UW_ERR_INVALID_ARG.
+ *   - Device work is launched asynchronously on the given stream (a
+ *     cudaStream_t passed as void*; NULL = legacy default stream).  Argument
+ *     errors are reported synchronously.  Errors found by a kernel (corrupt
+ *     stream, spin-wait time-out) are OR-ed into the matrix's device status
+ *     word and returned by uw_device_status() after the stream is drained.
+ *   - The caller owns every device buffer: the device copy of a blob, its
+ *     status word, X, Y, decode/transcode outputs and workspaces.  The library
+ *     allocates no device memory.  It owns only the host blobs that uw_encode
+ *     returns; free them with uw_blob_free.
+ *   - Calls are thread-safe as long as no two calls write the same buffers.
+ */
+#ifndef UW_H
+#define UW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum uw_status {
+    UW_OK = 0,
+    UW_ERR_INVALID_ARG = 1,        /* null pointer, non-positive size, bad plan field */
+    UW_ERR_UNSUPPORTED_SHAPE = 2,  /* n or k not a multiple of 64, or too large */
+    UW_ERR_CORRUPT = 3,            /* blob header/CRC/section check failed, or a kernel
+                                      found an inconsistent bitstream */
+    UW_ERR_CUDA = 4,               /* a CUDA runtime call failed */
+    UW_ERR_NOMEM = 5,              /* host allocation failed */
+    UW_ERR_TIMEOUT = 6,            /* a kernel's bounded spin-wait ran out */
+    UW_ERR_WORKSPACE = 7           /* workspace missing or smaller than uw_workspace_size */
+} uw_status;
+
+/* Human-readable name of a status code (static string). */
+const char *uw_status_str(int status);
+/* Library version string, e.g. "uw 1.0 (blob v1, sm_100a)". */
+const char *uw_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Host encoder (Unweight page §三, §四, §六).                                */
+
+#define UW_EMIT_HUFFMAN 1u   /* Huffman exponent stream (pipelines 1 and 3)    */
+#define UW_EMIT_PALETTE 2u   /* pre-transcoded 4-bit palette plane (pipeline 4) */
+
+/* Sections of a blob (each 256-byte aligned inside the blob). */
+enum {
+    UW_SEC_SM = 0,        /* uint8[n*k]   sign<<7 | mantissa of every weight          */
+    UW_SEC_RAWEXP = 1,    /* uint8[n_raw*64] exponents of raw groups, group order      */
+    UW_SEC_FLAGS = 2,     /* uint32[] bit g%32 of word g/32 = group g is raw           */
+    UW_SEC_RAWBASE = 3,   /* uint32[] raw groups before word w of FLAGS (prefix count) */
+    UW_SEC_STREAM = 4,    /* uint32[] Huffman bits, MSB of each word first, 0-padded   */
+    UW_SEC_CHUNKOFF = 5,  /* uint32[n_chunks+1] start bit of each 4-group chunk        */
+    UW_SEC_DLUT = 6,      /* uint32[4096] 12-bit-window multi-symbol decode table      */
+    UW_SEC_PAL = 7,       /* uint8[n*k/2] 4-bit palette indices: each little-endian
+                             u32 word holds 8 consecutive weights; weight j's index v
+                             has v&7 at bits 4j..4j+2 and v>>3 at bit 8j+7 (j<4) or
+                             bit 8(j-4)+3 (j>=4); raw groups hold 0                */
+    UW_NUM_SECTIONS = 8
+};
+
+typedef struct uw_blob uw_blob;   /* opaque host-side serialized matrix */
+
+typedef struct uw_blob_info {
+    int64_t n, k;
+    uint32_t flags;              /* UW_EMIT_* present in the blob */
+    int32_t palette_size;        /* 1..16 */
+    uint8_t palette[16];         /* exponent values, ascending; index = position */
+    uint8_t code_len[16];        /* Huffman code length per palette index (0 = unused) */
+    int64_t n_groups;            /* n*k/64 */
+    int64_t n_raw;               /* raw groups */
+    int64_t n_chunks;            /* ceil(n_groups/4) */
+    uint64_t stream_bits;
+    double entropy_bits;         /* Shannon entropy of the 256-bin exponent histogram */
+    double top16_coverage;       /* fraction of weights whose exponent is in the palette */
+    uint64_t total_bytes;        /* serialized size */
+    uint64_t huffman_bytes;      /* bytes needed to keep the Huffman form */
+    uint64_t palette_bytes;      /* bytes needed to keep the palette form */
+    uint64_t section_offset[UW_NUM_SECTIONS];
+    uint64_t section_bytes[UW_NUM_SECTIONS];
+} uw_blob_info;
+
+/* Encode one BF16 matrix w[n,k] (host memory, raw bit patterns).
+ * flags: UW_EMIT_HUFFMAN and/or UW_EMIT_PALETTE (0 means both).
+ * On success *out owns a new blob (free with uw_blob_free).  Bit-exact and
+ * deterministic: the same input always gives the same bytes.
+ * Errors: INVALID_ARG (null), UNSUPPORTED_SHAPE (n,k not multiples of 64, or a
+ * Huffman stream that would exceed 2^32 bits), NOMEM.                        */
+uw_status uw_encode(const uint16_t *w, int64_t n, int64_t k, uint32_t flags, uw_blob **out);
+
+/* Pointer to the serialized bytes of a blob and their count (owned by blob). */
+const void *uw_blob_data(const uw_blob *blob, size_t *bytes);
+void uw_blob_free(uw_blob *blob);
+
+/* Parse and check a serialized blob held in host memory (e.g. read from
+ * disk).  Checks magic, version, header CRC and section bounds; with
+ * verify_payload != 0 also the CRC over all sections.  Fills *info.        */
+uw_status uw_blob_info_get(const void *host_blob, size_t bytes, int verify_payload,
+                           uw_blob_info *info);
+
+/* ------------------------------------------------------------------------ */
+/* Device view of a blob.                                                     */
+
+typedef struct uw_dmat {
+    int64_t n, k;
+    uint32_t flags;
+    int32_t palette_size;
+    uint8_t palette[16];
+    uint8_t code_len[16];
+    int64_t n_groups, n_raw, n_chunks;
+    uint64_t stream_bits;
+    uint64_t stream_words;          /* padded word count of the stream section */
+    const uint8_t *sm;              /* device pointers into the device blob */
+    const uint8_t *rawexp;
+    const uint32_t *flagbits;
+    const uint32_t *rawbase;
+    const uint32_t *stream;
+    const uint32_t *chunk_off;
+    const uint32_t *dlut;
+    const uint8_t *pal;             /* NULL if the blob has no palette plane */
+    uint32_t *dev_status;           /* caller's device word for kernel error flags */
+} uw_dmat;
+
+/* Bind a device copy of a blob.  host_blob/bytes is a host copy used to read
+ * the header (no device read happens); dev_blob must hold the same bytes and
+ * be 256-byte aligned.  dev_status points to one caller-owned device uint32
+ * (zero it before use) that kernels OR error bits into.  verify_payload as in
+ * uw_blob_info_get.  Fills *out; keeps no reference to host_blob.            */
+uw_status uw_matrix_bind(const void *host_blob, size_t bytes, const void *dev_blob,
+                         uint32_t *dev_status, int verify_payload, uw_dmat *out);
+
+/* Device error bits OR-ed into *dev_status by kernels. */
+#define UW_DEVERR_CORRUPT 1u
+#define UW_DEVERR_TIMEOUT 2u
+
+/* Synchronize `stream`, read and clear *w->dev_status.  Returns UW_OK,
+ * UW_ERR_CORRUPT or UW_ERR_TIMEOUT (CORRUPT wins if both are set).           */
+uw_status uw_device_status(const uw_dmat *w, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Preprocessing kernels (Unweight page §六, pipelines 1 and 3).              */
+
+/* Full Huffman decode to BF16: out_dev is uint16[n*k] (caller-owned, device,
+ * 16-byte aligned).  Needs UW_EMIT_HUFFMAN.  Bit-exact inverse of uw_encode. */
+uw_status uw_decode_to_bf16(const uw_dmat *w, uint16_t *out_dev, void *stream);
+
+/* Runtime transcode of the Huffman stream to the 4-bit palette plane:
+ * pal_dev is uint8[n*k/2] (device, 16-byte aligned), byte-identical to the
+ * blob's own UW_SEC_PAL section.  Needs UW_EMIT_HUFFMAN.                     */
+uw_status uw_transcode_palette(const uw_dmat *w, uint8_t *pal_dev, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Matmul (Unweight page §六-§七).                                            */
+
+typedef enum uw_pipeline {
+    UW_PIPE_DECODE_GEMM = 1,      /* decode to BF16 in the workspace, then the plain kernel */
+    UW_PIPE_TRANSCODE_FUSED = 3,  /* transcode to the palette plane in the workspace, then
+                                     the fused kernel                                    */
+    UW_PIPE_DIRECT_PALETTE = 4    /* fused kernel on the blob's (or a given) palette plane */
+} uw_pipeline;
+
+typedef enum uw_kernel {
+    UW_KERNEL_FMA = 1,   /* CUDA-core FMA GEMV, one warp per `bn` rows, m <= 8       */
+    UW_KERNEL_TC = 2     /* tcgen05 MMA with a TMEM accumulator, token tile `bn`      */
+} uw_kernel;
+
+#define UW_DEBUG_NEVER_ARRIVE 1u   /* TC kernel: wait on a barrier nobody signals, so
+                                      the bounded wait runs out (time-out test)      */
+
+typedef struct uw_plan {
+    int32_t pipeline;     /* uw_pipeline */
+    int32_t kernel;       /* uw_kernel */
+    int32_t bn;           /* TC: tokens per tile, one of 16,32,64,128,256;
+                             FMA: weight rows per warp, 1 or 2 */
+    int32_t split_k;      /* TC: K split into this many slices (>= 1), reduced in a
+                             fixed order; FMA: must be 1 */
+    int32_t stages;       /* TC: shared-memory ring depth (0 = largest that fits) */
+    uint32_t debug_flags; /* UW_DEBUG_* (0 in production) */
+    int64_t timeout_ns;   /* spin-wait limit inside kernels (0 = 2 s) */
+} uw_plan;
+
+/* A reasonable plan without measuring (FMA for m <= 4, TC otherwise). */
+uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pipeline, uw_plan *plan);
+
+/* Workspace bytes uw_fused_matmul needs for this plan (0 is possible). */
+uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw_plan *plan,
+                            size_t *bytes);
+
+/* Y = X * W^T with W compressed.  x_dev: uint16[m,k] BF16 (16-byte aligned
+ * rows); y_dev: float[m,n]; pal_dev: a palette plane to use instead of the
+ * blob's (pipeline 4 only; may be NULL).  ws/ws_bytes: caller workspace of at
+ * least uw_workspace_size bytes (256-byte aligned).  For every plan the
+ * result is bit-identical to uw_matmul_bf16 with the same kernel, bn and
+ * split_k on the decoded weights.                                            */
+uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_dmat *w,
+                          const uint8_t *pal_dev, float *y_dev, const uw_plan *plan,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/* The same kernels on plain BF16 weights w_dev[n,k] (the parity twin and the
+ * uncompressed baseline).  plan->pipeline is ignored.  dev_status: a device
+ * uint32 for kernel error bits (may be NULL when no error reporting is wanted). */
+uw_status uw_matmul_bf16(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev,
+                         int64_t n, int64_t k, float *y_dev, const uw_plan *plan,
+                         void *ws, size_t ws_bytes, uint32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Autotuner (Unweight page §九).                                             */
+
+/* For every matrix mats[i] and batch size ms[j], time the candidate
+ * (pipeline, kernel, bn, split_k) plans with CUDA events on `stream` and
+ * store the fastest in plans_out[i*n_ms + j].  x_dev must hold at least
+ * max(ms) x max(k) BF16 values, y_dev max(ms) x max(n) floats, and ws at least
+ * the largest uw_workspace_size of any candidate (uw_autotune_workspace_size).
+ * If json_out is non-NULL a JSON plan file (per matrix, per m: the chosen plan
+ * and the measured microseconds of every candidate) is written into it.     */
+uw_status uw_autotune_workspace_size(const uw_dmat *const *mats, int n_mats,
+                                     const int64_t *ms, int n_ms, size_t *bytes);
+uw_status uw_plan_autotune(const uw_dmat *const *mats, int n_mats, const int64_t *ms,
+                           int n_ms, const uint16_t *x_dev, float *y_dev, void *ws,
+                           size_t ws_bytes, int reps, uw_plan *plans_out, char *json_out,
+                           size_t json_cap, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* UW_H */

@@ -1,0 +1,223 @@
+"""GPU parity: libuw kernels (through the C ABI) against the CPU oracle.
+
+* decode: bit-exact against the original weights (which the oracle's own
+  decode reproduces, pinned in test_oracle_pins) and transcode bit-exact
+  against the oracle's 4-bit palette plane;
+* matmul: the fused kernel is bit-identical to the same kernel on plain BF16
+  weights, and every output lies within |y - y_oracle| <= 1e-4 * sum|x w|
+  of the float64 oracle;
+* corrupt device streams and exhausted spin-waits come back as status codes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from decode_gemm_exponent_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-4       # |y - y_oracle| <= TOL * sum_k |x_k w_k|
+
+
+@pytest.fixture(scope="module")
+def uw():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from decode_gemm_exponent_b200 import uw as U
+    return U
+
+
+def dev16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def host16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def check_bound(y_gpu: np.ndarray, y_ref: np.ndarray, a_ref: np.ndarray):
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bad = err > TOL * a_ref + 1e-30
+    assert not bad.any(), "max err/bound %.3g at %s" % (
+        float((err / np.maximum(TOL * a_ref, 1e-30)).max()), np.argwhere(bad)[:5].tolist())
+
+
+# ---------------------------------------------------------------- decode / transcode
+
+DECODE_CASES = {
+    "cfg_small_1024": lambda: synth.small_matrix(seed=0),
+    "all_patterns": lambda: np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(1024, 64),
+    "heavy_outliers_5pct": lambda: synth.weights_bf16(256, 1024, 0.015, 0.05, 1.0, seed=5),
+    "ragged_last_tile": lambda: synth.weights_bf16(192, 1344, 0.02, 0.002, 1.0, seed=6),
+    "one_exponent": lambda: ((np.uint16(121) << 7) |
+                             (np.random.default_rng(1).integers(0, 256, 64 * 128).astype(np.uint16)
+                              & 0x807F)).astype(np.uint16).reshape(64, 128),
+    "all_raw": lambda: np.tile(((np.tile(np.arange(60, 124, dtype=np.uint16), 8) << 7) |
+                                np.random.default_rng(2).integers(0, 128, 512).astype(np.uint16)
+                                ).reshape(4, 128), (16, 1)),
+    "sigma_0.005": lambda: synth.weights_bf16(128, 2048, 0.005, 0.0, 1.0, seed=7),
+    "sigma_0.05": lambda: synth.weights_bf16(128, 2048, 0.05, 0.001, 1.0, seed=8),
+}
+
+
+@pytest.mark.parametrize("case", list(DECODE_CASES))
+def test_decode_and_transcode_bit_exact(uw, case):
+    w = DECODE_CASES[case]()
+    m = uw.Matrix(uw.encode(w), verify_payload=True)
+    d = m.decode()
+    p = m.transcode()
+    assert m.device_status() == 0
+    assert np.array_equal(host16(d), w)
+    ref = O.encode(w)
+    assert np.array_equal(p.cpu().numpy(), ref.pal_plane)
+    assert np.array_equal(O.decode(ref), w)
+
+
+@pytest.mark.slow
+def test_decode_transcode_full_size_8b_gate(uw):
+    w = synth.weights_bf16(14336, 4096, 0.02, 0.0005, 1.0, seed=1)
+    m = uw.Matrix(uw.encode(w))
+    assert np.array_equal(host16(m.decode()), w)
+    ref = O.encode(w)
+    assert np.array_equal(m.transcode().cpu().numpy(), ref.pal_plane)
+    assert m.device_status() == 0
+
+
+def test_corrupt_device_stream_is_reported(uw):
+    w = synth.weights_bf16(128, 1024, 0.02, 0.001, 1.0, seed=9)
+    blob = uw.encode(w)
+    m = uw.Matrix(blob)
+    info = m.info
+    # flip bits in the middle of the stream on the device copy only
+    off = info.section_offset[uw.SEC_STREAM] + 64
+    m.dev[off:off + 8] ^= 0x5A
+    m.decode()
+    assert m.device_status() == 3          # UW_ERR_CORRUPT
+    # the context stays usable and a clean matrix still decodes
+    m2 = uw.Matrix(blob)
+    assert np.array_equal(host16(m2.decode()), w) and m2.device_status() == 0
+
+
+# ---------------------------------------------------------------- matmul
+
+def _matmul_case(uw, n, k, m, plan_kw, seed=0, frac=0.002, pipelines=(1, 3, 4)):
+    w = synth.weights_bf16(n, k, 0.02, frac, 1.0, seed=seed)
+    x = synth.activations_bf16(m, k, seed=seed)
+    mat = uw.Matrix(uw.encode(w))
+    xd, wd = dev16(x), dev16(w)
+    plan = uw.make_plan(**{**plan_kw, "pipeline": 4})
+    y_plain = uw.matmul_bf16(xd, wd, plan).cpu().numpy()
+    outs = {}
+    for pipe in pipelines:
+        p = uw.make_plan(**{**plan_kw, "pipeline": pipe})
+        outs[pipe] = mat.matmul(xd, p).cpu().numpy()
+    assert mat.device_status() == 0
+    for pipe, y in outs.items():
+        assert np.array_equal(y.view(np.uint32), y_plain.view(np.uint32)), "pipeline %d differs" % pipe
+    y_ref, a_ref = O.gemm(x, w)
+    check_bound(y_plain, y_ref, a_ref)
+    return y_plain
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("rows", [1, 2])
+def test_fma_gemv_parity(uw, m, rows):
+    _matmul_case(uw, 320, 1600, m, dict(kernel=uw.KERNEL_FMA, bn=rows, split_k=1), seed=m)
+
+
+@pytest.mark.parametrize("bn,m", [(16, 1), (16, 16), (32, 20), (64, 64), (64, 100), (128, 128),
+                                  (128, 300), (256, 256), (256, 513)])
+def test_tc_gemm_parity(uw, bn, m):
+    _matmul_case(uw, 384, 1024, m, dict(kernel=uw.KERNEL_TC, bn=bn, split_k=1), seed=bn + m)
+
+
+@pytest.mark.parametrize("split,stages", [(2, 0), (3, 2), (5, 3), (16, 0)])
+def test_tc_gemm_split_and_stages(uw, split, stages):
+    _matmul_case(uw, 256, 1024, 48, dict(kernel=uw.KERNEL_TC, bn=64, split_k=split, stages=stages),
+                 seed=split)
+
+
+def test_tc_gemm_ragged_n_and_raw_heavy(uw):
+    # n not a multiple of the 128-row tile, many raw groups
+    _matmul_case(uw, 320, 704, 40, dict(kernel=uw.KERNEL_TC, bn=64, split_k=2), seed=3, frac=0.05)
+
+
+def test_tc_stage_depth_does_not_change_bits(uw):
+    ys = [_matmul_case(uw, 256, 768, 32, dict(kernel=uw.KERNEL_TC, bn=32, split_k=1, stages=s),
+                       seed=11, pipelines=(4,)) for s in (2, 3, 4)]
+    assert all(np.array_equal(ys[0], y) for y in ys[1:])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("m,plan_kw", [(1, dict(kernel=1, bn=1, split_k=1)),
+                                       (16, dict(kernel=2, bn=16, split_k=4)),
+                                       (64, dict(kernel=2, bn=64, split_k=2)),
+                                       (1024, dict(kernel=2, bn=256, split_k=1))])
+def test_full_size_8b_sampled(uw, m, plan_kw):
+    """8B gate shape at the bench's launch configurations: fused == plain bit
+    for bit, and 512 sampled outputs within the bound of the oracle."""
+    n, k = 14336, 4096
+    w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1)
+    x = synth.activations_bf16(m, k, seed=1)
+    mat = uw.Matrix(uw.encode(w))
+    xd, wd = dev16(x), dev16(w)
+    plan = uw.make_plan(pipeline=4, **plan_kw)
+    yf = mat.matmul(xd, plan).cpu().numpy()
+    yp = uw.matmul_bf16(xd, wd, plan).cpu().numpy()
+    assert mat.device_status() == 0
+    assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32))
+    rng = np.random.default_rng(0)
+    ri = rng.integers(0, m, 512)
+    rj = rng.integers(0, n, 512)
+    ri[:2], rj[:2] = [0, m - 1], [0, n - 1]
+    y_ref, a_ref = O.gemm_sampled(x, w, ri, rj)
+    check_bound(yf[ri, rj], y_ref, a_ref)
+
+
+# ---------------------------------------------------------------- failure paths
+
+def test_bounded_wait_times_out_and_context_survives(uw):
+    w = synth.weights_bf16(256, 512, 0.02, 0.001, 1.0, seed=12)
+    x = synth.activations_bf16(16, 512, seed=12)
+    mat = uw.Matrix(uw.encode(w))
+    xd = dev16(x)
+    p = uw.make_plan(pipeline=4, kernel=uw.KERNEL_TC, bn=16, split_k=1,
+                     debug_flags=uw.DEBUG_NEVER_ARRIVE, timeout_ns=2_000_000)
+    mat.matmul(xd, p)
+    assert mat.device_status() == 6        # UW_ERR_TIMEOUT
+    ok = uw.make_plan(pipeline=4, kernel=uw.KERNEL_TC, bn=16, split_k=1)
+    y = mat.matmul(xd, ok).cpu().numpy()
+    assert mat.device_status() == 0
+    y_ref, a_ref = O.gemm(x, w)
+    check_bound(y, y_ref, a_ref)
+
+
+def test_workspace_errors(uw):
+    w = synth.weights_bf16(128, 512, 0.02, 0.0, 1.0, seed=13)
+    mat = uw.Matrix(uw.encode(w))
+    xd = dev16(synth.activations_bf16(4, 512, seed=13))
+    p = uw.make_plan(pipeline=1, kernel=uw.KERNEL_FMA, bn=1)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(uw.UwError) as e:
+        mat.matmul(xd, p, ws=small)
+    assert e.value.status == 7
+
+
+def test_autotune_returns_valid_plans(uw):
+    mats = [uw.Matrix(uw.encode(synth.weights_bf16(512, 1024, 0.02, 0.001, 1.0, seed=s)))
+            for s in (20, 21)]
+    plans, js = uw.autotune(mats, [1, 64], reps=2)
+    import json
+    doc = json.loads(js)
+    assert len(doc["plans"]) == 4
+    for row in plans:
+        for p in row:
+            assert p.kernel in (1, 2) and p.pipeline in (1, 3, 4)
+    # the chosen plan reproduces the plain kernel bit for bit
+    w = synth.weights_bf16(512, 1024, 0.02, 0.001, 1.0, seed=20)
+    x = synth.activations_bf16(64, 1024, seed=20)
+    p = plans[0][1]
+    yf = mats[0].matmul(dev16(x), p).cpu().numpy()
+    yp = uw.matmul_bf16(dev16(x), dev16(w), p).cpu().numpy()
+    assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32))

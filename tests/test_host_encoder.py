@@ -1,0 +1,217 @@
+"""Host side of libuw on CPU: exports, encoder vs oracle, blob checks, plans.
+
+No GPU is needed: these tests load libuw.so, call only host entry points (and
+device entry points with invalid arguments, which must fail before touching
+the GPU) and compare the production encoder with the CPU oracle section by
+section.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from decode_gemm_exponent_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def uw():
+    from decode_gemm_exponent_b200 import build
+    build.build()
+    from decode_gemm_exponent_b200 import uw as U
+    return U
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "uw.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(uw_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(uw):
+    declared = _declared_functions()
+    assert len(declared) >= 16
+    lib = ctypes.CDLL(uw.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(uw.EXPORTS) == declared
+    assert "sm_100a" in uw.version()
+
+
+# ------------------------------------------------------------------ encoder parity
+
+def _cases():
+    rng = np.random.default_rng(0)
+    e = np.tile(np.arange(60, 124, dtype=np.uint16), 8)
+    all_raw = ((e << 7) | rng.integers(0, 128, e.size).astype(np.uint16)).reshape(4, 128)
+    one_exp = ((np.uint16(121) << 7) | (rng.integers(0, 256, 64 * 128).astype(np.uint16) & 0x807F))
+    return {
+        "small_cfg": synth.weights_bf16(128, 1024, 0.02, 0.001, 2.0, seed=0),
+        "ragged_chunk": synth.weights_bf16(64, 192, 0.02, 0.01, 1.0, seed=2),
+        "all_patterns": np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(1024, 64),
+        "all_raw": np.tile(all_raw, (16, 1)),
+        "one_exponent": one_exp.astype(np.uint16).reshape(64, 128),
+        "heavy_outliers": synth.weights_bf16(64, 512, 0.015, 0.05, 1.0, seed=5),
+        "wide_sigma": synth.weights_bf16(64, 256, 0.05, 0.0, 1.0, seed=6),
+    }
+
+
+def _bits(words: np.ndarray, count: int) -> np.ndarray:
+    """u32 word array -> 0/1 flags (LSB of word 0 first)."""
+    return ((words[:, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.uint8).ravel()[:count]
+
+
+@pytest.mark.parametrize("case", list(_cases().keys()))
+def test_encoder_matches_oracle(uw, case):
+    w = _cases()[case]
+    if w.shape[0] % 64:
+        pytest.skip("rows must be a multiple of 64")
+    blob = uw.encode(w)
+    info = uw.blob_info(blob, verify_payload=True)
+    ref = O.encode(w)
+    n, k = w.shape
+    assert (info.n, info.k) == (n, k)
+    assert list(info.palette)[:info.palette_size] == list(ref.palette)
+    assert list(info.code_len) == list(ref.code_len)
+    assert info.n_raw == ref.n_raw and info.stream_bits == ref.stream_bits
+    assert np.array_equal(uw.section(blob, uw.SEC_SM, info), ref.sm)
+    assert np.array_equal(uw.section(blob, uw.SEC_RAWEXP, info), ref.rawexp)
+    flags = uw.section(blob, uw.SEC_FLAGS, info).view("<u4")
+    assert np.array_equal(_bits(flags, n * k // 64), ref.raw)
+    base = uw.section(blob, uw.SEC_RAWBASE, info).view("<u4")
+    nw = (n * k // 64 + 31) // 32
+    pc = np.array([bin(int(x)).count("1") for x in flags[:nw]], np.int64)
+    assert np.array_equal(base[:nw].astype(np.int64), np.concatenate([[0], np.cumsum(pc)[:-1]]))
+    stream = uw.section(blob, uw.SEC_STREAM, info).view("<u4")
+    nwords = len(ref.stream)
+    assert np.array_equal(stream[:nwords], ref.stream) and not stream[nwords:].any()
+    off = uw.section(blob, uw.SEC_CHUNKOFF, info).view("<u4")
+    assert np.array_equal(off[:len(ref.chunk_off)], ref.chunk_off)
+    assert np.array_equal(uw.section(blob, uw.SEC_PAL, info), ref.pal_plane)
+    # statistics reported in the header
+    h = O.histogram(w)
+    assert info.entropy_bits == pytest.approx(O.entropy_bits(h), abs=1e-9)
+    assert info.top16_coverage == pytest.approx(float(h[ref.palette].sum()) / w.size, abs=1e-12)
+
+
+def test_encoder_is_deterministic_and_sizes(uw):
+    w = synth.weights_bf16(256, 1024, 0.02, 0.0005, 1.0, seed=3)
+    a, b = uw.encode(w), uw.encode(w)
+    assert a == b
+    info = uw.blob_info(a)
+    # Huffman form is smaller than BF16, the palette form in between
+    assert info.huffman_bytes < info.palette_bytes < w.nbytes
+    only_h = uw.blob_info(uw.encode(w, uw.EMIT_HUFFMAN))
+    only_p = uw.blob_info(uw.encode(w, uw.EMIT_PALETTE))
+    assert only_h.section_bytes[uw.SEC_PAL] == 0 and only_p.section_bytes[uw.SEC_STREAM] == 0
+    for s in range(uw.NUM_SECTIONS):
+        assert info.section_offset[s] % 256 == 0
+
+
+def test_decode_table_reproduces_oracle_symbols(uw):
+    """Decode the production stream on the CPU with the production 12-bit
+    multi-symbol table and compare the symbols with the oracle's palette
+    indices (catches table bugs before any kernel runs)."""
+    w = synth.weights_bf16(64, 512, 0.02, 0.002, 1.0, seed=8)
+    blob = uw.encode(w)
+    info = uw.blob_info(blob)
+    lut = uw.section(blob, uw.SEC_DLUT, info).view("<u4")
+    stream = uw.section(blob, uw.SEC_STREAM, info).view("<u4")
+    ref = O.encode(w)
+    want = []
+    e = ((w.ravel() >> 7) & 0xFF)
+    raw_el = np.repeat(ref.raw.astype(bool), 64)
+    want = np.searchsorted(ref.palette, e[~raw_el])
+    got = []
+    p = 0
+    total = len(want)
+    while len(got) < total:
+        wi = p >> 5
+        win = ((int(stream[wi]) << 32 | int(stream[wi + 1])) >> (64 - 12 - (p & 31))) & 0xFFF
+        ent = int(lut[win])
+        cnt, nb, l0 = (ent >> 20) & 7, (ent >> 23) & 15, ent >> 27
+        assert cnt > 0
+        if cnt <= total - len(got):
+            got += [(ent >> (4 * j)) & 15 for j in range(cnt)]
+            p += nb
+        else:
+            got.append(ent & 15)
+            p += l0
+    assert p == info.stream_bits
+    assert np.array_equal(np.array(got), want)
+
+
+# ------------------------------------------------------------------ fault injection (host)
+
+def test_blob_corruption_is_rejected(uw):
+    w = synth.weights_bf16(64, 256, 0.02, 0.001, 1.0, seed=4)
+    blob = bytearray(uw.encode(w))
+    uw.blob_info(bytes(blob), verify_payload=True)
+
+    def status(b, verify=True):
+        try:
+            uw.blob_info(bytes(b), verify_payload=verify)
+            return 0
+        except uw.UwError as e:
+            return e.status
+
+    CORRUPT = 3
+    assert status(blob[:-256]) == CORRUPT                       # truncated
+    assert status(blob[:100]) == CORRUPT                        # shorter than a header
+    bad = bytearray(blob); bad[0] ^= 0xFF
+    assert status(bad) == CORRUPT                               # magic
+    bad = bytearray(blob); bad[4] = 7
+    assert status(bad) == CORRUPT                               # version (and header CRC)
+    bad = bytearray(blob); bad[40] ^= 1
+    assert status(bad) == CORRUPT                               # any header byte (CRC)
+    bad = bytearray(blob); bad[len(bad) - 300] ^= 0x10
+    assert status(bad, verify=True) == CORRUPT                  # payload CRC
+    assert status(bad, verify=False) == 0                       # header-only check passes
+
+
+def test_invalid_arguments(uw):
+    lib = uw.lib()
+    out = ctypes.c_void_p()
+    w = np.zeros((64, 64), np.uint16)
+    assert lib.uw_encode(None, 64, 64, 0, ctypes.byref(out)) == 1
+    assert lib.uw_encode(w.ctypes.data, 0, 64, 0, ctypes.byref(out)) == 1
+    w2 = np.zeros((64, 96), np.uint16)
+    assert lib.uw_encode(w2.ctypes.data, 64, 96, 0, ctypes.byref(out)) == 2
+    w3 = np.zeros((63, 64), np.uint16)
+    assert lib.uw_encode(w3.ctypes.data, 63, 64, 0, ctypes.byref(out)) == 2
+    assert lib.uw_encode(w.ctypes.data, 64, 64, 8, ctypes.byref(out)) == 1
+    # device entry points reject bad arguments before any CUDA call
+    dm = uw.DMat()
+    assert lib.uw_decode_to_bf16(None, None, None) == 1
+    assert lib.uw_decode_to_bf16(ctypes.byref(dm), None, None) == 1
+    p = uw.make_plan()
+    assert lib.uw_fused_matmul(None, 1, ctypes.byref(dm), None, None, ctypes.byref(p), None, 0, None) == 1
+    assert lib.uw_matmul_bf16(None, 1, None, 64, 64, None, ctypes.byref(p), None, 0, None, None) == 1
+    # a misaligned device blob is refused by bind
+    blob = np.frombuffer(uw.encode(w), np.uint8)
+    assert lib.uw_matrix_bind(blob.ctypes.data, blob.size, ctypes.c_void_p(0x1001), None, 0,
+                              ctypes.byref(dm)) == 1
+
+
+def test_plans_and_workspace(uw):
+    p = uw.plan_default(1, 14336, 4096)
+    assert p.kernel == uw.KERNEL_FMA and p.split_k == 1
+    p = uw.plan_default(1024, 14336, 4096)
+    assert p.kernel == uw.KERNEL_TC and p.bn == 256
+    p = uw.plan_default(64, 4096, 14336)
+    assert p.kernel == uw.KERNEL_TC and p.bn == 64 and p.split_k >= 1
+    n, k = 4096, 1024
+    assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_FMA, 1)) == 0
+    assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_DECODE_GEMM, uw.KERNEL_FMA, 1)) == n * k * 2
+    assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_TRANSCODE_FUSED, uw.KERNEL_FMA, 1)) == n * k // 2
+    assert uw.workspace_size(16, n, k, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 16, 4)) == 4 * 16 * n * 4
+    for bad in (uw.make_plan(kernel=9), uw.make_plan(bn=48), uw.make_plan(pipeline=2),
+                uw.make_plan(kernel=uw.KERNEL_FMA, bn=1, split_k=2), uw.make_plan(split_k=0)):
+        with pytest.raises(uw.UwError):
+            uw.workspace_size(4, n, k, bad)
+    with pytest.raises(uw.UwError):
+        uw.workspace_size(16, n, k, uw.make_plan(kernel=uw.KERNEL_FMA, bn=1))   # FMA needs m <= 8
