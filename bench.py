@@ -45,6 +45,27 @@ WORKLOAD = "llama-3.1-8b MLP layer (gate/up/down), M in {1,4,16,64}, autotuned p
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def rank_seed(proj_index: int, rank: int) -> int:
+    """Seed of projection `proj_index` on `rank`: every rank owns an independent layer."""
+    return 1 + proj_index + 100 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest `value` over all ranks (a no-op for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(bytes_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job GB/s: the bytes every rank processed over the slowest rank's time."""
+    return bytes_per_rank * world / (ms * 1e-3) / 1e9
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -60,54 +81,70 @@ def load_peaks():
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, power and clock-event reasons through NVML (read-only)
+    from a background thread every ~1 ms while the timed region runs, and
+    keeps a CSV of the samples under gpurun_out/."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, gpu_index: int):
-        self.proc = None
         self.gpu = gpu_index
+        self.samples = []
+        self.error = None
         self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
 
+    def _run(self):
+        import pynvml as N
+        h = N.nvmlDeviceGetHandleByIndex(self.gpu)
+        self.sm_max = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+        masks = [(name, getattr(N, attr)) for name, attr in self.REASONS]
+        while not self.stop.is_set():
+            sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+            reasons = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+            power = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+            self.samples.append((time.time(), sm, power, [n for n, m in masks if reasons & m]))
+            self.stop.wait(0.001)
+
     def __enter__(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as N
+            N.nvmlInit()
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 2.0:
+                time.sleep(0.001)
+        except Exception as e:   # NVML missing: report it, keep benchmarking
+            self.error = repr(e)
+            self.thread = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
+                os.makedirs(os.path.dirname(self.path), exist_ok=True)
+                with open(self.path, "w") as f:
+                    f.write("time,sm_mhz,power_w,reasons\n")
+                    for t, sm, pw, rs in self.samples:
+                        f.write("%.4f,%d,%.1f,%s\n" % (t, sm, pw, "|".join(rs)))
+            except OSError:
+                pass
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
+                    "reasons": ["nvml unavailable: %s" % self.error]}
+        reasons = sorted({r for _, _, _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(s[1] for s in self.samples), "sm_max_mhz": self.sm_max,
+                "samples": len(self.samples), "power_w_max": max(s[2] for s in self.samples),
+                "reasons": reasons, "source": "nvml, 1 ms polling during the timed region"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
@@ -184,6 +221,18 @@ def alg_bytes(mat, m, plan):
     return {"transcode": huff_in + n * k // 2, "fused": common + n * k // 2 + xy}
 
 
+def plans_from_json(text, n_mats, uw):
+    """Plans from a plan file written by the autotuner (--plan-json)."""
+    doc = json.loads(text)
+    pipes = {"decode_gemm": 1, "transcode_fused": 3, "direct_palette": 4}
+    plans = [[None] * len(MS) for _ in range(n_mats)]
+    for e in doc["plans"]:
+        b = e["best"]
+        plans[e["matrix"]][MS.index(e["m"])] = uw.make_plan(
+            pipes[b["pipeline"]], 1 if b["kernel"] == "fma" else 2, b["bn"], b["split_k"])
+    return plans
+
+
 def launches_per_call(plan):
     n = 1 + (1 if plan.pipeline in (1, 3) else 0)
     if plan.kernel == 2 and plan.split_k > 1:
@@ -210,12 +259,17 @@ def run_gpu(args, rank, world):
     # ---- inputs (host encode is the offline step, outside any timing)
     mats = []
     for i, (name, n, k) in enumerate(PROJ):
-        w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1 + i + 100 * rank)
+        w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=rank_seed(i, rank))
         mats.append(uw.Matrix(uw.encode(w), device=dev))
     xs = {m: {k: torch.from_numpy(synth.activations_bf16(m, k, seed=m).view(np.int16)).to(dev)
               for k in {p[2] for p in PROJ}} for m in MS}
 
-    plans, plan_json = uw.autotune(mats, list(MS), reps=10)
+    if args.plans_in:
+        with open(args.plans_in) as f:
+            plan_json = f.read()
+        plans = plans_from_json(plan_json, len(mats), uw)
+    else:
+        plans, plan_json = uw.autotune(mats, list(MS), reps=10)
     calls = []
     for j, m in enumerate(MS):
         for i, mat in enumerate(mats):
@@ -257,13 +311,9 @@ def run_gpu(args, rank, world):
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
-    step_ms = t_start.elapsed_time(t_end) / args.steps
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
     weight_bytes = sum(2 * c["mat"].n * c["mat"].k for c in calls)
-    value = weight_bytes * world / (step_ms * 1e-3) / 1e9
+    value = aggregate_gbs(weight_bytes, world, step_ms)
 
     # per-call durations -> kernel groups
     per_call = [statistics.median(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps))
@@ -296,11 +346,7 @@ def run_gpu(args, rank, world):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     for mat in mats:
         st = mat.device_status()
         if st != 0:
@@ -334,7 +380,7 @@ def run_gpu(args, rank, world):
                      "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                      "peak_source": peaks["_source"] + " hbm_gbs"},
         "cpu_baseline": cpu,
-        "e2e": {"value": weight_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": aggregate_gbs(weight_bytes, world, e2e_ms), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": sum(launches_per_call(c["plan"]) for c in calls) * args.steps,
         "clocks": clocks,
@@ -354,6 +400,7 @@ def main():
     ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--plan-json", default=None, help="write the autotuner's plan file here")
+    ap.add_argument("--plans-in", default=None, help="use this plan file instead of autotuning")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

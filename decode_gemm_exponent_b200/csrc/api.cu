@@ -53,7 +53,7 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
                      const uint8_t *pal, int64_t n, int64_t k, float *y, const uw_plan *plan,
                      float *partial, uint32_t *status, cudaStream_t stream) {
     if (plan->kernel == UW_KERNEL_FMA)
-        return cuda_status(launch_gemv_fma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, stream));
+        return cuda_status(launch_gemv_fma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, status, stream));
     TcLaunch t{};
     t.x = x;
     t.m = m;

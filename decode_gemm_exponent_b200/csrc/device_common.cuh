@@ -61,25 +61,28 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
         : "memory");
 }
 
+// Non-blocking test of phase completion (the waiter spins; no suspension).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
         : "=r"(ok)
         : "r"(smem_addr(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
 
-// Wait until the phase with the given parity has completed, or until
-// `timeout_ns` of wall time has passed.  Returns false on time-out.
+// Wait until the phase with the given parity has completed, or give up after
+// about `timeout_ns`.  The bound is counted in SM cycles (clock64 is cheap to
+// read; 2 cycles per ns keeps the bound at least timeout_ns for clocks up to
+// 2 GHz).  Returns false on time-out.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > timeout_ns) return false;
-    }
+    const long long limit = (long long)(timeout_ns * 2);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > limit) return false;
+    return true;
 }
 
 // ---------------------------------------------------------------- TMA
@@ -108,6 +111,26 @@ __device__ __forceinline__ void tma_load_2d(void *dst_smem, const CUtensorMap *m
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+
+// 16-byte asynchronous global -> shared copy (not TMA), L1 bypassed
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src)
+                 : "memory");
+}
+
+// Make `bar`'s current phase also wait for this thread's earlier cp.async
+// copies (the pending count is raised now and lowered when they land).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Same, but the arrival is counted in the barrier's expected count instead
+// of raising the pending count (the barrier must be initialised with it).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // generic-proxy shared-memory writes -> visible to the async proxy (MMA, TMA)
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -191,59 +214,92 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
 }
 
 // ---------------------------------------------------------------- rebuild
+//
+// A BF16 pattern s<<15 | e<<7 | m has high byte s<<7 | e>>1 and low byte
+// (e&1)<<7 | m.  With the palette stored as r = rotr8(e) = (e>>1) | (e&1)<<7
+// both bytes come from one looked-up byte r and the sign/mantissa byte
+// sm = s<<7 | m:  high = (r & 0x7F) | (sm & 0x80),  low = (r & 0x80) | (sm & 0x7F).
 
 struct Palette16 {
-    uint32_t p0, p1, p2, p3;   // palette[0..3], [4..7], [8..11], [12..15] as bytes
+    uint32_t p0, p1, p2, p3;   // rotr8(palette[0..15]) as bytes, 4 per word
 };
 
-// One 4-bit-palette word (8 weights) -> their exponent bytes: e0 = weights
-// 0..3, e1 = weights 4..7 (one byte each, weight 0 lowest).  The low three
-// index bits are prmt selectors into the 8-byte half-palettes; bit 3 of each
-// index sits in a byte's top bit (of the word, or of the word shifted by 4),
-// so a sign-replicating prmt turns it into a whole-byte mask.
-__device__ __forceinline__ void pal_exponents(uint32_t x, const Palette16 &P, uint32_t &e0,
-                                              uint32_t &e1) {
-    const uint32_t s0 = x & 0x7777u;
-    const uint32_t s1 = (x >> 16) & 0x7777u;
-    const uint32_t m0 = prmt(x, 0u, 0xBA98u);
-    const uint32_t m1 = prmt(x << 4, 0u, 0xBA98u);
-    const uint32_t lo0 = prmt(P.p0, P.p1, s0), hi0 = prmt(P.p2, P.p3, s0);
-    const uint32_t lo1 = prmt(P.p0, P.p1, s1), hi1 = prmt(P.p2, P.p3, s1);
-    e0 = (hi0 & m0) | (lo0 & ~m0);
-    e1 = (hi1 & m1) | (lo1 & ~m1);
+__host__ __device__ inline uint8_t rotr8(uint8_t e) { return uint8_t((e >> 1) | ((e & 1u) << 7)); }
+
+__host__ inline Palette16 make_palette16(const uint8_t palette[16]) {
+    auto word = [&](int i) {
+        return uint32_t(rotr8(palette[i])) | uint32_t(rotr8(palette[i + 1])) << 8 |
+               uint32_t(rotr8(palette[i + 2])) << 16 | uint32_t(rotr8(palette[i + 3])) << 24;
+    };
+    return Palette16{word(0), word(4), word(8), word(12)};
 }
 
-// t = [e1 sm1 e0 sm0] (bytes, low first) -> two BF16 patterns
-// s<<15 | e<<7 | m in the low and high halves.
-__device__ __forceinline__ uint32_t join2(uint32_t t) {
-    const uint32_t a = t >> 1;
-    const uint32_t c = t << 8;
-    const uint32_t sel = (t & 0x007F007Fu) | (c & ~0x007F007Fu);
-    return (a & 0x7F807F80u) | (sel & ~0x7F807F80u);
+// rotr8 of four raw exponent bytes
+__device__ __forceinline__ uint32_t rot4(uint32_t e) {
+    return ((e >> 1) & 0x7F7F7F7Fu) | ((e << 7) & 0x80808080u);
 }
 
-// 4 exponents (e) + 4 sign/mantissa bytes (s) -> 4 BF16 in two words
-__device__ __forceinline__ void join4(uint32_t e, uint32_t s, uint32_t &w01, uint32_t &w23) {
-    w01 = join2(prmt(s, e, 0x5140u));
-    w23 = join2(prmt(s, e, 0x7362u));
+// 16-entry byte lookup for four indices: low three bits as prmt selectors
+// (bit 3 cleared) into each 8-byte half-palette, then a byte mask picks the
+// upper half where the index has bit 3 set.
+__device__ __forceinline__ uint32_t lookup4(uint32_t sel, uint32_t mask, const Palette16 &P) {
+    const uint32_t lo = prmt(P.p0, P.p1, sel), hi = prmt(P.p2, P.p3, sel);
+    return (hi & mask) | (lo & ~mask);
 }
 
-// 8 weights: exponents (e0,e1) + sm bytes (s0,s1) -> uint4 of 8 BF16
-__device__ __forceinline__ uint4 join8(uint32_t e0, uint32_t e1, uint32_t s0, uint32_t s1) {
-    uint4 r;
-    join4(e0, s0, r.x, r.y);
-    join4(e1, s1, r.z, r.w);
-    return r;
+// One stored 4-bit-palette word (8 weights) -> rotated exponent bytes:
+// r0 = weights 0..3, r1 = weights 4..7.  In the stored layout bit 3 of index
+// j sits in the top bit of byte j (j < 4) or of byte j-4 of the word shifted
+// left by 4 (j >= 4), so a sign-replicating prmt yields the byte masks.
+__device__ __forceinline__ void pal_rot(uint32_t x, const Palette16 &P, uint32_t &r0, uint32_t &r1) {
+    r0 = lookup4(x & 0x7777u, prmt(x, 0u, 0xBA98u), P);
+    r1 = lookup4((x >> 16) & 0x7777u, prmt(x << 4, 0u, 0xBA98u), P);
 }
 
-// 8 palette indices in natural order (index j in bits 4j..4j+3) -> the
-// stored 4-bit-palette word layout (index bit 3 moved to a byte top bit).
+// Same for 8 indices in natural nibble order (index j in bits 4j..4j+3).
+__device__ __forceinline__ void nat_rot(uint32_t x, const Palette16 &P, uint32_t &r0, uint32_t &r1) {
+    const uint32_t m_odd = prmt(x, 0u, 0xBA98u);         // bit 3 of indices 1,3,5,7
+    const uint32_t m_even = prmt(x << 4, 0u, 0xBA98u);   // bit 3 of indices 0,2,4,6
+    r0 = lookup4(x & 0x7777u, prmt(m_even, m_odd, 0x5140u), P);
+    r1 = lookup4((x >> 16) & 0x7777u, prmt(m_even, m_odd, 0x7362u), P);
+}
+
+// 4 rotated exponents + 4 sign/mantissa bytes -> 4 BF16 (w01 = weights 0,1)
+__device__ __forceinline__ void join4(uint32_t r, uint32_t s, uint32_t &w01, uint32_t &w23) {
+    const uint32_t hi = (r & 0x7F7F7F7Fu) | (s & 0x80808080u);
+    const uint32_t lo = (r & 0x80808080u) | (s & 0x7F7F7F7Fu);
+    w01 = prmt(lo, hi, 0x5140u);
+    w23 = prmt(lo, hi, 0x7362u);
+}
+
+// 8 weights -> uint4 of 8 BF16
+__device__ __forceinline__ uint4 join8(uint32_t r0, uint32_t r1, uint32_t s0, uint32_t s1) {
+    uint4 o;
+    join4(r0, s0, o.x, o.y);
+    join4(r1, s1, o.z, o.w);
+    return o;
+}
+
+// 8 palette indices in natural order -> the stored 4-bit-palette word layout.
 __device__ __forceinline__ uint32_t natural_to_pal(uint32_t x) {
     const uint32_t low3 = x & 0x77777777u;
-    const uint32_t b = (x >> 3) & 0x11111111u;                          // bit 3 of j at bit 4j
-    const uint32_t vlo = (((b & 0x1111u) * 0x1248u) >> 12) & 0xFu;      // j = 0..3 -> bits 0..3
+    const uint32_t b = (x >> 3) & 0x11111111u;                              // bit 3 of j at bit 4j
+    const uint32_t vlo = (((b & 0x1111u) * 0x1248u) >> 12) & 0xFu;          // j = 0..3 -> bits 0..3
     const uint32_t vhi = ((((b >> 16) & 0x1111u) * 0x1248u) >> 12) & 0xFu;  // j = 4..7
     return low3 | ((vlo * 0x10204080u) & 0x80808080u) | ((vhi * 0x01020408u) & 0x08080808u);
+}
+
+// acc += a * b over the two BF16 halves of each operand (exact products,
+// one rounding per FMA: identical to fmaf on the widened values)
+__device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float acc) {
+    asm("{ .reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0; }"
+        : "+f"(acc)
+        : "r"(a), "r"(b));
+    return acc;
 }
 
 }  // namespace dev

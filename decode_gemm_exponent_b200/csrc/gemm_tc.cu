@@ -1,29 +1,44 @@
 // gemm_tc.cu -- tensor-core GEMM Y = X * W^T on sm_100a with tcgen05 MMA and a
-// TMEM accumulator, in two flavours sharing one template:
+// TMEM accumulator, in two flavours that issue the identical MMA sequence (so
+// their outputs are bit-identical):
 //   * fused: W arrives compressed (4-bit palette plane + sign/mantissa plane +
 //     raw groups) and is rebuilt to BF16 in shared memory (Unweight page §七,
 //     the reconstructive matmul; §五, decompress on chip, never back to HBM);
 //   * plain: W arrives as BF16 through TMA (the uncompressed baseline and the
 //     bit-exactness twin of the fused flavour).
-// Both issue the identical MMA sequence, so their outputs are bit-identical.
 //
-// CTA tile: 128 rows of W (the MMA "M") x `BN` tokens (the MMA "N"), K in
-// steps of 64 (one group).  Grid = (n/128, ceil(m/BN), split_k).  Warps:
-//   warp 0     producer: per K-step TMA of the X tile and either the BF16 W
-//              tile or the compressed tiles (sm plane 64 B/row with the
-//              64-byte swizzle, palette plane 32 B/row with the 32-byte
-//              swizzle); raw rows are fetched by 64-byte bulk copies; the
-//              stage's raw-row bitmap is written to shared memory.
-//   warp 1     MMA issuer (one thread): 4 x tcgen05.mma (K = 16 each) per
-//              K-step into the TMEM accumulator; tcgen05.commit frees the
-//              stage; a final commit signals the epilogue.  Also owns TMEM.
-//   warps 2-5  fused: each thread rebuilds one W row per K-step into the
-//              128-byte-swizzled K-major tile, then fences the async proxy
-//              and arrives.  Then all four read the accumulator back
-//              (tcgen05.ld, one TMEM lane quarter each) and store Y (fp32).
-// Every wait is bounded (globaltimer); on time-out the kernel raises
-// UW_DEVERR_TIMEOUT, stops issuing work, lets copies and MMAs in flight
-// finish, frees TMEM and returns.
+// CTA tile: 128 rows of W (the MMA "M") x `BN` tokens (the MMA "N"); K in
+// steps of 64 (one group).  Grid = (n/128, ceil(m/BN), split_k); split-K
+// slices are summed afterwards in a fixed order.
+//
+// Plain kernel (6 warps): warp 0 TMA producer (X tile + W tile per K-step,
+// 128-byte swizzle) into an S-stage ring; warp 1 allocates TMEM and issues 4
+// x tcgen05.mma (K = 16) per K-step, tcgen05.commit freeing the stage; warps
+// 2-5 read the accumulator (tcgen05.ld) and store Y.
+//
+// Fused kernel (15 warps), three rings so that no load waits for the MMA and
+// no MMA operand waits for a load issued late:
+//   compressed ring (CS stages): sign/mantissa tile (64-byte swizzle),
+//     palette tile (32-byte swizzle) and the exponents of the tile's raw rows
+//     (one 64-byte slot per row); freed as soon as the rebuild has read it;
+//   W ring (4 stages for BN <= 64, else 2): rebuilt BF16 W tiles (128-byte
+//     swizzle, K-major); freed by the MMA's commit;
+//   X ring (8 / 4 / 2 stages): X tiles, freed by the MMA's commit.
+//   warp 0     compressed tiles: two TMA loads per K-step.
+//   warp 1     MMA issuer and TMEM owner.
+//   warp 2     X producer (TMA).
+//   warps 3-6  raw producers: lane l of warp j owns row 32j + l and copies the
+//              row's raw exponents for each raw K-step with 16-byte cp.async,
+//              arriving on the stage barrier when they land.
+//   warps 7-14 two rebuild groups of 4 warps; group j rebuilds the K-steps
+//              ks = j (mod 2), each thread one row (64 weights).  The ring
+//              depths are even, so a group only ever touches its own stages
+//              and meets their barrier phases strictly in order (a parity wait
+//              issued a phase early would pass on the previous phase).  Then
+//              all eight read the accumulator back and store Y.
+// The raw-group bitmap of the tile's rows is staged in shared memory at start.
+// Every wait is bounded; on time-out the kernel raises UW_DEVERR_TIMEOUT,
+// stops issuing, waits (bounded) for its copies and MMAs, frees TMEM, returns.
 #include <algorithm>
 #include <cstring>
 
@@ -36,23 +51,12 @@ namespace {
 
 using namespace dev;
 
-constexpr int kThreads = 192;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kMaxSmem = 232448;   // 227 KB opt-in per CTA
-
-template <int BN, bool PAL>
-struct Cfg {
-    static constexpr int kW = kBM * kBK * 2;             // rebuilt / loaded W tile
-    static constexpr int kX = BN * kBK * 2;              // X tile
-    static constexpr int kSM = PAL ? kBM * kBK : 0;      // sign/mantissa tile
-    static constexpr int kPL = PAL ? kBM * kBK / 2 : 0;  // palette-index tile
-    static constexpr int kRAW = PAL ? kBM * kBK : 0;     // raw exponents, one slot per row
-    static constexpr int kStage = kW + kX + kSM + kPL + kRAW;
-    static constexpr int kOffX = kW, kOffSM = kW + kX, kOffPL = kOffSM + kSM, kOffRAW = kOffPL + kPL;
-    static constexpr uint32_t kTmemCols = BN < 32 ? 32u : uint32_t(BN);
-    static_assert(kStage % 1024 == 0, "stage tiles must keep 1024-byte alignment");
-};
+constexpr int kMaxSmem = 232448;          // 227 KB opt-in per CTA
+constexpr int kPlainThreads = 192;
+constexpr int kFusedThreads = (3 + 4) * 32 + 2 * 128;   // producers, MMA, raw producers, 2 rebuild groups
+constexpr int kGroups = 2;                // rebuild groups (K-steps alternate between them)
 
 struct TcArgs {
     int64_t m, n, k;
@@ -68,42 +72,82 @@ struct TcArgs {
     uint32_t *status;
 };
 
-__host__ __device__ constexpr int tail_bytes(int stages) {
-    // barriers (3 per stage + 2), raw bitmaps (4 words per stage), TMEM slot, abort flag
-    return (3 * stages + 2) * 8 + stages * 16 + 16;
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int BN, bool PAL>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
-              const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
-    using C = Cfg<BN, PAL>;
+// 4 x tcgen05.mma (K = 16 each) for one 64-wide K-step; A = W tile, B = X tile
+template <int BN>
+__device__ __forceinline__ void mma_kstep(uint32_t tmem, uint32_t sa, uint32_t sb, bool first) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+#pragma unroll
+    for (int kk = 0; kk < kBK / 16; kk++)
+        tc_mma_bf16(tmem, smem_desc_k128(sa + 32 * kk), smem_desc_k128(sb + 32 * kk), idesc,
+                    (!first || kk) ? 1u : 0u);
+}
+
+// Accumulator -> Y (or this split's slice of the partial sums).  Warp with
+// TMEM lane quarter q reads rows q*32..q*32+31; `slot` of `nslots` warps per
+// quarter take interleaved 16-column chunks.
+template <int BN>
+__device__ __forceinline__ void store_accumulator(uint32_t tmem, int q, int slot, int nslots, int lane,
+                                                  int64_t n0, int64_t m0, int split, const TcArgs &a) {
+    const int64_t row = n0 + q * 32 + lane;
+    float *out = a.split_k > 1 ? a.partial + int64_t(split) * a.m * a.n : a.y;
+#pragma unroll 1
+    for (int c0 = 16 * slot; c0 < BN; c0 += 16 * nslots) {
+        uint32_t v[16];
+        tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(c0), v);
+        tmem_ld_wait();
+        if (row < a.n) {
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                const int64_t mm = m0 + c0 + j;
+                if (mm < a.m) out[mm * a.n + row] = __uint_as_float(v[j]);
+            }
+        }
+    }
+}
+
+// ============================================================== plain kernel
+
+template <int BN>
+struct PlainCfg {
+    static constexpr int kW = kBM * kBK * 2;
+    static constexpr int kX = BN * kBK * 2;
+    static constexpr int kStage = kW + kX;
+    static constexpr uint32_t kTmemCols = BN < 32 ? 32u : uint32_t(BN);
+    static_assert(kStage % 1024 == 0, "stage tiles must keep 1024-byte alignment");
+};
+
+__host__ __device__ constexpr int plain_tail(int stages) { return (2 * stages + 2) * 8 + 16; }
+
+template <int BN>
+__global__ void __launch_bounds__(kPlainThreads, 1)
+    k_gemm_tc_plain(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const TcArgs a) {
+    using C = PlainCfg<BN>;
     extern __shared__ uint8_t smem_dyn[];
-    uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
-                                                 ~uintptr_t(1023));
+    uint8_t *tiles = align1024(smem_dyn);
     const int S = a.stages;
     uint64_t *full = reinterpret_cast<uint64_t *>(tiles + size_t(S) * C::kStage);
-    uint64_t *wready = full + S;
-    uint64_t *empty = wready + S;
+    uint64_t *empty = full + S;
     uint64_t *accf = empty + S;
     uint64_t *never = accf + 1;
-    uint32_t *rawmap = reinterpret_cast<uint32_t *>(never + 1);   // 4 words per stage
-    uint32_t *tmem_slot = rawmap + 4 * S;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(never + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n0 = int64_t(blockIdx.x) * kBM;
     const int64_t m0 = int64_t(blockIdx.y) * BN;
     const int split = blockIdx.z;
-    const int nks_total = int(a.k / kBK);
     const int ks_begin = split * a.ks_per_split;
-    const int nks = max(0, min(nks_total - ks_begin, a.ks_per_split));
+    const int nks = max(0, min(int(a.k / kBK) - ks_begin, a.ks_per_split));
     const uint64_t T = a.timeout_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&wready[s], 128);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
@@ -111,8 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmX);
-        prefetch_tensormap(&tmA);
-        if (PAL) prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmW);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -124,164 +167,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        int issued = 0;
-        const int64_t gpr = a.k / kGroup;   // groups per row of W
-        for (int ks = 0; ks < nks; ks++) {
-            const int s = ks % S;
-            const uint32_t ph = uint32_t(ks / S) & 1u;
-            if (ks >= S) {
-                const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ph ^ 1u, T));
-                if (!ok) {
-                    if (lane == 0) {
-                        flag_error(a.status, UW_DEVERR_TIMEOUT);
-                        *abort_flag = 1;
-                    }
+        if (lane == 0) {
+            int issued = 0;
+            for (int ks = 0; ks < nks; ks++) {
+                const int s = ks % S;
+                if (ks >= S && !mbar_wait(&empty[s], (uint32_t(ks / S) & 1u) ^ 1u, T)) {
+                    flag_error(a.status, UW_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
                     break;
                 }
-            }
-            if (*abort_flag) break;
-            const int kg = ks_begin + ks;
-            uint8_t *st = tiles + size_t(s) * C::kStage;
-            if (PAL) {
-                uint32_t mk[4];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int64_t row = n0 + lane + 32 * i;
-                    bool raw = false;
-                    if (row < a.n) {
-                        const int64_t g = row * gpr + kg;
-                        raw = (__ldg(a.flagbits + (g >> 5)) >> (g & 31)) & 1u;
-                    }
-                    mk[i] = __ballot_sync(0xFFFFFFFFu, raw);
-                }
-                if (lane < 4) rawmap[4 * s + lane] = lane == 0 ? mk[0] : lane == 1 ? mk[1] : lane == 2 ? mk[2] : mk[3];
-                const int nraw = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[s], uint32_t(C::kX + C::kSM + C::kPL + 64 * nraw));
-                    tma_load_2d(st + C::kOffX, &tmX, kg * kBK, int32_t(m0), &full[s]);
-                    tma_load_2d(st + C::kOffSM, &tmA, kg * kBK, int32_t(n0), &full[s]);
-                    tma_load_2d(st + C::kOffPL, &tmB, kg * (kBK / 2), int32_t(n0), &full[s]);
-                }
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    if ((mk[i] >> lane) & 1u) {
-                        const int r = lane + 32 * i;
-                        const int64_t g = (n0 + r) * gpr + kg;
-                        const uint32_t fw = __ldg(a.flagbits + (g >> 5));
-                        const uint32_t rank = __ldg(a.rawbase + (g >> 5)) + __popc(fw & ((1u << (g & 31)) - 1u));
-                        bulk_g2s(st + C::kOffRAW + r * 64, a.rawexp + uint64_t(rank) * kGroup, 64, &full[s]);
-                    }
-                }
-            } else if (lane == 0) {
+                if (*abort_flag) break;
+                const int kg = ks_begin + ks;
+                uint8_t *st = tiles + size_t(s) * C::kStage;
                 mbar_arrive_expect_tx(&full[s], uint32_t(C::kX + C::kW));
-                tma_load_2d(st + C::kOffX, &tmX, kg * kBK, int32_t(m0), &full[s]);
-                tma_load_2d(st, &tmA, kg * kBK, int32_t(n0), &full[s]);
+                tma_load_2d(st + C::kW, &tmX, kg * kBK, int32_t(m0), &full[s]);
+                tma_load_2d(st, &tmW, kg * kBK, int32_t(n0), &full[s]);
+                issued = ks + 1;
             }
-            issued = ks + 1;
+            for (int ks = max(0, issued - S); ks < issued; ks++)
+                mbar_wait(&full[ks % S], uint32_t(ks / S) & 1u, T);
         }
-        // let every copy this warp issued land before the CTA can exit
-        for (int ks = max(0, issued - S); ks < issued; ks++)
-            mbar_wait(&full[ks % S], uint32_t(ks / S) & 1u, T);
+        __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
             bool ok = true;
             if (a.debug_flags & UW_DEBUG_NEVER_ARRIVE) ok = mbar_wait(never, 0, T);
             for (int ks = 0; ks < nks && ok; ks++) {
                 const int s = ks % S;
-                const uint32_t ph = uint32_t(ks / S) & 1u;
-                ok = mbar_wait(&full[s], ph, T);
-                if (ok && PAL) ok = mbar_wait(&wready[s], ph, T);
+                ok = mbar_wait(&full[s], uint32_t(ks / S) & 1u, T);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t sa = smem_addr(tiles + size_t(s) * C::kStage);
-                const uint32_t sb = sa + C::kOffX;
-#pragma unroll
-                for (int kk = 0; kk < kBK / 16; kk++)
-                    tc_mma_bf16(tmem, smem_desc_k128(sa + 32 * kk), smem_desc_k128(sb + 32 * kk), idesc,
-                                (ks | kk) != 0);
+                mma_kstep<BN>(tmem, sa, sa + C::kW, ks == 0);
                 tc_commit(&empty[s]);
             }
             if (!ok) {
                 flag_error(a.status, UW_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
-            tc_commit(accf);   // fires once every MMA issued above has completed
+            tc_commit(accf);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ rebuild + epilogue
-        const int q = warp & 3;          // TMEM lane quarter this warp may access
-        const int r = q * 32 + lane;     // tile row
-        if (PAL) {
-            for (int ks = 0; ks < nks; ks++) {
-                const int s = ks % S;
-                const uint32_t ph = uint32_t(ks / S) & 1u;
-                if (!mbar_wait(&full[s], ph, T)) {
-                    flag_error(a.status, UW_DEVERR_TIMEOUT);
-                    break;
-                }
-                uint8_t *st = tiles + size_t(s) * C::kStage;
-                const uint8_t *smrow = st + C::kOffSM + r * 64;
-                const uint8_t *plrow = st + C::kOffPL + r * 32;
-                uint8_t *wrow = st + r * 128;
-                const int sw64 = (r >> 1) & 3, sw32 = (r >> 2) & 1, sw128 = r & 7;
-                uint4 smv[4], ev[4];
-#pragma unroll
-                for (int c = 0; c < 4; c++)
-                    smv[c] = *reinterpret_cast<const uint4 *>(smrow + ((c ^ sw64) << 4));
-                if ((rawmap[4 * s + q] >> lane) & 1u) {
-#pragma unroll
-                    for (int c = 0; c < 4; c++)
-                        ev[c] = *reinterpret_cast<const uint4 *>(st + C::kOffRAW + r * 64 + c * 16);
-                } else {
-                    const uint4 p0 = *reinterpret_cast<const uint4 *>(plrow + ((0 ^ sw32) << 4));
-                    const uint4 p1 = *reinterpret_cast<const uint4 *>(plrow + ((1 ^ sw32) << 4));
-                    pal_exponents(p0.x, a.pal, ev[0].x, ev[0].y);
-                    pal_exponents(p0.y, a.pal, ev[0].z, ev[0].w);
-                    pal_exponents(p0.z, a.pal, ev[1].x, ev[1].y);
-                    pal_exponents(p0.w, a.pal, ev[1].z, ev[1].w);
-                    pal_exponents(p1.x, a.pal, ev[2].x, ev[2].y);
-                    pal_exponents(p1.y, a.pal, ev[2].z, ev[2].w);
-                    pal_exponents(p1.z, a.pal, ev[3].x, ev[3].y);
-                    pal_exponents(p1.w, a.pal, ev[3].z, ev[3].w);
-                }
-#pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    *reinterpret_cast<uint4 *>(wrow + (((2 * c) ^ sw128) << 4)) =
-                        join8(ev[c].x, ev[c].y, smv[c].x, smv[c].y);
-                    *reinterpret_cast<uint4 *>(wrow + (((2 * c + 1) ^ sw128) << 4)) =
-                        join8(ev[c].z, ev[c].w, smv[c].z, smv[c].w);
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&wready[s]);
-            }
-        }
         const bool ok = mbar_wait(accf, 0, T);
         tc_fence_after();
         const bool skip = __any_sync(0xFFFFFFFFu, !ok || *abort_flag != 0 || nks == 0);
         if (!ok && lane == 0) flag_error(a.status, UW_DEVERR_TIMEOUT);
-        if (!skip) {
-            const int64_t row = n0 + r;
-            float *out = a.split_k > 1 ? a.partial + int64_t(split) * a.m * a.n : a.y;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(c0), v);
-                tmem_ld_wait();
-                if (row < a.n) {
-#pragma unroll
-                    for (int j = 0; j < 16; j++) {
-                        const int64_t mm = m0 + c0 + j;
-                        if (mm < a.m) out[mm * a.n + row] = __uint_as_float(v[j]);
-                    }
-                }
-            }
-        }
+        if (!skip) store_accumulator<BN>(tmem, warp & 3, 0, 1, lane, n0, m0, split, a);
     }
 
     tc_fence_before();
@@ -291,6 +223,282 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, C::kTmemCols);
     }
 }
+
+// ============================================================== fused kernel
+
+template <int BN>
+struct FusedCfg {
+    static constexpr int kWS = BN <= 64 ? 4 : 2;        // rebuilt-W ring (multiple of kGroups)
+    static constexpr int kXS = BN <= 64 ? 8 : (BN == 128 ? 4 : 2);   // X ring
+    static constexpr int kW = kBM * kBK * 2;            // rebuilt W tile
+    static constexpr int kX = BN * kBK * 2;             // X tile
+    static constexpr int kSM = kBM * kBK;               // sign/mantissa tile
+    static constexpr int kPL = kBM * kBK / 2;           // palette tile
+    static constexpr int kRAW = kBM * kGroup;           // raw exponents, one 64-byte slot per row
+    static constexpr int kCStage = kSM + kPL + kRAW;    // compressed ring stage
+    static constexpr int kOffPL = kSM, kOffRAW = kSM + kPL;
+    static constexpr uint32_t kTmemCols = BN < 32 ? 32u : uint32_t(BN);
+    static_assert(kW % 1024 == 0 && kX % 1024 == 0 && kCStage % 1024 == 0, "1024-byte alignment");
+};
+
+constexpr int kRawProducers = 4;      // warps; lane l of warp j owns tile row 32 j + l
+
+// after the rings: raw bitmap (128 rows x bw words), first raw rank per row,
+// barriers (c_full, c_empty per compressed stage; w_full, w_empty per W stage;
+// x_full, x_empty per X stage; accf, never), TMEM slot, abort flag
+__host__ __device__ constexpr int fused_tail(int cs, int ws, int xs, int bw) {
+    return kBM * bw * 4 + kBM * 4 + (2 * cs + 2 * ws + 2 * xs + 2) * 8 + 16;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    k_gemm_tc_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmSM,
+                    const __grid_constant__ CUtensorMap tmPL, const TcArgs a, int bw) {
+    using C = FusedCfg<BN>;
+    constexpr int WS = C::kWS, XS = C::kXS;
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *wring = align1024(smem_dyn);
+    uint8_t *xring = wring + WS * C::kW;
+    uint8_t *cring = xring + XS * C::kX;
+    const int CS = a.stages;                      // compressed stages (even)
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(cring + size_t(CS) * C::kCStage);   // [128][bw]
+    uint32_t *rank0 = bitmap + kBM * bw;                                                // [128]
+    uint64_t *c_full = reinterpret_cast<uint64_t *>(rank0 + kBM);
+    uint64_t *c_empty = c_full + CS;
+    uint64_t *w_full = c_empty + CS;
+    uint64_t *w_empty = w_full + WS;
+    uint64_t *x_full = w_empty + WS;
+    uint64_t *x_empty = x_full + XS;
+    uint64_t *accf = x_empty + XS;
+    uint64_t *never = accf + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(never + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = int64_t(blockIdx.x) * kBM;
+    const int64_t m0 = int64_t(blockIdx.y) * BN;
+    const int split = blockIdx.z;
+    const int ks_begin = split * a.ks_per_split;
+    const int nks = max(0, min(int(a.k / kBK) - ks_begin, a.ks_per_split));
+    const uint64_t T = a.timeout_ns;
+    constexpr int kFirstRebuildWarp = 3 + kRawProducers;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < CS; s++) {
+            mbar_init(&c_full[s], 1 + 32 * kRawProducers);   // TMA producer + raw-producer lanes
+            mbar_init(&c_empty[s], 128);
+        }
+        for (int s = 0; s < WS; s++) {
+            mbar_init(&w_full[s], 128);
+            mbar_init(&w_empty[s], 1);
+        }
+        for (int s = 0; s < XS; s++) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(never, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmSM);
+        prefetch_tensormap(&tmPL);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp >= kFirstRebuildWarp) {
+        // raw-group bitmap of the tile's rows over this split's K-steps (word j
+        // of row r holds K-steps 32j..32j+31) and each row's first raw rank
+        const int t = threadIdx.x - 32 * kFirstRebuildWarp, r = t & (kBM - 1), part = t >> 7;   // part 0..1
+        const int64_t row = n0 + r;
+        const int64_t gpr = a.k / kGroup;
+        const int64_t nflag = (a.n * gpr + 31) >> 5;
+        const int64_t g0 = row * gpr + ks_begin;
+        for (int j = part; j < bw; j += 2) {
+            uint32_t bits = 0u;
+            const int base = 32 * j;
+            if (row < a.n && base < nks) {
+                const int64_t gb = g0 + base;
+                const int64_t w = gb >> 5;
+                const uint32_t lo = __ldg(a.flagbits + w);
+                const uint32_t hi = w + 1 < nflag ? __ldg(a.flagbits + w + 1) : 0u;
+                bits = __funnelshift_r(lo, hi, uint32_t(gb & 31));
+                const int valid = nks - base;
+                if (valid < 32) bits &= (1u << valid) - 1u;
+            }
+            bitmap[r * bw + j] = bits;
+        }
+        if (part == 0) {
+            uint32_t rk = 0u;
+            if (row < a.n && nks > 0) {
+                const uint32_t fw = __ldg(a.flagbits + (g0 >> 5));
+                rk = __ldg(a.rawbase + (g0 >> 5)) + __popc(fw & ((1u << (g0 & 31)) - 1u));
+            }
+            rank0[r] = rk;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ compressed tiles (TMA)
+        if (lane == 0) {
+            int issued = 0;
+            for (int ks = 0; ks < nks; ks++) {
+                const int s = ks % CS;
+                if (ks >= CS && !mbar_wait(&c_empty[s], (uint32_t(ks / CS) & 1u) ^ 1u, T)) {
+                    flag_error(a.status, UW_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                const int kg = ks_begin + ks;
+                uint8_t *st = cring + size_t(s) * C::kCStage;
+                mbar_arrive_expect_tx(&c_full[s], uint32_t(C::kSM + C::kPL));
+                tma_load_2d(st, &tmSM, kg * kBK, int32_t(n0), &c_full[s]);
+                tma_load_2d(st + C::kOffPL, &tmPL, kg * (kBK / 2), int32_t(n0), &c_full[s]);
+                issued = ks + 1;
+            }
+            for (int ks = max(0, issued - CS); ks < issued; ks++)
+                mbar_wait(&c_full[ks % CS], uint32_t(ks / CS) & 1u, T);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            if (a.debug_flags & UW_DEBUG_NEVER_ARRIVE) ok = mbar_wait(never, 0, T);
+            for (int ks = 0; ks < nks && ok; ks++) {
+                const int ws = ks % WS, xs = ks % XS;
+                ok = mbar_wait(&x_full[xs], uint32_t(ks / XS) & 1u, T) &&
+                     mbar_wait(&w_full[ws], uint32_t(ks / WS) & 1u, T);
+                if (!ok) break;
+                tc_fence_after();
+                mma_kstep<BN>(tmem, smem_addr(wring + size_t(ws) * C::kW), smem_addr(xring + size_t(xs) * C::kX),
+                              ks == 0);
+                tc_commit(&w_empty[ws]);
+                tc_commit(&x_empty[xs]);
+            }
+            if (!ok) {
+                flag_error(a.status, UW_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            tc_commit(accf);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ------------------------------------------------ X producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int ks = 0; ks < nks; ks++) {
+                const int s = ks % XS;
+                if (ks >= XS && !mbar_wait(&x_empty[s], (uint32_t(ks / XS) & 1u) ^ 1u, T)) {
+                    flag_error(a.status, UW_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_arrive_expect_tx(&x_full[s], uint32_t(C::kX));
+                tma_load_2d(xring + size_t(s) * C::kX, &tmX, (ks_begin + ks) * kBK, int32_t(m0), &x_full[s]);
+                issued = ks + 1;
+            }
+            for (int ks = max(0, issued - XS); ks < issued; ks++)
+                mbar_wait(&x_full[ks % XS], uint32_t(ks / XS) & 1u, T);
+        }
+        __syncwarp();
+    } else if (warp < kFirstRebuildWarp) {
+        // ------------------------------------------------ raw producers
+        // lane owns row r; for every K-step it copies the row's raw exponents
+        // (64 B, four 16-byte cp.async) into the stage when the group is raw,
+        // and always arrives on c_full once its copies have landed
+        const int r = 32 * (warp - 3) + lane;
+        const uint32_t *bm = bitmap + r * bw;
+        uint32_t rank = rank0[r];
+        bool ok = true;
+        for (int ks = 0; ks < nks; ks++) {
+            const int s = ks % CS;
+            if (ks >= CS) ok = mbar_wait(&c_empty[s], (uint32_t(ks / CS) & 1u) ^ 1u, T);
+            if (!ok || *abort_flag) break;
+            if ((bm[ks >> 5] >> (ks & 31)) & 1u) {
+                const uint8_t *src = a.rawexp + uint64_t(rank) * kGroup;
+                uint8_t *dst = cring + size_t(s) * C::kCStage + C::kOffRAW + r * kGroup;
+#pragma unroll
+                for (int c = 0; c < 4; c++) cp_async16(dst + 16 * c, src + 16 * c);
+                rank++;
+            }
+            cp_async_mbar_arrive_noinc(&c_full[s]);
+        }
+        if (!ok) flag_error(a.status, UW_DEVERR_TIMEOUT);
+        cp_async_wait_all();
+    } else {
+        // ------------------------------------------------ rebuild groups, then epilogue
+        const int wi = warp - kFirstRebuildWarp;  // 0..7
+        const int q = warp & 3;               // TMEM lane quarter this warp may access
+        const int grp = wi >> 2;              // 0 or 1: K-steps ks = grp (mod 2)
+        const int r = q * 32 + lane;          // tile row
+        const int sw64 = (r >> 1) & 3, sw32 = (r >> 2) & 1, sw128 = r & 7;
+        const uint32_t *bm = bitmap + r * bw;
+        for (int ks = grp; ks < nks; ks += kGroups) {
+            const int cs = ks % CS, ws = ks % WS;
+            bool ok = mbar_wait(&c_full[cs], uint32_t(ks / CS) & 1u, T);
+            if (ok && ks >= WS) ok = mbar_wait(&w_empty[ws], (uint32_t(ks / WS) & 1u) ^ 1u, T);
+            if (!ok) {
+                flag_error(a.status, UW_DEVERR_TIMEOUT);
+                break;
+            }
+            const uint8_t *st = cring + size_t(cs) * C::kCStage;
+            const uint8_t *smrow = st + r * 64;
+            const uint8_t *plrow = st + C::kOffPL + r * 32;
+            uint8_t *wrow = wring + size_t(ws) * C::kW + r * 128;
+            const bool raw = (bm[ks >> 5] >> (ks & 31)) & 1u;
+#pragma unroll
+            for (int h = 0; h < 2; h++) {      // two halves of the row, 32 weights each
+                const uint4 s0 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h) ^ sw64) << 4));
+                const uint4 s1 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h + 1) ^ sw64) << 4));
+                uint32_t rv[8];
+                if (raw) {
+                    const uint8_t *rp = st + C::kOffRAW + r * kGroup + h * 32;
+                    const uint4 e0 = *reinterpret_cast<const uint4 *>(rp);
+                    const uint4 e1 = *reinterpret_cast<const uint4 *>(rp + 16);
+                    rv[0] = rot4(e0.x); rv[1] = rot4(e0.y); rv[2] = rot4(e0.z); rv[3] = rot4(e0.w);
+                    rv[4] = rot4(e1.x); rv[5] = rot4(e1.y); rv[6] = rot4(e1.z); rv[7] = rot4(e1.w);
+                } else {
+                    const uint4 p = *reinterpret_cast<const uint4 *>(plrow + ((h ^ sw32) << 4));
+                    pal_rot(p.x, a.pal, rv[0], rv[1]);
+                    pal_rot(p.y, a.pal, rv[2], rv[3]);
+                    pal_rot(p.z, a.pal, rv[4], rv[5]);
+                    pal_rot(p.w, a.pal, rv[6], rv[7]);
+                }
+                const int c0 = 4 * h;
+                *reinterpret_cast<uint4 *>(wrow + (((c0 + 0) ^ sw128) << 4)) = join8(rv[0], rv[1], s0.x, s0.y);
+                *reinterpret_cast<uint4 *>(wrow + (((c0 + 1) ^ sw128) << 4)) = join8(rv[2], rv[3], s0.z, s0.w);
+                *reinterpret_cast<uint4 *>(wrow + (((c0 + 2) ^ sw128) << 4)) = join8(rv[4], rv[5], s1.x, s1.y);
+                *reinterpret_cast<uint4 *>(wrow + (((c0 + 3) ^ sw128) << 4)) = join8(rv[6], rv[7], s1.z, s1.w);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&c_empty[cs]);
+            mbar_arrive(&w_full[ws]);
+        }
+        const bool ok = mbar_wait(accf, 0, T);
+        tc_fence_after();
+        const bool skip = __any_sync(0xFFFFFFFFu, !ok || *abort_flag != 0 || nks == 0);
+        if (!ok && lane == 0) flag_error(a.status, UW_DEVERR_TIMEOUT);
+        if (!skip) store_accumulator<BN>(tmem, q, grp, kGroups, lane, n0, m0, split, a);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ============================================================== split-K reduce
 
 __global__ void k_splitk_reduce(const float *__restrict__ partial, int split_k, int64_t count,
                                 float *__restrict__ y) {
@@ -315,7 +523,7 @@ __global__ void k_splitk_reduce(const float *__restrict__ partial, int split_k, 
     }
 }
 
-// ------------------------------------------------------------------ host side
+// ============================================================== host side
 
 bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
@@ -331,88 +539,117 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool PAL>
-cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
-    using C = Cfg<BN, PAL>;
-    int stages = p.stages;
-    const int max_stages = (kMaxSmem - 1024 - tail_bytes(8)) / C::kStage;
-    if (stages <= 0 || stages > max_stages) stages = max_stages;
-    if (stages > 8) stages = 8;
+// K split into slices of whole K-steps, none empty
+void split_k_slices(const TcLaunch &p, TcArgs &a) {
+    const int nks = int(p.k / kBK);
+    int split = std::max(1, std::min(p.split_k, nks));
+    a.ks_per_split = (nks + split - 1) / split;
+    a.split_k = (nks + a.ks_per_split - 1) / a.ks_per_split;
+}
+
+// one-time per (kernel, device, stage count): shared-memory opt-in and a check
+// that co-resident CTAs fit the 512 TMEM columns (tcgen05.alloc would block)
+template <class K>
+cudaError_t prepare(K kern, int threads, size_t smem, uint32_t tmem_cols, int key, int (&ready)[16]) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (ready[key] == dev) return cudaSuccess;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm * int(tmem_cols) > 512) return cudaErrorInvalidConfiguration;
+    ready[key] = dev;
+    return cudaSuccess;
+}
+
+template <int BN>
+cudaError_t launch_plain(const TcLaunch &p, cudaStream_t stream) {
+    using C = PlainCfg<BN>;
+    const int max_stages = std::min(8, (kMaxSmem - 1024 - plain_tail(8)) / C::kStage);
+    int stages = (p.stages <= 0 || p.stages > max_stages) ? max_stages : p.stages;
     if (stages < 2) return cudaErrorInvalidValue;
-    const size_t smem = size_t(stages) * C::kStage + 1024 + tail_bytes(stages);
-
-    CUtensorMap mx, ma, mb;
-    std::memset(&mb, 0, sizeof(mb));
-    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m),
-                  uint64_t(p.k) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    const size_t smem = size_t(stages) * C::kStage + 1024 + plain_tail(stages);
+    CUtensorMap mx, mw;
+    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2,
+                  kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.w_bf16, uint64_t(p.k), uint64_t(p.n),
+                  uint64_t(p.k) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (PAL) {
-        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n),
-                      uint64_t(p.k), kBK, kBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-            !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n),
-                      uint64_t(p.k / 2), kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
-            return cudaErrorInvalidValue;
-    } else {
-        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.w_bf16, uint64_t(p.k), uint64_t(p.n),
-                      uint64_t(p.k) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-        mb = ma;
-    }
-
     TcArgs a{};
     a.m = p.m;
     a.n = p.n;
     a.k = p.k;
-    const int nks = int(p.k / kBK);
-    int split = std::max(1, std::min(p.split_k, nks));
-    a.ks_per_split = (nks + split - 1) / split;
-    split = (nks + a.ks_per_split - 1) / a.ks_per_split;   // no empty slice
-    a.split_k = split;
+    split_k_slices(p, a);
     a.stages = stages;
     a.debug_flags = p.debug_flags;
     a.timeout_ns = p.timeout_ns;
     a.y = p.y;
     a.partial = p.partial;
     a.status = p.dev_status;
-    if (PAL) {
-        a.flagbits = p.w->flagbits;
-        a.rawbase = p.w->rawbase;
-        a.rawexp = p.w->rawexp;
-        auto pack = [&](int i) {
-            return uint32_t(p.w->palette[i]) | uint32_t(p.w->palette[i + 1]) << 8 |
-                   uint32_t(p.w->palette[i + 2]) << 16 | uint32_t(p.w->palette[i + 3]) << 24;
-        };
-        a.pal = Palette16{pack(0), pack(4), pack(8), pack(12)};
-    }
-    if (split > 1 && !p.partial) return cudaErrorInvalidValue;
-
-    auto kern = k_gemm_tc<BN, PAL>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (a.split_k > 1 && !p.partial) return cudaErrorInvalidValue;
+    static thread_local int ready[16] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
+    cudaError_t err = prepare(k_gemm_tc_plain<BN>, kPlainThreads, smem, C::kTmemCols, stages, ready);
     if (err != cudaSuccess) return err;
-    // TMEM: co-resident CTAs must fit in 512 columns, or tcgen05.alloc would block
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm * int(C::kTmemCols) > 512) return cudaErrorInvalidConfiguration;
-
-    dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN - 1) / BN), unsigned(split));
-    kern<<<grid, kThreads, smem, stream>>>(mx, ma, mb, a);
+    dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN - 1) / BN), unsigned(a.split_k));
+    k_gemm_tc_plain<BN><<<grid, kPlainThreads, smem, stream>>>(mx, mw, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    if (split > 1) return launch_splitk_reduce(p.partial, split, p.m * p.n, p.y, stream);
+    if (a.split_k > 1) return launch_splitk_reduce(p.partial, a.split_k, p.m * p.n, p.y, stream);
     return cudaSuccess;
 }
 
-template <bool PAL>
-cudaError_t launch_pal(const TcLaunch &p, cudaStream_t stream) {
-    switch (p.bn) {
-        case 16: return launch_bn<16, PAL>(p, stream);
-        case 32: return launch_bn<32, PAL>(p, stream);
-        case 64: return launch_bn<64, PAL>(p, stream);
-        case 128: return launch_bn<128, PAL>(p, stream);
-        case 256: return launch_bn<256, PAL>(p, stream);
-        default: return cudaErrorInvalidValue;
-    }
+template <int BN>
+cudaError_t launch_fused(const TcLaunch &p, cudaStream_t stream) {
+    using C = FusedCfg<BN>;
+    TcArgs a{};
+    a.m = p.m;
+    a.n = p.n;
+    a.k = p.k;
+    split_k_slices(p, a);
+    const int bw = (a.ks_per_split + 31) / 32;     // raw bitmap words per row
+    const int fixed = C::kWS * C::kW + C::kXS * C::kX + 1024 + fused_tail(8, C::kWS, C::kXS, bw);
+    int max_cs = (kMaxSmem - fixed) / C::kCStage;
+    max_cs = std::min(8, max_cs) & ~1;      // even: each rebuild group owns every other stage
+    int cs = (p.stages <= 0 || p.stages > max_cs) ? max_cs : (p.stages & ~1);
+    if (cs < 2) return cudaErrorInvalidValue;
+    const size_t smem = size_t(C::kWS) * C::kW + size_t(C::kXS) * C::kX + size_t(cs) * C::kCStage + 1024 +
+                        fused_tail(cs, C::kWS, C::kXS, bw);
+    CUtensorMap mx, msm, mpl;
+    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2,
+                  kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&msm, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k),
+                  kBK, kBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map(&mpl, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n),
+                  uint64_t(p.k / 2), kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
+        return cudaErrorInvalidValue;
+    a.stages = cs;
+    a.debug_flags = p.debug_flags;
+    a.timeout_ns = p.timeout_ns;
+    a.y = p.y;
+    a.partial = p.partial;
+    a.status = p.dev_status;
+    a.flagbits = p.w->flagbits;
+    a.rawbase = p.w->rawbase;
+    a.rawexp = p.w->rawexp;
+    a.pal = make_palette16(p.w->palette);
+    if (a.split_k > 1 && !p.partial) return cudaErrorInvalidValue;
+    static thread_local int ready[16] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
+    cudaError_t err = prepare(k_gemm_tc_fused<BN>, kFusedThreads, smem, C::kTmemCols, cs, ready);
+    if (err != cudaSuccess) return err;
+    dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN - 1) / BN), unsigned(a.split_k));
+    k_gemm_tc_fused<BN><<<grid, kFusedThreads, smem, stream>>>(mx, msm, mpl, a, bw);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    if (a.split_k > 1) return launch_splitk_reduce(p.partial, a.split_k, p.m * p.n, p.y, stream);
+    return cudaSuccess;
+}
+
+template <int BN>
+cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
+    return p.w_bf16 ? launch_plain<BN>(p, stream) : launch_fused<BN>(p, stream);
 }
 
 }  // namespace
@@ -426,7 +663,14 @@ cudaError_t launch_splitk_reduce(const float *partial, int split_k, int64_t coun
 }
 
 cudaError_t launch_gemm_tc(const TcLaunch &p, cudaStream_t stream) {
-    return p.w_bf16 ? launch_pal<false>(p, stream) : launch_pal<true>(p, stream);
+    switch (p.bn) {
+        case 16: return launch_bn<16>(p, stream);
+        case 32: return launch_bn<32>(p, stream);
+        case 64: return launch_bn<64>(p, stream);
+        case 128: return launch_bn<128>(p, stream);
+        case 256: return launch_bn<256>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 EncodeTiledFn encode_tiled_fn() {

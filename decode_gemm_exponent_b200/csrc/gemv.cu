@@ -1,17 +1,23 @@
-// gemv.cu -- CUDA-core FMA GEMV for small batches (m <= 8), Y = X * W^T.
+// gemv.cu -- CUDA-core GEMV for small batches (m <= 8), Y = X * W^T.
 //
 // The Unweight page (§十) names the fixed cost of the reconstructive matmul at
 // small batch as a main overhead, and (§六) notes that at batch 1-64 the
 // plain path often wins.  At m <= 4 the job is a pure HBM stream, so this
 // kernel reads the compressed planes with coalesced 16-byte loads straight
 // into registers and rebuilds BF16 there (§五: the rebuilt weights never go
-// back to HBM), with no shared-memory staging at all.
+// back to HBM), with no shared-memory staging.
 //
 // One warp owns R consecutive rows of W and walks K in steps of 512: lane l
-// handles weights [k0 + 16 l, k0 + 16 l + 16).  Per lane the products are
-// accumulated in a fixed order (k ascending) and the 32 lane sums are then
-// combined by a fixed xor-butterfly, so the fused kernel and its plain-BF16
-// twin (same template, other loader) give bit-identical results.
+// handles weights [k0 + 16 l, k0 + 16 l + 16); the loads of the next step
+// are issued before the current step's arithmetic.  Before the loop the warp
+// loads the raw-group bitmap words of its rows and their prefix counts (one
+// word per lane) and later broadcasts them with shuffles, so the loop issues
+// only independent loads.  Products are accumulated with the mixed-precision
+// FMA (BF16 x BF16 + FP32, one rounding) in a fixed order (k ascending) and
+// the 32 lane sums are combined by a fixed xor-butterfly, so the fused kernel
+// and its plain-BF16 twin (same template, other loader) are bit-identical.
+#include <algorithm>
+
 #include "device_common.cuh"
 #include "kernels.h"
 #include "uw_format.h"
@@ -34,40 +40,69 @@ struct GemvArgs {
     Palette16 palette;
     int64_t n, k;
     float *y;
+    uint32_t *status;
 };
 
-__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+// Loads of one 16-weight piece of one row (issued one iteration ahead).
+struct Piece {
+    uint4 a;          // plain: weights 0..7 (BF16); fused: sign/mantissa bytes
+    uint4 b;          // plain: weights 8..15;       fused: .x/.y palette words
+    uint32_t rank;    // fused: raw-group rank
+    bool raw;
+};
 
-// 16 weights of row `row` starting at column k0, as 8 BF16 pairs.
 template <bool PAL>
-__device__ __forceinline__ void load_weights(const GemvArgs &a, int64_t row, int64_t k0,
-                                             uint32_t (&wv)[8]) {
+__device__ __forceinline__ Piece load_piece(const GemvArgs &a, int64_t row, int64_t k0, bool live,
+                                            uint32_t fw, uint32_t rb, int64_t g) {
+    Piece p;
+    p.a = make_uint4(0u, 0u, 0u, 0u);
+    p.b = p.a;
+    p.raw = false;
+    p.rank = 0;
     const int64_t e0 = row * a.k + k0;
     if (!PAL) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(a.w_bf16 + e0);
-        const uint4 v0 = __ldcs(p), v1 = __ldcs(p + 1);
-        wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
-        wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
-    } else {
-        const uint2 pw = __ldcs(reinterpret_cast<const uint2 *>(a.pal + e0 / 8));
-        const uint4 s = __ldcs(reinterpret_cast<const uint4 *>(a.sm + e0));
-        const int64_t g = e0 / kGroup;
-        const uint32_t fw = __ldg(a.flagbits + (g >> 5));
-        uint32_t e[4];
-        if ((fw >> (g & 31)) & 1u) {
-            const uint32_t rank = __ldg(a.rawbase + (g >> 5)) + __popc(fw & ((1u << (g & 31)) - 1u));
-            const uint4 r = __ldg(reinterpret_cast<const uint4 *>(a.rawexp + uint64_t(rank) * kGroup +
-                                                                 (e0 & (kGroup - 1))));
-            e[0] = r.x; e[1] = r.y; e[2] = r.z; e[3] = r.w;
-        } else {
-            pal_exponents(pw.x, a.palette, e[0], e[1]);
-            pal_exponents(pw.y, a.palette, e[2], e[3]);
+        if (live) {
+            const uint4 *q = reinterpret_cast<const uint4 *>(a.w_bf16 + e0);
+            p.a = __ldcs(q);
+            p.b = __ldcs(q + 1);
         }
-        join4(e[0], s.x, wv[0], wv[1]);
-        join4(e[1], s.y, wv[2], wv[3]);
-        join4(e[2], s.z, wv[4], wv[5]);
-        join4(e[3], s.w, wv[6], wv[7]);
+    } else {
+        const uint32_t bit = uint32_t(g) & 31u;
+        p.raw = live && ((fw >> bit) & 1u);
+        p.rank = rb + __popc(fw & ((1u << bit) - 1u));
+        if (live) {
+            p.a = __ldcs(reinterpret_cast<const uint4 *>(a.sm + e0));
+            const uint2 pw = __ldcs(reinterpret_cast<const uint2 *>(a.pal + e0 / 8));
+            p.b.x = pw.x;
+            p.b.y = pw.y;
+        }
+    }
+    return p;
+}
+
+// Piece -> 8 BF16 pairs
+template <bool PAL>
+__device__ __forceinline__ void rebuild_piece(const GemvArgs &a, const Piece &p, int64_t k0,
+                                              uint32_t (&wv)[8]) {
+    if (!PAL) {
+        wv[0] = p.a.x; wv[1] = p.a.y; wv[2] = p.a.z; wv[3] = p.a.w;
+        wv[4] = p.b.x; wv[5] = p.b.y; wv[6] = p.b.z; wv[7] = p.b.w;
+    } else {
+        uint32_t r0, r1, r2, r3;
+        if (p.raw) {
+            const uint4 rx = __ldg(reinterpret_cast<const uint4 *>(a.rawexp + uint64_t(p.rank) * kGroup + (k0 & 63)));
+            r0 = rot4(rx.x);
+            r1 = rot4(rx.y);
+            r2 = rot4(rx.z);
+            r3 = rot4(rx.w);
+        } else {
+            pal_rot(p.b.x, a.palette, r0, r1);
+            pal_rot(p.b.y, a.palette, r2, r3);
+        }
+        join4(r0, p.a.x, wv[0], wv[1]);
+        join4(r1, p.a.y, wv[2], wv[3]);
+        join4(r2, p.a.z, wv[4], wv[5]);
+        join4(r3, p.a.w, wv[6], wv[7]);
     }
 }
 
@@ -76,6 +111,59 @@ __global__ void __launch_bounds__(kWarps * 32) k_gemv_fma(const GemvArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = (int64_t(blockIdx.x) * kWarps + warp) * R;
     if (row0 >= a.n) return;
+    const int64_t gpr = a.k >> 6;                 // groups per row
+    const int nit = int((a.k + 511) >> 9);
+
+    // raw-group bitmap words covering each row, one per lane
+    uint32_t fw_l[R], rb_l[R];
+    int64_t wfirst[R];
+    bool direct = false;
+    if (PAL) {
+#pragma unroll
+        for (int r = 0; r < R; r++) {
+            const int64_t row = min(row0 + r, a.n - 1);
+            const int64_t g0 = row * gpr;
+            wfirst[r] = g0 >> 5;
+            const int64_t nw = ((g0 + gpr - 1) >> 5) - wfirst[r] + 1;
+            direct |= nw > 32;
+            fw_l[r] = lane < nw ? __ldg(a.flagbits + wfirst[r] + lane) : 0u;
+            rb_l[r] = lane < nw ? __ldg(a.rawbase + wfirst[r] + lane) : 0u;
+        }
+    }
+
+    // issue the loads of iteration `it` (all lanes take part: shuffles)
+    auto load_it = [&](int it, Piece (&pc)[R], uint4 (&xc)[M][2]) {
+        const int64_t k0 = int64_t(it) * 512 + lane * 16;
+        const bool act = k0 < a.k;
+#pragma unroll
+        for (int r = 0; r < R; r++) {
+            const int64_t row = row0 + r;
+            const bool live = act && row < a.n;
+            uint32_t fw = 0u, rb = 0u;
+            int64_t g = 0;
+            if (PAL) {
+                g = min(row, a.n - 1) * gpr + (k0 >> 6);
+                if (!direct) {
+                    const int idx = int((g >> 5) - wfirst[r]) & 31;
+                    fw = __shfl_sync(0xFFFFFFFFu, fw_l[r], idx);
+                    rb = __shfl_sync(0xFFFFFFFFu, rb_l[r], idx);
+                } else if (live) {
+                    fw = __ldg(a.flagbits + (g >> 5));
+                    rb = __ldg(a.rawbase + (g >> 5));
+                }
+            }
+            pc[r] = load_piece<PAL>(a, row, k0, live, fw, rb, g);
+        }
+#pragma unroll
+        for (int m = 0; m < M; m++) {
+            xc[m][0] = xc[m][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (act) {
+                const uint4 *xp = reinterpret_cast<const uint4 *>(a.x + int64_t(m) * a.k + k0);
+                xc[m][0] = __ldg(xp);
+                xc[m][1] = __ldg(xp + 1);
+            }
+        }
+    };
 
     float acc[M][R];
 #pragma unroll
@@ -83,31 +171,30 @@ __global__ void __launch_bounds__(kWarps * 32) k_gemv_fma(const GemvArgs a) {
 #pragma unroll
         for (int r = 0; r < R; r++) acc[m][r] = 0.f;
 
-#pragma unroll 2
-    for (int64_t k0 = int64_t(lane) * 16; k0 < a.k; k0 += 512) {
+    Piece pc[R], pn[R];
+    uint4 xc[M][2], xn[M][2];
+    load_it(0, pc, xc);
+    for (int it = 0; it < nit; it++) {
+        if (it + 1 < nit) load_it(it + 1, pn, xn);
+        const int64_t k0 = int64_t(it) * 512 + lane * 16;
         uint32_t wv[R][8];
 #pragma unroll
-        for (int r = 0; r < R; r++) {
-            if (row0 + r < a.n) load_weights<PAL>(a, row0 + r, k0, wv[r]);
-            else {
-#pragma unroll
-                for (int j = 0; j < 8; j++) wv[r][j] = 0u;
-            }
-        }
+        for (int r = 0; r < R; r++) rebuild_piece<PAL>(a, pc[r], k0, wv[r]);
 #pragma unroll
         for (int m = 0; m < M; m++) {
-            const uint4 *xp = reinterpret_cast<const uint4 *>(a.x + int64_t(m) * a.k + k0);
-            const uint4 x0 = __ldg(xp), x1 = __ldg(xp + 1);
-            const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            const uint32_t xv[8] = {xc[m][0].x, xc[m][0].y, xc[m][0].z, xc[m][0].w,
+                                    xc[m][1].x, xc[m][1].y, xc[m][1].z, xc[m][1].w};
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const float xl = bf_lo(xv[j]), xh = bf_hi(xv[j]);
+            for (int j = 0; j < 8; j++)
 #pragma unroll
-                for (int r = 0; r < R; r++) {
-                    acc[m][r] = fmaf(xl, bf_lo(wv[r][j]), acc[m][r]);
-                    acc[m][r] = fmaf(xh, bf_hi(wv[r][j]), acc[m][r]);
-                }
-            }
+                for (int r = 0; r < R; r++) acc[m][r] = fma2_bf16(xv[j], wv[r][j], acc[m][r]);
+        }
+#pragma unroll
+        for (int r = 0; r < R; r++) pc[r] = pn[r];
+#pragma unroll
+        for (int m = 0; m < M; m++) {
+            xc[m][0] = xn[m][0];
+            xc[m][1] = xn[m][1];
         }
     }
 
@@ -154,13 +241,14 @@ cudaError_t launch_r(const GemvArgs &a, int m, bool pal, cudaStream_t stream) {
 
 cudaError_t launch_gemv_fma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
                             const uint8_t *pal_plane, int64_t n, int64_t k, float *y,
-                            int rows_per_warp, cudaStream_t stream) {
+                            int rows_per_warp, uint32_t *status, cudaStream_t stream) {
     GemvArgs a{};
     a.x = x;
     a.w_bf16 = w_bf16;
     a.n = n;
     a.k = k;
     a.y = y;
+    a.status = status;
     const bool pal = pal_plane != nullptr;
     if (pal) {
         a.sm = w->sm;
@@ -168,11 +256,7 @@ cudaError_t launch_gemv_fma(const uint16_t *x, int m, const uint16_t *w_bf16, co
         a.flagbits = w->flagbits;
         a.rawbase = w->rawbase;
         a.rawexp = w->rawexp;
-        auto pack = [&](int i) {
-            return uint32_t(w->palette[i]) | uint32_t(w->palette[i + 1]) << 8 |
-                   uint32_t(w->palette[i + 2]) << 16 | uint32_t(w->palette[i + 3]) << 24;
-        };
-        a.palette = Palette16{pack(0), pack(4), pack(8), pack(12)};
+        a.palette = make_palette16(w->palette);
     }
     if (rows_per_warp == 1) return launch_r<1>(a, m, pal, stream);
     if (rows_per_warp == 2) return launch_r<2>(a, m, pal, stream);

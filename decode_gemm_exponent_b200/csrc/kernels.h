@@ -16,10 +16,11 @@ cudaError_t launch_huff_decode(const uw_dmat &w, uint16_t *out_bf16, uint8_t *ou
 
 // CUDA-core FMA GEMV, m <= 8 (Unweight page §七, small-batch case).
 // pal_plane == nullptr: plain BF16 weights `w_bf16`; otherwise the fused
-// palette path using `w` (sm/raw planes) and `pal_plane`.
+// palette path using `w` (sm/raw planes) and `pal_plane`.  One warp per
+// `rows_per_warp` (1 or 2) rows.
 cudaError_t launch_gemv_fma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
                             const uint8_t *pal_plane, int64_t n, int64_t k, float *y,
-                            int rows_per_warp, cudaStream_t stream);
+                            int rows_per_warp, uint32_t *status, cudaStream_t stream);
 
 // tcgen05 GEMM (Unweight page §七, reconstructive matmul), token tile `bn`.
 struct TcLaunch {

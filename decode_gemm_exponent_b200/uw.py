@@ -17,7 +17,8 @@ from typing import Optional, Sequence
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libuw.so")
+# the in-tree build; UW_LIBRARY may point at another build of the same library
+LIB_PATH = os.environ.get("UW_LIBRARY") or os.path.join(_HERE, "libuw.so")
 
 UW_OK = 0
 STATUS_NAMES = {0: "UW_OK", 1: "UW_ERR_INVALID_ARG", 2: "UW_ERR_UNSUPPORTED_SHAPE",
