@@ -36,7 +36,8 @@ DEBUG_NEVER_ARRIVE = 1
 EXPORTS = ("uw_status_str", "uw_version", "uw_encode", "uw_blob_data", "uw_blob_free",
            "uw_blob_info_get", "uw_matrix_bind", "uw_device_status", "uw_decode_to_bf16",
            "uw_transcode_palette", "uw_plan_default", "uw_workspace_size", "uw_fused_matmul",
-           "uw_matmul_bf16", "uw_autotune_workspace_size", "uw_plan_autotune")
+           "uw_matmul_bf16", "uw_autotune_workspace_size", "uw_plan_autotune",
+           "uw_fused_matmul_noalloc")
 
 
 class UwError(RuntimeError):
@@ -115,6 +116,7 @@ def lib() -> ctypes.CDLL:
         "uw_fused_matmul": (ctypes.c_int, [P, I64, ctypes.POINTER(DMat), P, P, ctypes.POINTER(Plan),
                                            P, SZ, P]),
         "uw_matmul_bf16": (ctypes.c_int, [P, I64, P, I64, I64, P, ctypes.POINTER(Plan), P, SZ, P, P]),
+        "uw_fused_matmul_noalloc": (ctypes.c_int, [P, I64, ctypes.POINTER(DMat), P, ctypes.POINTER(Plan), P]),
         "uw_autotune_workspace_size": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(DMat)), ctypes.c_int,
                                                       ctypes.POINTER(I64), ctypes.c_int,
                                                       ctypes.POINTER(SZ)]),
@@ -240,6 +242,18 @@ class Matrix:
                                     ctypes.byref(plan), _ptr(ws), ws.numel() if ws is not None else 0,
                                     _stream_handle(stream)), "uw_fused_matmul")
         return y
+
+
+def fused_matmul_noalloc(mat: "Matrix", x, plan: Plan, y=None, stream=None):
+    """uw_fused_matmul_noalloc: the fused matmul with no caller workspace (the
+    split-K partial sums live in a fixed library-owned device array)."""
+    import torch
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty(m, mat.n, dtype=torch.float32, device=x.device)
+    check(lib().uw_fused_matmul_noalloc(_ptr(x), m, ctypes.byref(mat.dmat), _ptr(y), ctypes.byref(plan),
+                                        _stream_handle(stream)), "uw_fused_matmul_noalloc")
+    return y
 
 
 def workspace_size(m: int, n: int, k: int, plan: Plan) -> int:

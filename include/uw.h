@@ -229,6 +229,32 @@ uw_status uw_matmul_bf16(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev
                          void *ws, size_t ws_bytes, uint32_t *dev_status, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Matmul without a caller workspace (no counterpart on the Unweight page).   */
+
+/* Bytes of the library-owned scratch array used by uw_fused_matmul_noalloc. */
+#define UW_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* uw_fused_matmul for callers that cannot give the library device memory
+ * (an engine that hands its plug-ins no allocator and forbids cudaMalloc
+ * after start-up, or a process whose device memory is already reserved by
+ * another allocator).  Same arguments and results as uw_fused_matmul with
+ * pal_dev = NULL, but no workspace: the split-K partial sums go to a fixed
+ * array of UW_NOALLOC_SCRATCH_BYTES in the library's own device memory, which
+ * every GPU that loads the library holds until the process exits.  Nothing is
+ * allocated per call (no cudaMalloc, no allocating library routine).
+ *   - plan->pipeline must be UW_PIPE_DIRECT_PALETTE (INVALID_ARG otherwise);
+ *     a plan whose uw_workspace_size exceeds UW_NOALLOC_SCRATCH_BYTES is
+ *     rejected with UW_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array: calls that may overlap on
+ *     the GPU (other streams, other threads) race and must be serialised by
+ *     the caller.  No state carries over between calls; every partial sum a
+ *     call reads was written by that same call.                             */
+uw_status uw_fused_matmul_noalloc(const uint16_t *x_dev, int64_t m, const uw_dmat *w,
+                                  float *y_dev, const uw_plan *plan, void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Autotuner (Unweight page §九).                                             */
 
 /* For every matrix mats[i] and batch size ms[j], time the candidate
