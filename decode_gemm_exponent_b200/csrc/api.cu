@@ -92,7 +92,7 @@ extern "C" const char *uw_status_str(int s) {
     }
 }
 
-extern "C" const char *uw_version(void) { return "uw 1.0 (blob v1, sm_100a)"; }
+extern "C" const char *uw_version(void) { return "uw 1.1 (blob v2, sm_100a)"; }
 
 extern "C" uw_status uw_matrix_bind(const void *host_blob, size_t bytes, const void *dev_blob,
                                     uint32_t *dev_status, int verify_payload, uw_dmat *out) {

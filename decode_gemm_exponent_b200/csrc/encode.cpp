@@ -137,17 +137,16 @@ void build_dlut(const uint8_t len[16], const uint32_t code[16], uint32_t *lut) {
         }
     }
     for (uint32_t v = 0; v < uint32_t(kLutEntries); v++) {
-        uint32_t syms = 0, cnt = 0, pos = 0, first_len = 0;
+        uint32_t syms = 0, cnt = 0, pos = 0;
         while (cnt < uint32_t(kLutMaxSyms)) {
             uint32_t rest = (v << pos) & uint32_t(kLutEntries - 1);
             uint32_t l = len1[rest];
             if (!l || pos + l > uint32_t(kLutBits)) break;
             syms |= uint32_t(sym1[rest]) << (4 * cnt);
-            if (!cnt) first_len = l;
             cnt++;
             pos += l;
         }
-        lut[v] = syms | (cnt << 20) | (pos << 23) | (first_len << 27);
+        lut[v] = lut_entry(syms, cnt, pos);
     }
 }
 

@@ -1,4 +1,4 @@
-// uw_format.h -- serialized blob layout (version 1) and helpers shared by the
+// uw_format.h -- serialized blob layout (version 2) and helpers shared by the
 // host encoder and the C-ABI.  Little-endian throughout.
 //
 // A blob is a 512-byte header followed by the sections listed in uw.h
@@ -14,7 +14,7 @@
 namespace uw {
 
 constexpr uint32_t kMagic = 0x31425755u;     // "UWB1"
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 constexpr int kChunkGroups = 4;              // groups (of 64 weights) per stream chunk
 constexpr int kGroup = 64;                   // weights per group ("row of 64 weights")
 constexpr int kMaxCodeLen = 12;              // code-length limit == decode window bits
@@ -52,12 +52,26 @@ static_assert(sizeof(Header) <= kHeaderBytes, "header too large");
 
 // Decode-table entry (UW_SEC_DLUT), indexed by the next 12 stream bits:
 //   bits  0..19  up to 5 decoded symbols (palette indices), 4 bits each, first lowest
-//   bits 20..22  number of whole codes found in the window (0 = no code matches)
-//   bits 23..26  total bits those codes use
-//   bits 27..30  length of the first code
-constexpr uint32_t lut_nsym(uint32_t e) { return (e >> 20) & 7u; }
-constexpr uint32_t lut_bits(uint32_t e) { return (e >> 23) & 15u; }
-constexpr uint32_t lut_len0(uint32_t e) { return (e >> 27) & 15u; }
+//   bits 20..24  4 x the number of whole codes in the window, i.e. the number
+//                of symbol bits in 0..19 (0 = no code matches the window)
+//   bit  25      set when no code matches the window (corrupt stream or an
+//                incomplete one-symbol code)
+//   bits 28..31  total stream bits those codes use (12 when none matches, so a
+//                decoder that keeps going over a corrupt window still advances)
+// The symbol-bit count and the stream-bit count are the two shift amounts a
+// decoder needs per lookup, so both are stored ready to use.
+#ifdef __CUDACC__
+#define UW_HOST_DEVICE __host__ __device__
+#else
+#define UW_HOST_DEVICE
+#endif
+constexpr uint32_t kLutInvalid = 1u << 25;
+UW_HOST_DEVICE constexpr uint32_t lut_symbits(uint32_t e) { return (e >> 20) & 31u; }
+UW_HOST_DEVICE constexpr uint32_t lut_nsym(uint32_t e) { return lut_symbits(e) >> 2; }
+UW_HOST_DEVICE constexpr uint32_t lut_bits(uint32_t e) { return e >> 28; }
+constexpr uint32_t lut_entry(uint32_t syms, uint32_t nsym, uint32_t bits) {
+    return nsym ? syms | (4u * nsym) << 20 | bits << 28 : kLutInvalid | uint32_t(kLutBits) << 28;
+}
 
 uint32_t crc32(const void *data, size_t bytes, uint32_t crc = 0);
 uint32_t header_crc(const Header &h);

@@ -59,7 +59,7 @@ typedef enum uw_status {
 
 /* Human-readable name of a status code (static string). */
 const char *uw_status_str(int status);
-/* Library version string, e.g. "uw 1.0 (blob v1, sm_100a)". */
+/* Library version string, e.g. "uw 1.1 (blob v2, sm_100a)". */
 const char *uw_version(void);
 
 /* ------------------------------------------------------------------------ */
@@ -76,7 +76,10 @@ enum {
     UW_SEC_RAWBASE = 3,   /* uint32[] raw groups before word w of FLAGS (prefix count) */
     UW_SEC_STREAM = 4,    /* uint32[] Huffman bits, MSB of each word first, 0-padded   */
     UW_SEC_CHUNKOFF = 5,  /* uint32[n_chunks+1] start bit of each 4-group chunk        */
-    UW_SEC_DLUT = 6,      /* uint32[4096] 12-bit-window multi-symbol decode table      */
+    UW_SEC_DLUT = 6,      /* uint32[4096] 12-bit-window multi-symbol decode table:
+                             bits 0..19 up to 5 symbols (first lowest), bits 20..24
+                             4 x their count, bit 25 no code matches, bits 28..31
+                             stream bits they use (12 when none matches)        */
     UW_SEC_PAL = 7,       /* uint8[n*k/2] 4-bit palette indices: each little-endian
                              u32 word holds 8 consecutive weights; weight j's index v
                              has v&7 at bits 4j..4j+2 and v>>3 at bit 8j+7 (j<4) or

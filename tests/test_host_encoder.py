@@ -133,16 +133,37 @@ def test_decode_table_reproduces_oracle_symbols(uw):
         wi = p >> 5
         win = ((int(stream[wi]) << 32 | int(stream[wi + 1])) >> (64 - 12 - (p & 31))) & 0xFFF
         ent = int(lut[win])
-        cnt, nb, l0 = (ent >> 20) & 7, (ent >> 23) & 15, ent >> 27
-        assert cnt > 0
+        symbits, invalid, nb = (ent >> 20) & 31, (ent >> 25) & 1, ent >> 28
+        cnt = symbits // 4
+        assert cnt > 0 and symbits % 4 == 0 and not invalid and (ent >> 26) & 3 == 0
+        assert ent & 0xFFFFF < 1 << symbits
         if cnt <= total - len(got):
             got += [(ent >> (4 * j)) & 15 for j in range(cnt)]
             p += nb
         else:
-            got.append(ent & 15)
-            p += l0
+            s0 = ent & 15
+            got.append(s0)
+            p += int(info.code_len[s0])
     assert p == info.stream_bits
     assert np.array_equal(np.array(got), want)
+
+
+def test_decode_table_one_symbol_code(uw):
+    """With one palette symbol the code is the single bit 0: a window that
+    starts with z zero bits holds min(z, 5) codes in as many bits; windows
+    that start with 1 match no code, are marked invalid and skip the whole
+    12-bit window."""
+    rng = np.random.default_rng(5)
+    w = (0x3C80 | rng.integers(0, 1 << 7, (64, 256)) | (rng.integers(0, 2, (64, 256)) << 15)).astype(np.uint16)
+    blob = uw.encode(w)
+    info = uw.blob_info(blob)
+    assert info.palette_size == 1 and info.code_len[0] == 1
+    lut = uw.section(blob, uw.SEC_DLUT, info).view("<u4").astype(np.int64)
+    for v in range(2048):
+        cnt = min(5, 12 - v.bit_length())
+        assert lut[v] == (cnt << 28) | (4 * cnt << 20), v
+    assert np.all(lut[2048:] == (12 << 28) | (1 << 25))
+    assert info.stream_bits == 64 * 256
 
 
 # ------------------------------------------------------------------ fault injection (host)
