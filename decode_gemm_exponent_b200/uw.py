@@ -21,6 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("UW_LIBRARY") or os.path.join(_HERE, "libuw.so")
 
 UW_OK = 0
+ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CORRUPT, ERR_CUDA, ERR_NOMEM, ERR_TIMEOUT, ERR_WORKSPACE = range(1, 8)
 STATUS_NAMES = {0: "UW_OK", 1: "UW_ERR_INVALID_ARG", 2: "UW_ERR_UNSUPPORTED_SHAPE",
                 3: "UW_ERR_CORRUPT", 4: "UW_ERR_CUDA", 5: "UW_ERR_NOMEM", 6: "UW_ERR_TIMEOUT",
                 7: "UW_ERR_WORKSPACE"}
@@ -37,7 +38,7 @@ EXPORTS = ("uw_status_str", "uw_version", "uw_encode", "uw_blob_data", "uw_blob_
            "uw_blob_info_get", "uw_matrix_bind", "uw_device_status", "uw_decode_to_bf16",
            "uw_transcode_palette", "uw_plan_default", "uw_workspace_size", "uw_fused_matmul",
            "uw_matmul_bf16", "uw_autotune_workspace_size", "uw_plan_autotune",
-           "uw_fused_matmul_noalloc")
+           "uw_fused_matmul_noalloc", "uw_stack_workspace_size", "uw_stack_run")
 
 
 class UwError(RuntimeError):
@@ -82,6 +83,11 @@ class Plan(ctypes.Structure):
         return "Plan(%s)" % ", ".join("%s=%s" % kv for kv in self.as_dict().items())
 
 
+class StackStep(ctypes.Structure):
+    _fields_ = [("w", ctypes.POINTER(DMat)), ("x_dev", ctypes.c_void_p), ("m", ctypes.c_int64),
+                ("y_dev", ctypes.c_void_p), ("plan", Plan), ("pal_dev", ctypes.c_void_p)]
+
+
 def make_plan(pipeline=PIPE_DIRECT_PALETTE, kernel=KERNEL_TC, bn=16, split_k=1, stages=0,
               debug_flags=0, timeout_ns=0) -> Plan:
     return Plan(pipeline, kernel, bn, split_k, stages, debug_flags, timeout_ns)
@@ -117,6 +123,8 @@ def lib() -> ctypes.CDLL:
                                            P, SZ, P]),
         "uw_matmul_bf16": (ctypes.c_int, [P, I64, P, I64, I64, P, ctypes.POINTER(Plan), P, SZ, P, P]),
         "uw_fused_matmul_noalloc": (ctypes.c_int, [P, I64, ctypes.POINTER(DMat), P, ctypes.POINTER(Plan), P]),
+        "uw_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, ctypes.POINTER(SZ)]),
+        "uw_stack_run": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, P, SZ, P, P]),
         "uw_autotune_workspace_size": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(DMat)), ctypes.c_int,
                                                       ctypes.POINTER(I64), ctypes.c_int,
                                                       ctypes.POINTER(SZ)]),
@@ -254,6 +262,40 @@ def fused_matmul_noalloc(mat: "Matrix", x, plan: Plan, y=None, stream=None):
     check(lib().uw_fused_matmul_noalloc(_ptr(x), m, ctypes.byref(mat.dmat), _ptr(y), ctypes.byref(plan),
                                         _stream_handle(stream)), "uw_fused_matmul_noalloc")
     return y
+
+
+class Stack:
+    """A fixed sequence of matmuls run by uw_stack_run: matmuls in order on the
+    main stream, decodes / transcodes of pipeline-1 / pipeline-3 steps on a
+    side stream ahead of their matmuls (cross-layer overlap).
+
+    steps: (Matrix, x, y, plan) tuples, or (Matrix, x, y, plan, pal) for a
+    pipeline-4 step with its own palette plane.  The tensors are kept alive
+    by this object; the workspace is allocated once here."""
+
+    def __init__(self, steps):
+        import torch
+        self.keep = list(steps)
+        arr = (StackStep * len(steps))()
+        for i, st in enumerate(steps):
+            mat, x, y, plan = st[:4]
+            pal = st[4] if len(st) > 4 else None
+            if x.shape[1] != mat.k or y.shape != (x.shape[0], mat.n):
+                raise ValueError("step %d: shapes do not match the matrix" % i)
+            arr[i] = StackStep(ctypes.pointer(mat.dmat), x.data_ptr(), x.shape[0], y.data_ptr(), plan,
+                               pal.data_ptr() if pal is not None else None)
+        self.steps = arr
+        size = ctypes.c_size_t()
+        check(lib().uw_stack_workspace_size(arr, len(steps), ctypes.byref(size)), "uw_stack_workspace_size")
+        self.ws_bytes = int(size.value)
+        dev = steps[0][1].device
+        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def run(self, stream=None, side_stream=None):
+        """Issue the whole stack; side_stream=None runs everything on `stream`."""
+        side = ctypes.c_void_p(side_stream.cuda_stream) if side_stream is not None else ctypes.c_void_p(0)
+        check(lib().uw_stack_run(self.steps, len(self.steps), _ptr(self.ws), self.ws.numel(),
+                                 _stream_handle(stream), side), "uw_stack_run")
 
 
 def workspace_size(m: int, n: int, k: int, plan: Plan) -> int:

@@ -274,6 +274,39 @@ uw_status uw_plan_autotune(const uw_dmat *const *mats, int n_mats, const int64_t
                            size_t ws_bytes, int reps, uw_plan *plans_out, char *json_out,
                            size_t json_cap, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* Layer stacks with cross-layer overlap (Unweight page §八).                 */
+
+/* One matmul of a stack: y_dev[m, w->n] = x_dev[m, w->k] * W^T with `plan`
+ * (any pipeline).  pal_dev as in uw_fused_matmul (pipeline 4 only).        */
+typedef struct uw_stack_step {
+    const uw_dmat *w;
+    const uint16_t *x_dev;
+    int64_t m;
+    float *y_dev;
+    uw_plan plan;
+    const uint8_t *pal_dev;
+} uw_stack_step;
+
+/* Workspace of uw_stack_run: two preprocessing slots, each the largest
+ * decode (2nk bytes) or transcode (nk/2 bytes) buffer of the stack, plus the
+ * largest split-K scratch of any step.                                       */
+uw_status uw_stack_workspace_size(const uw_stack_step *steps, int n_steps, size_t *bytes);
+
+/* Run the steps in order on `stream`.  The decode (pipeline 1) or transcode
+ * (pipeline 3) of a step is issued on `side_stream` into one of the two
+ * workspace slots as soon as that slot is free, so it overlaps the matmuls
+ * of the steps before it; the step's matmul waits for it.  Each step's result
+ * is bit-identical to uw_fused_matmul with the same plan.  A step may read
+ * an earlier step's y (matmuls keep step order on `stream`); no step may
+ * write any weights.  side_stream NULL or equal to `stream`: everything runs
+ * on `stream`.  All work, side stream included, is complete once `stream`
+ * has completed it.  ws: >= uw_stack_workspace_size bytes, 256-byte aligned.
+ * Arguments are checked before anything is launched; errors as in
+ * uw_fused_matmul.  Device errors are OR-ed into each matrix's dev_status. */
+uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void *ws, size_t ws_bytes,
+                       void *stream, void *side_stream);
+
 #ifdef __cplusplus
 }
 #endif

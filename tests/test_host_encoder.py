@@ -236,3 +236,40 @@ def test_plans_and_workspace(uw):
             uw.workspace_size(4, n, k, bad)
     with pytest.raises(uw.UwError):
         uw.workspace_size(16, n, k, uw.make_plan(kernel=uw.KERNEL_FMA, bn=1))   # FMA needs m <= 8
+
+
+def test_stack_workspace_and_argument_checks(uw):
+    """uw_stack_workspace_size / uw_stack_run host logic.  The matrix is bound
+    to a device address that is never dereferenced (binding reads only the
+    host copy), and every uw_stack_run call here fails its argument checks,
+    which come before any launch."""
+    w = synth.weights_bf16(128, 256, 0.02, 0.002, 1.0, seed=3)
+    host = np.frombuffer(uw.encode(w), np.uint8)
+    fake = 1 << 40
+    dm = uw.DMat()
+    uw.check(uw.lib().uw_matrix_bind(host.ctypes.data, host.size, fake, fake, 0, ctypes.byref(dm)),
+             "uw_matrix_bind")
+    n, k = 128, 256
+    plans = [uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 64, 4),
+             uw.make_plan(uw.PIPE_TRANSCODE_FUSED, uw.KERNEL_FMA, 1, 1),
+             uw.make_plan(uw.PIPE_DECODE_GEMM, uw.KERNEL_TC, 16, 2)]
+    ms = [64, 1, 16]
+    steps = (uw.StackStep * 3)()
+    for i, (p, m) in enumerate(zip(plans, ms)):
+        steps[i] = uw.StackStep(ctypes.pointer(dm), fake, m, fake, p, None)
+    size = ctypes.c_size_t()
+    assert uw.lib().uw_stack_workspace_size(steps, 3, ctypes.byref(size)) == 0
+    slot = max(2 * n * k, n * k // 2)                      # decode buffer is the larger
+    partial = max(4 * 64 * n * 4, 2 * 16 * n * 4)         # split-K scratch, reused by every step
+    assert size.value == 2 * slot + partial
+    run = uw.lib().uw_stack_run
+    assert run(steps, 3, None, 0, None, None) == uw.ERR_WORKSPACE
+    assert run(steps, 3, fake + 1, size.value, None, None) == uw.ERR_WORKSPACE   # misaligned
+    assert run(steps, 3, fake, size.value - 1, None, None) == uw.ERR_WORKSPACE
+    assert run(steps, 0, fake, size.value, None, None) == uw.ERR_INVALID_ARG
+    bad = (uw.StackStep * 3)(*steps)
+    bad[1].x_dev = None
+    assert run(bad, 3, fake, size.value, None, None) == uw.ERR_INVALID_ARG
+    bad = (uw.StackStep * 3)(*steps)
+    bad[2].plan.bn = 24                                   # not a tcgen05 token tile
+    assert uw.lib().uw_stack_workspace_size(bad, 3, ctypes.byref(size)) == uw.ERR_INVALID_ARG
