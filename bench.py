@@ -229,7 +229,7 @@ def plans_from_json(text, n_mats, uw):
     for e in doc["plans"]:
         b = e["best"]
         plans[e["matrix"]][MS.index(e["m"])] = uw.make_plan(
-            pipes[b["pipeline"]], 1 if b["kernel"] == "fma" else 2, b["bn"], b["split_k"])
+            pipes[b["pipeline"]], {"fma": 1, "tc": 2, "mma": 3}[b["kernel"]], b["bn"], b["split_k"])
     return plans
 
 
@@ -241,7 +241,7 @@ def launches_per_call(plan):
 
 
 def kernel_group(plan):
-    kern = "fma_gemv" if plan.kernel == 1 else "tcgen05_bn%d" % plan.bn
+    kern = {1: "fma_gemv", 3: "mma_gemv_s%d" % plan.bn}.get(plan.kernel, "tcgen05_bn%d" % plan.bn)
     pipe = {1: "decode+plain", 3: "transcode+fused", 4: "fused"}[plan.pipeline]
     return "%s/%s" % (pipe, kern)
 

@@ -4,8 +4,9 @@
 //
 // For each matrix and each batch size m the candidates are the pipelines the
 // blob supports (decode + plain kernel, runtime transcode + fused kernel,
-// direct palette + fused kernel) crossed with the kernel variants: the FMA
-// GEMV (m <= 8, 1 or 2 rows per warp) and the tcgen05 kernel with token tiles
+// direct palette + fused kernel) crossed with the kernel variants: the
+// warp-MMA kernel (m <= 16, 1-8 K slices per tile), the FMA GEMV (m <= 8, 1
+// or 2 rows per warp) and the tcgen05 kernel with token tiles
 // around m and split-K factors that fill the 148 SMs.  Each candidate is run
 // once to warm up (its status is checked) and then `reps` times between CUDA
 // events; the fastest average wins.
@@ -31,6 +32,15 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
     if ((w.flags & UW_EMIT_PALETTE) && w.pal) pipes.push_back(UW_PIPE_DIRECT_PALETTE);
     std::vector<uw_plan> out;
     for (int pipe : pipes) {
+        if (m <= 16)
+            for (int slices : {1, 2, 4, 8}) {
+                uw_plan p{};
+                p.pipeline = pipe;
+                p.kernel = UW_KERNEL_MMA;
+                p.bn = slices;
+                p.split_k = 1;
+                out.push_back(p);
+            }
         if (m <= 8)
             for (int rows : {1, 2}) {
                 uw_plan p{};
@@ -70,7 +80,8 @@ std::string plan_json(const uw_plan &p, double us) {
     char buf[256];
     std::snprintf(buf, sizeof buf,
                   "{\"pipeline\": \"%s\", \"kernel\": \"%s\", \"bn\": %d, \"split_k\": %d, \"us\": %.3f}",
-                  pipe_name(p.pipeline), p.kernel == UW_KERNEL_FMA ? "fma" : "tc", p.bn, p.split_k, us);
+                  pipe_name(p.pipeline), p.kernel == UW_KERNEL_FMA ? "fma" : p.kernel == UW_KERNEL_MMA ? "mma" : "tc",
+                  p.bn, p.split_k, us);
     return buf;
 }
 

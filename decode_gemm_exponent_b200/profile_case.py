@@ -22,11 +22,11 @@ from . import synth, uw
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", required=True,
-                    choices=["decode", "transcode", "fma", "tc", "plain_fma", "plain_tc"])
+                    choices=["decode", "transcode", "fma", "tc", "mma", "plain_fma", "plain_tc", "plain_mma"])
     ap.add_argument("--n", type=int, default=28672)
     ap.add_argument("--k", type=int, default=8192)
     ap.add_argument("--m", type=int, default=1)
-    ap.add_argument("--bn", type=int, default=0, help="TC token tile or FMA rows per warp")
+    ap.add_argument("--bn", type=int, default=0, help="TC token tile, FMA rows per warp or MMA K slices")
     ap.add_argument("--split", type=int, default=1)
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--sigma", type=float, default=0.015)
@@ -48,6 +48,8 @@ def main(argv=None):
     flops = 2.0 * a.m * nk
     if a.kernel in ("fma", "plain_fma"):
         plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_FMA, a.bn or 1, 1)
+    elif a.kernel in ("mma", "plain_mma"):
+        plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, a.bn or 2, 1)
     else:
         plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, a.bn or 16, a.split, a.stages)
     ws_bytes = uw.workspace_size(a.m, a.n, a.k, plan) if a.kernel not in ("decode", "transcode") else 0
@@ -61,7 +63,7 @@ def main(argv=None):
         out = torch.empty(nk // 2, dtype=torch.uint8, device="cuda")
         run = lambda: mat.transcode(out)
         alg = huff_in + nk // 2
-    elif a.kernel in ("fma", "tc"):
+    elif a.kernel in ("fma", "tc", "mma"):
         run = lambda: mat.matmul(x, plan, y=y, ws=ws)
         alg = common + nk // 2 + xy
     else:

@@ -30,7 +30,7 @@ EMIT_PALETTE = 2
 SEC_SM, SEC_RAWEXP, SEC_FLAGS, SEC_RAWBASE, SEC_STREAM, SEC_CHUNKOFF, SEC_DLUT, SEC_PAL = range(8)
 NUM_SECTIONS = 8
 PIPE_DECODE_GEMM, PIPE_TRANSCODE_FUSED, PIPE_DIRECT_PALETTE = 1, 3, 4
-KERNEL_FMA, KERNEL_TC = 1, 2
+KERNEL_FMA, KERNEL_TC, KERNEL_MMA = 1, 2, 3
 DEBUG_NEVER_ARRIVE = 1
 
 # every symbol include/uw.h declares

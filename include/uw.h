@@ -189,7 +189,10 @@ typedef enum uw_pipeline {
 
 typedef enum uw_kernel {
     UW_KERNEL_FMA = 1,   /* CUDA-core FMA GEMV, one warp per `bn` rows, m <= 8       */
-    UW_KERNEL_TC = 2     /* tcgen05 MMA with a TMEM accumulator, token tile `bn`      */
+    UW_KERNEL_TC = 2,    /* tcgen05 MMA with a TMEM accumulator, token tile `bn`      */
+    UW_KERNEL_MMA = 3    /* m <= 16: W rebuilt in registers straight into warp-level
+                            MMA fragments; 8 rows of W per warp, `bn` warps per CTA
+                            split K and are summed in a fixed order              */
 } uw_kernel;
 
 #define UW_DEBUG_NEVER_ARRIVE 1u   /* TC kernel: wait on a barrier nobody signals, so
@@ -199,9 +202,10 @@ typedef struct uw_plan {
     int32_t pipeline;     /* uw_pipeline */
     int32_t kernel;       /* uw_kernel */
     int32_t bn;           /* TC: tokens per tile, one of 16,32,64,128,256;
-                             FMA: weight rows per warp, 1 or 2 */
+                             FMA: weight rows per warp, 1 or 2;
+                             MMA: K slices (warps) per 8-row tile, 1..8 */
     int32_t split_k;      /* TC: K split into this many slices (>= 1), reduced in a
-                             fixed order; FMA: must be 1 */
+                             fixed order; FMA, MMA: must be 1 */
     int32_t stages;       /* TC: shared-memory ring depth (0 = largest that fits) */
     uint32_t debug_flags; /* UW_DEBUG_* (0 in production) */
     int64_t timeout_ns;   /* spin-wait limit inside kernels (0 = 2 s) */

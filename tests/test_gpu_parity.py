@@ -126,6 +126,20 @@ def test_fma_gemv_parity(uw, m, rows):
     _matmul_case(uw, 320, 1600, m, dict(kernel=uw.KERNEL_FMA, bn=rows, split_k=1), seed=m)
 
 
+@pytest.mark.parametrize("m", [1, 2, 3, 7, 8, 9, 12, 16])
+@pytest.mark.parametrize("slices", [1, 2, 3, 8])
+def test_mma_gemv_parity(uw, m, slices):
+    # k = 1600 = 25 chunks: uneven K slices; n = 320 = 40 tiles of 8 rows
+    _matmul_case(uw, 320, 1600, m, dict(kernel=uw.KERNEL_MMA, bn=slices, split_k=1), seed=100 + m)
+
+
+def test_mma_gemv_raw_heavy_and_long_k(uw):
+    # 5% outliers: most groups raw; k = 14336 (224 chunks per row, bitmap
+    # words of a tile not aligned to rows)
+    _matmul_case(uw, 64, 704, 5, dict(kernel=uw.KERNEL_MMA, bn=2, split_k=1), seed=4, frac=0.05)
+    _matmul_case(uw, 128, 14336, 16, dict(kernel=uw.KERNEL_MMA, bn=4, split_k=1), seed=5, frac=0.001)
+
+
 @pytest.mark.parametrize("bn,m", [(16, 1), (16, 16), (32, 20), (64, 64), (64, 100), (128, 128),
                                   (128, 300), (256, 256), (256, 513)])
 def test_tc_gemm_parity(uw, bn, m):
@@ -151,6 +165,8 @@ def test_tc_stage_depth_does_not_change_bits(uw):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("m,plan_kw", [(1, dict(kernel=1, bn=1, split_k=1)),
+                                       (1, dict(kernel=3, bn=2, split_k=1)),
+                                       (16, dict(kernel=3, bn=4, split_k=1)),
                                        (16, dict(kernel=2, bn=16, split_k=4)),
                                        (64, dict(kernel=2, bn=64, split_k=2)),
                                        (1024, dict(kernel=2, bn=256, split_k=1))])
