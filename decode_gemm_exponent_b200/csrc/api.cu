@@ -20,8 +20,8 @@ inline uw_status cuda_status(cudaError_t e) { return e == cudaSuccess ? UW_OK : 
 
 bool valid_bn_tc(int bn) { return bn == 16 || bn == 32 || bn == 64 || bn == 128 || bn == 256; }
 
-uw_status check_plan(const uw_plan *p, int64_t m) {
-    if (!p) return UW_ERR_INVALID_ARG;
+uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
+    if (!p || k <= 0) return UW_ERR_INVALID_ARG;
     if (p->pipeline != UW_PIPE_DECODE_GEMM && p->pipeline != UW_PIPE_TRANSCODE_FUSED &&
         p->pipeline != UW_PIPE_DIRECT_PALETTE)
         return UW_ERR_INVALID_ARG;
@@ -196,7 +196,7 @@ extern "C" uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pi
 extern "C" uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw_plan *plan,
                                        size_t *bytes) {
     if (!bytes || m <= 0 || n <= 0 || k <= 0) return UW_ERR_INVALID_ARG;
-    uw_status st = check_plan(plan, m);
+    uw_status st = check_plan(plan, m, k);
     if (st != UW_OK) return st;
     *bytes = size_t(prep_bytes(n, k, plan) + partial_bytes(m, n, plan));
     return UW_OK;
@@ -209,7 +209,7 @@ extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_
     if (st != UW_OK) return st;
     if (!x_dev || !y_dev || m <= 0) return UW_ERR_INVALID_ARG;
     if (!aligned(x_dev, 16) || !aligned(y_dev, 16)) return UW_ERR_INVALID_ARG;
-    st = check_plan(plan, m);
+    st = check_plan(plan, m, w->k);
     if (st != UW_OK) return st;
     const uint64_t need_prep = prep_bytes(w->n, w->k, plan), need_part = partial_bytes(m, w->n, plan);
     if (need_prep + need_part > 0 && (!ws || ws_bytes < need_prep + need_part || !aligned(ws, 256)))
@@ -245,7 +245,7 @@ extern "C" uw_status uw_matmul_bf16(const uint16_t *x_dev, int64_t m, const uint
     if (!x_dev || !w_dev || !y_dev || m <= 0 || n <= 0 || k <= 0) return UW_ERR_INVALID_ARG;
     if (n % 64 || k % 64) return UW_ERR_UNSUPPORTED_SHAPE;
     if (!aligned(x_dev, 16) || !aligned(w_dev, 16) || !aligned(y_dev, 16)) return UW_ERR_INVALID_ARG;
-    uw_status st = check_plan(plan, m);
+    uw_status st = check_plan(plan, m, k);
     if (st != UW_OK) return st;
     const uint64_t need = partial_bytes(m, n, plan);
     if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 256))) return UW_ERR_WORKSPACE;

@@ -191,8 +191,8 @@ typedef enum uw_kernel {
     UW_KERNEL_FMA = 1,   /* CUDA-core FMA GEMV, one warp per `bn` rows, m <= 8       */
     UW_KERNEL_TC = 2,    /* tcgen05 MMA with a TMEM accumulator, token tile `bn`      */
     UW_KERNEL_MMA = 3    /* m <= 16: W rebuilt in registers straight into warp-level
-                            MMA fragments; 8 rows of W per warp, `bn` warps per CTA
-                            split K and are summed in a fixed order              */
+                            MMA fragments; one CTA per 16-row tile, whose `bn`
+                            warps split K (summed in a fixed order)               */
 } uw_kernel;
 
 #define UW_DEBUG_NEVER_ARRIVE 1u   /* TC kernel: wait on a barrier nobody signals, so
@@ -203,7 +203,7 @@ typedef struct uw_plan {
     int32_t kernel;       /* uw_kernel */
     int32_t bn;           /* TC: tokens per tile, one of 16,32,64,128,256;
                              FMA: weight rows per warp, 1 or 2;
-                             MMA: K slices (warps) per 8-row tile, 1..8 */
+                             MMA: warps per CTA = K slices per 16-row tile, 1..8 */
     int32_t split_k;      /* TC: K split into this many slices (>= 1), reduced in a
                              fixed order; FMA, MMA: must be 1 */
     int32_t stages;       /* TC: shared-memory ring depth (0 = largest that fits) */
@@ -266,11 +266,15 @@ uw_status uw_fused_matmul_noalloc(const uint16_t *x_dev, int64_t m, const uw_dma
 
 /* For every matrix mats[i] and batch size ms[j], time the candidate
  * (pipeline, kernel, bn, split_k) plans with CUDA events on `stream` and
- * store the fastest in plans_out[i*n_ms + j].  x_dev must hold at least
- * max(ms) x max(k) BF16 values, y_dev max(ms) x max(n) floats, and ws at least
- * the largest uw_workspace_size of any candidate (uw_autotune_workspace_size).
- * If json_out is non-NULL a JSON plan file (per matrix, per m: the chosen plan
- * and the measured microseconds of every candidate) is written into it.     */
+ * store the fastest in plans_out[i*n_ms + j].  Every timed call is preceded
+ * by a 192 MB read of the end of the workspace, so the weights come from HBM
+ * (not from the 126 MB L2), as they do when a model's layers run in turn.
+ * x_dev must hold at least max(ms) x max(k) BF16 values, y_dev max(ms) x
+ * max(n) floats, and ws (256-byte aligned) at least
+ * uw_autotune_workspace_size bytes: the largest uw_workspace_size of any
+ * candidate plus the 192 MB scratch.  If json_out is non-NULL a JSON plan
+ * file (per matrix, per m: the chosen plan and the measured microseconds of
+ * every candidate) is written into it.                                      */
 uw_status uw_autotune_workspace_size(const uw_dmat *const *mats, int n_mats,
                                      const int64_t *ms, int n_ms, size_t *bytes);
 uw_status uw_plan_autotune(const uw_dmat *const *mats, int n_mats, const int64_t *ms,

@@ -129,8 +129,13 @@ def test_fma_gemv_parity(uw, m, rows):
 @pytest.mark.parametrize("m", [1, 2, 3, 7, 8, 9, 12, 16])
 @pytest.mark.parametrize("slices", [1, 2, 3, 8])
 def test_mma_gemv_parity(uw, m, slices):
-    # k = 1600 = 25 chunks: uneven K slices; n = 320 = 40 tiles of 8 rows
+    # k = 1600 = 25 chunks: uneven K slices; n = 320 = 20 tiles of 16 rows
     _matmul_case(uw, 320, 1600, m, dict(kernel=uw.KERNEL_MMA, bn=slices, split_k=1), seed=100 + m)
+
+
+def test_mma_gemv_many_tiles(uw):
+    _matmul_case(uw, 4096, 512, 3, dict(kernel=uw.KERNEL_MMA, bn=4, split_k=1), seed=77, pipelines=(4,))
+    _matmul_case(uw, 4096, 512, 11, dict(kernel=uw.KERNEL_MMA, bn=8, split_k=1), seed=78, pipelines=(4,))
 
 
 def test_mma_gemv_raw_heavy_and_long_k(uw):
@@ -229,7 +234,7 @@ def test_autotune_returns_valid_plans(uw):
     assert len(doc["plans"]) == 4
     for row in plans:
         for p in row:
-            assert p.kernel in (1, 2) and p.pipeline in (1, 3, 4)
+            assert p.kernel in (1, 2, 3) and p.pipeline in (1, 3, 4)
     # the chosen plan reproduces the plain kernel bit for bit
     w = synth.weights_bf16(512, 1024, 0.02, 0.001, 1.0, seed=20)
     x = synth.activations_bf16(64, 1024, seed=20)

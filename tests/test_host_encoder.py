@@ -238,7 +238,7 @@ def test_plans_and_workspace(uw):
         uw.workspace_size(16, n, k, uw.make_plan(kernel=uw.KERNEL_FMA, bn=1))   # FMA needs m <= 8
     for slices in (1, 2, 4, 8):
         assert uw.workspace_size(16, n, k, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, slices)) == 0
-    for bad_m, bad in ((17, uw.make_plan(kernel=uw.KERNEL_MMA, bn=1)),           # MMA needs m <= 16
+    for bad_m, bad in ((17, uw.make_plan(kernel=uw.KERNEL_MMA, bn=1)),     # MMA needs m <= 16
                        (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=0)),
                        (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=9)),
                        (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, split_k=2))):
