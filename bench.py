@@ -229,7 +229,8 @@ def plans_from_json(text, n_mats, uw):
     for e in doc["plans"]:
         b = e["best"]
         plans[e["matrix"]][MS.index(e["m"])] = uw.make_plan(
-            pipes[b["pipeline"]], {"fma": 1, "tc": 2, "mma": 3}[b["kernel"]], b["bn"], b["split_k"])
+            pipes[b["pipeline"]], {"fma": 1, "tc": 2, "mma": 3}[b["kernel"]], b["bn"], b["split_k"],
+            b.get("stages", 0))
     return plans
 
 
@@ -241,7 +242,7 @@ def launches_per_call(plan):
 
 
 def kernel_group(plan):
-    kern = {1: "fma_gemv", 3: "mma_gemv_s%d" % plan.bn}.get(plan.kernel, "tcgen05_bn%d" % plan.bn)
+    kern = {1: "fma_gemv", 3: "mma_gemv_s%d_w%d" % (plan.bn, plan.stages)}.get(plan.kernel, "tcgen05_bn%d" % plan.bn)
     pipe = {1: "decode+plain", 3: "transcode+fused", 4: "fused"}[plan.pipeline]
     return "%s/%s" % (pipe, kern)
 

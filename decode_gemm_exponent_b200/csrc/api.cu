@@ -29,6 +29,7 @@ uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
         if (m > 8 || (p->bn != 1 && p->bn != 2) || p->split_k != 1) return UW_ERR_INVALID_ARG;
     } else if (p->kernel == UW_KERNEL_MMA) {
         if (m > 16 || p->bn < 1 || p->bn > 8 || p->split_k != 1) return UW_ERR_INVALID_ARG;
+        if (p->stages < 0 || p->stages > 2 || (p->stages == 2 && k % 128)) return UW_ERR_INVALID_ARG;
     } else if (p->kernel == UW_KERNEL_TC) {
         if (!valid_bn_tc(p->bn) || p->split_k < 1 || p->split_k > 64 || p->stages < 0 || p->stages > 8)
             return UW_ERR_INVALID_ARG;
@@ -57,7 +58,7 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
     if (plan->kernel == UW_KERNEL_FMA)
         return cuda_status(launch_gemv_fma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, status, stream));
     if (plan->kernel == UW_KERNEL_MMA)
-        return cuda_status(launch_gemv_mma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, stream));
+        return cuda_status(launch_gemv_mma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, plan->stages, stream));
     TcLaunch t{};
     t.x = x;
     t.m = m;

@@ -5,7 +5,8 @@
 // For each matrix and each batch size m the candidates are the pipelines the
 // blob supports (decode + plain kernel, runtime transcode + fused kernel,
 // direct palette + fused kernel) crossed with the kernel variants: the
-// warp-MMA kernel (m <= 16, 2-8 K slices per tile), the FMA GEMV (m <= 8, 1
+// warp-MMA kernel (m <= 16, 2-8 K slices per tile, 16 or 32 weights per
+// lane and step), the FMA GEMV (m <= 8, 1
 // or 2 rows per warp) and the tcgen05 kernel with token tiles
 // around m and split-K factors that fill the 148 SMs.  Each candidate is run
 // once to warm up (its status is checked) and then `reps` times between CUDA
@@ -44,13 +45,17 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
     std::vector<uw_plan> out;
     for (int pipe : pipes) {
         if (m <= 16)
-            for (int slices : {2, 4, 8}) {
-                uw_plan p{};
-                p.pipeline = pipe;
-                p.kernel = UW_KERNEL_MMA;
-                p.bn = slices;
-                p.split_k = 1;
-                out.push_back(p);
+            for (int width : {1, 2}) {
+                if (width == 2 && w.k % 128) continue;
+                for (int slices : {2, 4, 8}) {
+                    uw_plan p{};
+                    p.pipeline = pipe;
+                    p.kernel = UW_KERNEL_MMA;
+                    p.bn = slices;
+                    p.split_k = 1;
+                    p.stages = width;
+                    out.push_back(p);
+                }
             }
         if (m <= 8)
             for (int rows : {1, 2}) {
@@ -90,9 +95,10 @@ const char *pipe_name(int p) {
 std::string plan_json(const uw_plan &p, double us) {
     char buf[256];
     std::snprintf(buf, sizeof buf,
-                  "{\"pipeline\": \"%s\", \"kernel\": \"%s\", \"bn\": %d, \"split_k\": %d, \"us\": %.3f}",
+                  "{\"pipeline\": \"%s\", \"kernel\": \"%s\", \"bn\": %d, \"split_k\": %d, \"stages\": %d, "
+                  "\"us\": %.3f}",
                   pipe_name(p.pipeline), p.kernel == UW_KERNEL_FMA ? "fma" : p.kernel == UW_KERNEL_MMA ? "mma" : "tc",
-                  p.bn, p.split_k, us);
+                  p.bn, p.split_k, p.stages, us);
     return buf;
 }
 

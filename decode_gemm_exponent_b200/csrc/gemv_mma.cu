@@ -43,7 +43,6 @@ using namespace dev;
 
 constexpr int kTileRows = 16;
 constexpr int kChunk = 64;
-constexpr int kStages = 3;
 constexpr int kMaxSlices = 8;
 constexpr int kMaxSmem = 48 * 1024;    // dynamic shared memory without opt-in
 
@@ -62,10 +61,14 @@ struct MmaArgs {
     float *y;                  // [m, n]
 };
 
-// one lane's 16 weights of one chunk of one row, as loaded
+// One lane's 16*Q weights of one chunk (64*Q weights along K) of one row, as
+// loaded.  Plain: the weights, 16*Q BF16 in a[] then b[].  Fused: sign/mantissa
+// bytes in a[]; the palette words (2*Q of them) in b[0], or the raw
+// exponents (16*Q bytes) in b[].
+template <int Q>
 struct Half {
-    uint4 a;       // plain: weights 0..7; fused: sign/mantissa bytes
-    uint4 b;       // plain: weights 8..15; fused: palette words (.x, .y) or raw exponents
+    uint4 a[Q];
+    uint4 b[Q];
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -92,54 +95,71 @@ __device__ __forceinline__ uint64_t raw_window(const uint32_t *sflags, int nword
     return sh ? (lo | hi) : (uint64_t(v[1]) << 32 | v[0]);
 }
 
-template <bool PAL>
-__device__ __forceinline__ Half load_half(const MmaArgs &a, const uint8_t *smp, const uint32_t *palp,
-                                          const uint16_t *wp, bool raw, int64_t g, const uint32_t *sflags,
-                                          const uint32_t *srb, int64_t wbase, int c) {
-    Half h;
+// loads of one lane's weights of one chunk of one row; `g` is the lane's
+// group, `goff` the lane's byte offset inside that group's 64 raw exponents
+template <bool PAL, int Q>
+__device__ __forceinline__ Half<Q> load_half(const MmaArgs &a, const uint8_t *smp, const uint32_t *palp,
+                                             const uint16_t *wp, bool raw, int64_t g, int goff,
+                                             const uint32_t *sflags, const uint32_t *srb, int64_t wbase) {
+    Half<Q> h;
     if (!PAL) {
-        h.a = __ldcs(reinterpret_cast<const uint4 *>(wp));
-        h.b = __ldcs(reinterpret_cast<const uint4 *>(wp) + 1);
+        const uint4 *u = reinterpret_cast<const uint4 *>(wp);
+#pragma unroll
+        for (int i = 0; i < Q; i++) {
+            h.a[i] = __ldcs(u + i);
+            h.b[i] = __ldcs(u + Q + i);
+        }
     } else {
-        h.a = __ldcs(reinterpret_cast<const uint4 *>(smp));
+#pragma unroll
+        for (int i = 0; i < Q; i++) h.a[i] = __ldcs(reinterpret_cast<const uint4 *>(smp) + i);
         if (raw) {
             const int wi = int((g >> 5) - wbase);
             const uint32_t rank = srb[wi] + __popc(sflags[wi] & ((1u << (uint32_t(g) & 31u)) - 1u));
-            h.b = __ldcs(reinterpret_cast<const uint4 *>(a.rawexp + uint64_t(rank) * kGroup + c * 16));
-        } else {
+            const uint4 *e = reinterpret_cast<const uint4 *>(a.rawexp + uint64_t(rank) * kGroup + goff);
+#pragma unroll
+            for (int i = 0; i < Q; i++) h.b[i] = __ldcs(e + i);
+        } else if (Q == 1) {
             const uint2 p = __ldcs(reinterpret_cast<const uint2 *>(palp));
-            h.b = make_uint4(p.x, p.y, 0u, 0u);
+            h.b[0] = make_uint4(p.x, p.y, 0u, 0u);
+        } else {
+            h.b[0] = __ldcs(reinterpret_cast<const uint4 *>(palp));
+#pragma unroll
+            for (int i = 1; i < Q; i++) h.b[i] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
     return h;
 }
 
-// Half -> 8 BF16 pairs (weights 2i, 2i+1 in pair i)
-template <bool PAL>
-__device__ __forceinline__ void rebuild(const Half &h, bool raw, const Palette16 &P, uint32_t (&w)[8]) {
+__device__ __forceinline__ uint32_t word(const uint4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// Half -> 8*Q BF16 pairs (weights 2i, 2i+1 in pair i)
+template <bool PAL, int Q>
+__device__ __forceinline__ void rebuild(const Half<Q> &h, bool raw, const Palette16 &P, uint32_t (&w)[8 * Q]) {
     if (!PAL) {
-        w[0] = h.a.x; w[1] = h.a.y; w[2] = h.a.z; w[3] = h.a.w;
-        w[4] = h.b.x; w[5] = h.b.y; w[6] = h.b.z; w[7] = h.b.w;
+#pragma unroll
+        for (int i = 0; i < 4 * Q; i++) w[i] = word(h.a[i / 4], i % 4);
+#pragma unroll
+        for (int i = 0; i < 4 * Q; i++) w[4 * Q + i] = word(h.b[i / 4], i % 4);
     } else {
-        uint32_t r0, r1, r2, r3;
+        uint32_t r[4 * Q];   // rotated exponent bytes, 4 weights per word
         if (raw) {
-            r0 = rot4(h.b.x);
-            r1 = rot4(h.b.y);
-            r2 = rot4(h.b.z);
-            r3 = rot4(h.b.w);
+#pragma unroll
+            for (int i = 0; i < 4 * Q; i++) r[i] = rot4(word(h.b[i / 4], i % 4));
         } else {
-            pal_rot(h.b.x, P, r0, r1);
-            pal_rot(h.b.y, P, r2, r3);
+#pragma unroll
+            for (int i = 0; i < 2 * Q; i++) pal_rot(word(h.b[0], i), P, r[2 * i], r[2 * i + 1]);
         }
-        join4(r0, h.a.x, w[0], w[1]);
-        join4(r1, h.a.y, w[2], w[3]);
-        join4(r2, h.a.z, w[4], w[5]);
-        join4(r3, h.a.w, w[6], w[7]);
+#pragma unroll
+        for (int i = 0; i < 4 * Q; i++) join4(r[i], word(h.a[i / 4], i % 4), w[2 * i], w[2 * i + 1]);
     }
 }
 
-template <bool PAL, int NT>   // NT: 8-token tiles (1: m <= 8, 2: m <= 16)
+template <bool PAL, int NT, int Q>   // NT: 8-token tiles (1: m <= 8, 2: m <= 16); Q: 16*Q weights per lane and row
 __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
+    constexpr int kCh = kChunk * Q;               // weights per chunk along K
+    constexpr int kWl = 16 * Q;                   // weights per lane and row in a chunk
+    constexpr int kStages = Q == 1 ? 3 : 2;       // chunks of loads in flight per warp
+    constexpr int kWin = 64 / Q;                  // chunks per 64-group window of raw bits
     // dynamic shared memory: [bitmap words][prefix counts] (fused), then the
     // slice results [slices][32][8 * NT] (slices > 1)
     extern __shared__ __align__(16) uint32_t smem[];
@@ -150,7 +170,8 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
     const int g = lane >> 2, c = lane & 3;
     const int64_t row0 = int64_t(blockIdx.x) * kTileRows;
     const int64_t ra = row0 + g, rb = ra + 8;       // this lane's two rows
-    const int64_t gpr = a.k / kChunk;               // groups (chunks) per row
+    const int64_t gpr = a.k / kChunk;               // groups per row
+    const int64_t cpr = a.k / kCh;                  // chunks per row
     const int64_t wbase = (row0 * gpr) >> 5;        // first bitmap word of the tile's rows
     int nwords = 0;
     if (PAL) {
@@ -165,18 +186,20 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
     const Palette16 P = a.palette;
 
     // this warp's chunks [ch0, ch0 + nch)
-    const int64_t ch0 = gpr * warp / slices;
-    const int nch = int(gpr * (warp + 1) / slices - ch0);
+    const int64_t ch0 = cpr * warp / slices;
+    const int nch = int(cpr * (warp + 1) / slices - ch0);
 
     // per-lane streams, advanced one chunk at a time
-    const int64_t ea = ra * a.k + ch0 * kChunk + c * 16, eb = ea + 8 * a.k;
+    const int64_t ea = ra * a.k + ch0 * kCh + c * kWl, eb = ea + 8 * a.k;
     const uint8_t *sma = a.sm + ea, *smb = a.sm + eb;
     const uint32_t *pala = a.pal + ea / 8, *palb = a.pal + eb / 8;
     const uint16_t *wa = a.w_bf16 + ea, *wb = a.w_bf16 + eb;
-    const int64_t ga = ra * gpr + ch0, gb = rb * gpr + ch0;   // group of the slice's first chunk
+    const int coff = (c * kWl) / kChunk;                      // group of the lane inside a chunk
+    const int goff = (c * kWl) % kChunk;                      // the lane's offset inside its group
+    const int64_t ga = ra * gpr + ch0 * Q, gb = ga + 8 * gpr; // first group of the slice, rows g and g + 8
     // X rows of this lane's tokens (clamped: columns >= m are not stored)
-    const uint16_t *x0 = a.x + int64_t(min(g, a.m - 1)) * a.k + ch0 * kChunk + c * 16;
-    const uint16_t *x1 = a.x + int64_t(min(g + 8, a.m - 1)) * a.k + ch0 * kChunk + c * 16;
+    const uint16_t *x0 = a.x + int64_t(min(g, a.m - 1)) * a.k + ch0 * kCh + c * kWl;
+    const uint16_t *x1 = a.x + int64_t(min(g + 8, a.m - 1)) * a.k + ch0 * kCh + c * kWl;
 
     uint64_t rawa = 0, rawb = 0;
     if (PAL) {
@@ -190,38 +213,39 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
 #pragma unroll
         for (int q = 0; q < 4; q++) d0[t][q] = d1[t][q] = 0.f;
 
-    Half ha[kStages], hb[kStages];
+    Half<Q> ha[kStages], hb[kStages];
     bool fa[kStages], fb[kStages];
     auto issue = [&](int i, int s) {   // loads of chunk i into ring slot s
-        const int bit = i & 63;
+        const int bit = ((i * Q) & 63) + coff;
         fa[s] = PAL && ((rawa >> bit) & 1u);
         fb[s] = PAL && ((rawb >> bit) & 1u);
-        ha[s] = load_half<PAL>(a, sma + int64_t(i) * kChunk, pala + i * 8, wa + int64_t(i) * kChunk, fa[s], ga + i,
-                               sflags, srb, wbase, c);
-        hb[s] = load_half<PAL>(a, smb + int64_t(i) * kChunk, palb + i * 8, wb + int64_t(i) * kChunk, fb[s], gb + i,
-                               sflags, srb, wbase, c);
+        ha[s] = load_half<PAL, Q>(a, sma + int64_t(i) * kCh, pala + i * (kCh / 8), wa + int64_t(i) * kCh, fa[s],
+                                  ga + i * Q + coff, goff, sflags, srb, wbase);
+        hb[s] = load_half<PAL, Q>(a, smb + int64_t(i) * kCh, palb + i * (kCh / 8), wb + int64_t(i) * kCh, fb[s],
+                                  gb + i * Q + coff, goff, sflags, srb, wbase);
+    };
+    auto mma_tile = [&](int t, const uint32_t (&wA)[8 * Q], const uint32_t (&wB)[8 * Q], const uint16_t *xrow) {
+        uint32_t xw[8 * Q];
+#pragma unroll
+        for (int i = 0; i < 2 * Q; i++) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
+            xw[4 * i] = v.x;
+            xw[4 * i + 1] = v.y;
+            xw[4 * i + 2] = v.z;
+            xw[4 * i + 3] = v.w;
+        }
+        // step j: A = {row g pair 2j, row g+8 pair 2j, row g pair 2j+1, row g+8 pair 2j+1}
+#pragma unroll
+        for (int j = 0; j < 4 * Q; j++)
+            mma_16816((j & 1) ? d1[t] : d0[t], wA[2 * j], wB[2 * j], wA[2 * j + 1], wB[2 * j + 1], xw[2 * j],
+                      xw[2 * j + 1]);
     };
     auto consume = [&](int i, int s) {
-        uint32_t wA[8], wB[8];
-        rebuild<PAL>(ha[s], fa[s], P, wA);
-        rebuild<PAL>(hb[s], fb[s], P, wB);
-        const uint4 *xp0 = reinterpret_cast<const uint4 *>(x0 + int64_t(i) * kChunk);
-        const uint4 p0 = __ldg(xp0), q0 = __ldg(xp0 + 1);
-        const uint32_t xa[8] = {p0.x, p0.y, p0.z, p0.w, q0.x, q0.y, q0.z, q0.w};
-        // step j: A = {row g pair 2j, row g+8 pair 2j, row g pair 2j+1, row g+8 pair 2j+1}
-        mma_16816(d0[0], wA[0], wB[0], wA[1], wB[1], xa[0], xa[1]);
-        mma_16816(d1[0], wA[2], wB[2], wA[3], wB[3], xa[2], xa[3]);
-        mma_16816(d0[0], wA[4], wB[4], wA[5], wB[5], xa[4], xa[5]);
-        mma_16816(d1[0], wA[6], wB[6], wA[7], wB[7], xa[6], xa[7]);
-        if (NT == 2) {
-            const uint4 *xp1 = reinterpret_cast<const uint4 *>(x1 + int64_t(i) * kChunk);
-            const uint4 p1 = __ldg(xp1), q1 = __ldg(xp1 + 1);
-            const uint32_t xb[8] = {p1.x, p1.y, p1.z, p1.w, q1.x, q1.y, q1.z, q1.w};
-            mma_16816(d0[NT - 1], wA[0], wB[0], wA[1], wB[1], xb[0], xb[1]);
-            mma_16816(d1[NT - 1], wA[2], wB[2], wA[3], wB[3], xb[2], xb[3]);
-            mma_16816(d0[NT - 1], wA[4], wB[4], wA[5], wB[5], xb[4], xb[5]);
-            mma_16816(d1[NT - 1], wA[6], wB[6], wA[7], wB[7], xb[6], xb[7]);
-        }
+        uint32_t wA[8 * Q], wB[8 * Q];
+        rebuild<PAL, Q>(ha[s], fa[s], P, wA);
+        rebuild<PAL, Q>(hb[s], fb[s], P, wB);
+        mma_tile(0, wA, wB, x0 + int64_t(i) * kCh);
+        if (NT == 2) mma_tile(NT - 1, wA, wB, x1 + int64_t(i) * kCh);
     };
 
 #pragma unroll
@@ -235,9 +259,9 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
             consume(i, s);
             const int nx = i + kStages;
             if (nx < nch) {
-                if (PAL && (nx & 63) == 0) {   // next 64-chunk window of raw bits
-                    rawa = raw_window(sflags, nwords, wbase, ga + nx);
-                    rawb = raw_window(sflags, nwords, wbase, gb + nx);
+                if (PAL && nx % kWin == 0) {   // next 64-group window of raw bits
+                    rawa = raw_window(sflags, nwords, wbase, ga + nx * Q);
+                    rawb = raw_window(sflags, nwords, wbase, gb + nx * Q);
                 }
                 issue(nx, s);
             }
@@ -264,9 +288,9 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
         for (int t = 0; t < NT; t++)
 #pragma unroll
             for (int q = 0; q < 4; q++) {
-                float s = red[lane * 4 * NT + t * 4 + q];
-                for (int w = 1; w < slices; w++) s += red[(w * 32 + lane) * 4 * NT + t * 4 + q];
-                v[t][q] = s;
+                float acc = red[lane * 4 * NT + t * 4 + q];
+                for (int w = 1; w < slices; w++) acc += red[(w * 32 + lane) * 4 * NT + t * 4 + q];
+                v[t][q] = acc;
             }
     }
 #pragma unroll
@@ -286,10 +310,12 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
 }  // namespace
 
 cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
-                            const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices,
+                            const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices, int width,
                             cudaStream_t stream) {
     if (m < 1 || m > 16 || slices < 1 || slices > kMaxSlices || n % kTileRows || k % kChunk)
         return cudaErrorInvalidValue;
+    const int q = width == 1 ? 1 : width == 2 ? 2 : (k % (2 * kChunk) == 0 ? 2 : 1);
+    if (k % (q * kChunk)) return cudaErrorInvalidValue;
     MmaArgs a{};
     a.x = x;
     a.w_bf16 = w_bf16;
@@ -313,13 +339,15 @@ cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, co
     const unsigned block = unsigned(slices * 32);
     const size_t smem = size_t(2 * a.flag_words) * 4 + (slices > 1 ? size_t(slices) * 32 * 4 * nt * 4 : 0);
     if (smem > size_t(kMaxSmem)) return cudaErrorInvalidValue;
+#define UW_MMA_LAUNCH(P_, N_, Q_) k_gemv_mma<P_, N_, Q_><<<grid, block, smem, stream>>>(a)
     if (pal) {
-        if (nt == 2) k_gemv_mma<true, 2><<<grid, block, smem, stream>>>(a);
-        else k_gemv_mma<true, 1><<<grid, block, smem, stream>>>(a);
+        if (q == 2) { if (nt == 2) UW_MMA_LAUNCH(true, 2, 2); else UW_MMA_LAUNCH(true, 1, 2); }
+        else { if (nt == 2) UW_MMA_LAUNCH(true, 2, 1); else UW_MMA_LAUNCH(true, 1, 1); }
     } else {
-        if (nt == 2) k_gemv_mma<false, 2><<<grid, block, smem, stream>>>(a);
-        else k_gemv_mma<false, 1><<<grid, block, smem, stream>>>(a);
+        if (q == 2) { if (nt == 2) UW_MMA_LAUNCH(false, 2, 2); else UW_MMA_LAUNCH(false, 1, 2); }
+        else { if (nt == 2) UW_MMA_LAUNCH(false, 2, 1); else UW_MMA_LAUNCH(false, 1, 1); }
     }
+#undef UW_MMA_LAUNCH
     return cudaGetLastError();
 }
 

@@ -23,10 +23,11 @@ cudaError_t launch_gemv_fma(const uint16_t *x, int m, const uint16_t *w_bf16, co
                             int rows_per_warp, uint32_t *status, cudaStream_t stream);
 
 // Warp-level MMA skinny matmul, m <= 16 (Unweight page §七): W rebuilt in
-// registers into mma.m16n8k16 fragments, 8 rows per warp, `slices` (1..8)
-// warps per CTA splitting K.  pal_plane == nullptr: plain BF16 weights.
+// registers into mma.m16n8k16 fragments, 16 rows per CTA, `slices` (1..8)
+// warps per CTA splitting K; `width` 1: 16 weights per lane and row per step,
+// 2: 32, 0: 32 when k is a multiple of 128.  pal_plane == nullptr: plain BF16.
 cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
-                            const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices,
+                            const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices, int width,
                             cudaStream_t stream);
 
 // tcgen05 GEMM (Unweight page §七, reconstructive matmul), token tile `bn`.

@@ -52,7 +52,7 @@ def main(argv=None):
     if a.kernel in ("fma", "plain_fma"):
         plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_FMA, a.bn or 1, 1)
     elif a.kernel in ("mma", "plain_mma"):
-        plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, a.bn or 2, 1)
+        plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, a.bn or 2, 1, a.stages)
     else:
         plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, a.bn or 16, a.split, a.stages)
     ws_bytes = uw.workspace_size(a.m, a.n, a.k, plan) if a.kernel not in ("decode", "transcode") else 0

@@ -128,9 +128,17 @@ def test_fma_gemv_parity(uw, m, rows):
 
 @pytest.mark.parametrize("m", [1, 2, 3, 7, 8, 9, 12, 16])
 @pytest.mark.parametrize("slices", [1, 2, 3, 8])
-def test_mma_gemv_parity(uw, m, slices):
-    # k = 1600 = 25 chunks: uneven K slices; n = 320 = 20 tiles of 16 rows
-    _matmul_case(uw, 320, 1600, m, dict(kernel=uw.KERNEL_MMA, bn=slices, split_k=1), seed=100 + m)
+@pytest.mark.parametrize("width", [1, 2])
+def test_mma_gemv_parity(uw, m, slices, width):
+    # k = 1664 = 26 groups = 13 chunks of 128: uneven K slices for both chunk
+    # widths; n = 320 = 20 tiles of 16 rows
+    _matmul_case(uw, 320, 1664, m, dict(kernel=uw.KERNEL_MMA, bn=slices, split_k=1, stages=width),
+                 seed=100 + m)
+
+
+def test_mma_gemv_width_default_on_odd_groups(uw):
+    # k = 1600 (25 groups) is not a multiple of 128: the default width falls back to 64-weight chunks
+    _matmul_case(uw, 320, 1600, 5, dict(kernel=uw.KERNEL_MMA, bn=3, split_k=1), seed=7)
 
 
 def test_mma_gemv_many_tiles(uw):
@@ -142,7 +150,9 @@ def test_mma_gemv_raw_heavy_and_long_k(uw):
     # 5% outliers: most groups raw; k = 14336 (224 chunks per row, bitmap
     # words of a tile not aligned to rows)
     _matmul_case(uw, 64, 704, 5, dict(kernel=uw.KERNEL_MMA, bn=2, split_k=1), seed=4, frac=0.05)
+    _matmul_case(uw, 64, 768, 5, dict(kernel=uw.KERNEL_MMA, bn=2, split_k=1, stages=2), seed=4, frac=0.05)
     _matmul_case(uw, 128, 14336, 16, dict(kernel=uw.KERNEL_MMA, bn=4, split_k=1), seed=5, frac=0.001)
+    _matmul_case(uw, 128, 14336, 3, dict(kernel=uw.KERNEL_MMA, bn=8, split_k=1, stages=1), seed=6, frac=0.001)
 
 
 @pytest.mark.parametrize("bn,m", [(16, 1), (16, 16), (32, 20), (64, 64), (64, 100), (128, 128),

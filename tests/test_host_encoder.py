@@ -241,9 +241,12 @@ def test_plans_and_workspace(uw):
     for bad_m, bad in ((17, uw.make_plan(kernel=uw.KERNEL_MMA, bn=1)),     # MMA needs m <= 16
                        (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=0)),
                        (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=9)),
-                       (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, split_k=2))):
+                       (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, split_k=2)),
+                       (4, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, stages=3))):
         with pytest.raises(uw.UwError):
             uw.workspace_size(bad_m, n, k, bad)
+    with pytest.raises(uw.UwError):   # 128-weight steps need K a multiple of 128
+        uw.workspace_size(4, n, 1600, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, stages=2))
 
 
 def test_stack_workspace_and_argument_checks(uw):
