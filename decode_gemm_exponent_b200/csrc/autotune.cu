@@ -5,12 +5,16 @@
 // For each matrix and each batch size m the candidates are the pipelines the
 // blob supports (decode + plain kernel, runtime transcode + fused kernel,
 // direct palette + fused kernel) crossed with the kernel variants: the
-// warp-MMA kernel (m <= 16, 2-8 K slices per tile, 16 or 32 weights per
-// lane and step), the FMA GEMV (m <= 8, 1
-// or 2 rows per warp) and the tcgen05 kernel with token tiles
-// around m and split-K factors that fill the 148 SMs.  Each candidate is run
-// once to warm up (its status is checked) and then `reps` times between CUDA
-// events; the fastest average wins.
+// warp-MMA kernel (m <= 16, 2-8 K slices per tile, 16 or 32 weights per lane
+// and step), the FMA GEMV (m <= 8, 1 or 2 rows per warp) and the tcgen05
+// kernel with token tiles around m and split-K factors 1-8 (so that some
+// candidate fills the 148 SMs with close to whole waves).  Each candidate is
+// run once to warm up (its status is checked) and then `reps` times, each
+// call timed on its own between CUDA events after a 192 MB read of scratch
+// space has pushed the matrix out of the 126 MB L2 (a read, so the evicted
+// lines are clean and no write-back lands in the timed call): the weights
+// stream from HBM as they do in a model's layer sequence.  The fastest
+// average wins.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -72,7 +76,7 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
             if (bn < 16) continue;
             const int64_t tiles = ((w.n + 127) / 128) * ((m + bn - 1) / bn);
             const int ksteps = int(w.k / 64);
-            for (int split : {1, 2, 4, 8}) {
+            for (int split : {1, 2, 3, 4, 5, 6, 8}) {
                 if (split > 1 && (tiles * split > 4 * kSMs || ksteps / split < 4)) continue;
                 if (split > 1 && tiles >= 2 * kSMs) continue;
                 uw_plan p{};
