@@ -207,6 +207,34 @@ def run_reference(args, rank):
 
 # ----------------------------------------------------------------------------- GPU leg
 
+# DRAM traffic of the dominant kernel group's launch, from one ncu capture
+# (profiles/k_gemv_mma_traffic_8b_gate_m1.md): bytes per launch, the
+# algorithmic bytes of that launch, and a SHA-256 over the kernel's sources;
+# the figure is reported only while those sources are unchanged.
+MEASURED_TRAFFIC = {
+    "fused/mma_gemv_s4_w2": {
+        "bytes": 92491520, "alg_bytes": 89956928,
+        "files": ("decode_gemm_exponent_b200/csrc/gemv_mma.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
+        "sha256": "df094ee9d9d6c79e12b1b3523a46faa5d9680990a4707e53ffe7ac5d0ec21fc2",
+    },
+}
+
+
+def measured_traffic(group: str, alg_bytes_per_launch: float):
+    """ncu DRAM bytes per launch of `group`, scaled by algorithmic bytes, or None."""
+    import hashlib
+    rec = MEASURED_TRAFFIC.get(group)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for f in rec["files"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes"] * alg_bytes_per_launch / rec["alg_bytes"]
+
+
 def alg_bytes(mat, m, plan):
     """Algorithmic HBM bytes of the kernels one matmul call launches."""
     info = mat.info
@@ -378,7 +406,8 @@ def run_gpu(args, rank, world):
             "per_call_us": {"%s@M=%d" % (c["name"], c["m"]): round(1e3 * t, 2) for c, t in zip(calls, per_call)},
         },
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": measured_traffic(dom_name, dom["bytes"] / dom["calls"]),
                      "peak_source": peaks["_source"] + " hbm_gbs"},
         "cpu_baseline": cpu,
         "e2e": {"value": aggregate_gbs(weight_bytes, world, e2e_ms), "unit": "GB/s",

@@ -569,7 +569,9 @@ template <int BN>
 cudaError_t launch_plain(const TcLaunch &p, cudaStream_t stream) {
     using C = PlainCfg<BN>;
     const int max_stages = std::min(8, (kMaxSmem - 1024 - plain_tail(8)) / C::kStage);
-    int stages = (p.stages <= 0 || p.stages > max_stages) ? max_stages : p.stages;
+    // default depth 4: deeper rings measured slower (more outstanding TMA
+    // loads per SM than HBM serves efficiently), 2 too shallow
+    int stages = p.stages <= 0 ? std::min(4, max_stages) : std::min(p.stages, max_stages);
     if (stages < 2) return cudaErrorInvalidValue;
     const size_t smem = size_t(stages) * C::kStage + 1024 + plain_tail(stages);
     CUtensorMap mx, mw;

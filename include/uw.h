@@ -206,7 +206,8 @@ typedef struct uw_plan {
                              MMA: warps per CTA = K slices per 16-row tile, 1..8 */
     int32_t split_k;      /* TC: K split into this many slices (>= 1), reduced in a
                              fixed order; FMA, MMA: must be 1 */
-    int32_t stages;       /* TC: shared-memory ring depth (0 = largest that fits);
+    int32_t stages;       /* TC: shared-memory ring depth (0 = default: 4 for the plain
+                             kernel, the largest that fits for the fused one);
                              MMA: weights per lane and row per step, 1 = 16, 2 = 32
                              (K a multiple of 128), 0 = 32 when K allows, else 16 */
     uint32_t debug_flags; /* UW_DEBUG_* (0 in production) */

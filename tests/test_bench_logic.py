@@ -1,0 +1,46 @@
+"""Host-side logic of bench.py that needs no GPU: the measured-traffic
+lookup and the plan-file round trip."""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_measured_traffic_lookup():
+    # unknown kernel group: no figure
+    assert bench.measured_traffic("fused/no_such_kernel", 1e6) is None
+    for group, rec in bench.MEASURED_TRAFFIC.items():
+        got = bench.measured_traffic(group, 2 * rec["alg_bytes"])
+        # either the sources still match the capture (scaled figure) or they
+        # changed since (None); never a figure for different sources
+        assert got is None or abs(got - 2 * rec["bytes"]) < 1e-6 * rec["bytes"]
+    saved = dict(bench.MEASURED_TRAFFIC)
+    try:
+        name, rec = next(iter(saved.items()))
+        bench.MEASURED_TRAFFIC[name] = dict(rec, sha256="0" * 64)   # pretend the kernel changed
+        assert bench.measured_traffic(name, rec["alg_bytes"]) is None
+    finally:
+        bench.MEASURED_TRAFFIC.clear()
+        bench.MEASURED_TRAFFIC.update(saved)
+
+
+def test_plans_from_json_round_trip():
+    from decode_gemm_exponent_b200 import uw
+    doc = {"plans": []}
+    kinds = [("fma", 1, 1, 0), ("tc", 64, 4, 0), ("mma", 4, 1, 2)]
+    for i in range(3):
+        for j, m in enumerate(bench.MS):
+            kern, bn, split, stages = kinds[(i + j) % 3]
+            doc["plans"].append({"matrix": i, "m": m, "best": {"pipeline": "direct_palette", "kernel": kern,
+                                                                "bn": bn, "split_k": split, "stages": stages}})
+    plans = bench.plans_from_json(json.dumps(doc), 3, uw)
+    for i in range(3):
+        for j in range(len(bench.MS)):
+            kern, bn, split, stages = kinds[(i + j) % 3]
+            p = plans[i][j]
+            assert p.kernel == {"fma": 1, "tc": 2, "mma": 3}[kern] and p.bn == bn and p.split_k == split
+            assert p.stages == stages and p.pipeline == uw.PIPE_DIRECT_PALETTE
