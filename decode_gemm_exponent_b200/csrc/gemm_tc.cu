@@ -23,7 +23,11 @@
 //     (one 64-byte slot per row); freed as soon as the rebuild has read it;
 //   W ring (4 stages for BN <= 64, else 2): rebuilt BF16 W tiles (128-byte
 //     swizzle, K-major); freed by the MMA's commit;
-//   X ring (8 / 4 / 2 stages): X tiles, freed by the MMA's commit.
+//   X ring (8 / 4 / 2 stages): X tiles, freed by the MMA's commit.  With a
+//   256-token tile and more than 256 tokens, a CTA owns two token tiles: an
+//   X stage holds both, the MMA thread issues each K-step for both against
+//   the same rebuilt W stage (two accumulators filling the 512 TMEM
+//   columns), so a W tile is rebuilt once per 512 tokens instead of 256.
 //   warp 0     compressed tiles: two TMA loads per K-step.
 //   warp 1     MMA issuer and TMEM owner.
 //   warp 2     X producer (TMA).
@@ -226,19 +230,21 @@ __global__ void __launch_bounds__(kPlainThreads, 1)
 
 // ============================================================== fused kernel
 
-template <int BN>
+template <int BN, int TT>   // TT: token tiles per CTA sharing each rebuilt W tile
 struct FusedCfg {
     static constexpr int kWS = BN <= 64 ? 4 : 2;        // rebuilt-W ring (multiple of kGroups)
     static constexpr int kXS = BN <= 64 ? 8 : (BN == 128 ? 4 : 2);   // X ring
     static constexpr int kW = kBM * kBK * 2;            // rebuilt W tile
     static constexpr int kX = BN * kBK * 2;             // X tile
+    static constexpr int kXT = TT * kX;                 // X ring stage: TT token tiles
     static constexpr int kSM = kBM * kBK;               // sign/mantissa tile
     static constexpr int kPL = kBM * kBK / 2;           // palette tile
     static constexpr int kRAW = kBM * kGroup;           // raw exponents, one 64-byte slot per row
     static constexpr int kCStage = kSM + kPL + kRAW;    // compressed ring stage
     static constexpr int kOffPL = kSM, kOffRAW = kSM + kPL;
-    static constexpr uint32_t kTmemCols = BN < 32 ? 32u : uint32_t(BN);
+    static constexpr uint32_t kTmemCols = uint32_t(TT) * (BN < 32 ? 32u : uint32_t(BN));
     static_assert(kW % 1024 == 0 && kX % 1024 == 0 && kCStage % 1024 == 0, "1024-byte alignment");
+    static_assert(kTmemCols <= 512, "accumulators exceed TMEM");
 };
 
 constexpr int kRawProducers = 4;      // warps; lane l of warp j owns tile row 32 j + l
@@ -250,16 +256,16 @@ __host__ __device__ constexpr int fused_tail(int cs, int ws, int xs, int bw) {
     return kBM * bw * 4 + kBM * 4 + (2 * cs + 2 * ws + 2 * xs + 2) * 8 + 16;
 }
 
-template <int BN>
+template <int BN, int TT>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_gemm_tc_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmSM,
                     const __grid_constant__ CUtensorMap tmPL, const TcArgs a, int bw) {
-    using C = FusedCfg<BN>;
+    using C = FusedCfg<BN, TT>;
     constexpr int WS = C::kWS, XS = C::kXS;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *wring = align1024(smem_dyn);
     uint8_t *xring = wring + WS * C::kW;
-    uint8_t *cring = xring + XS * C::kX;
+    uint8_t *cring = xring + XS * C::kXT;
     const int CS = a.stages;                      // compressed stages (even)
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(cring + size_t(CS) * C::kCStage);   // [128][bw]
     uint32_t *rank0 = bitmap + kBM * bw;                                                // [128]
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n0 = int64_t(blockIdx.x) * kBM;
-    const int64_t m0 = int64_t(blockIdx.y) * BN;
+    const int64_t m0 = int64_t(blockIdx.y) * BN * TT;
     const int split = blockIdx.z;
     const int ks_begin = split * a.ks_per_split;
     const int nks = max(0, min(int(a.k / kBK) - ks_begin, a.ks_per_split));
@@ -378,8 +384,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                      mbar_wait(&w_full[ws], uint32_t(ks / WS) & 1u, T);
                 if (!ok) break;
                 tc_fence_after();
-                mma_kstep<BN>(tmem, smem_addr(wring + size_t(ws) * C::kW), smem_addr(xring + size_t(xs) * C::kX),
-                              ks == 0);
+#pragma unroll
+                for (int t = 0; t < TT; t++)
+                    mma_kstep<BN>(tmem + uint32_t(t * BN), smem_addr(wring + size_t(ws) * C::kW),
+                                  smem_addr(xring + size_t(xs) * C::kXT + size_t(t) * C::kX), ks == 0);
                 tc_commit(&w_empty[ws]);
                 tc_commit(&x_empty[xs]);
             }
@@ -402,8 +410,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     break;
                 }
                 if (*abort_flag) break;
-                mbar_arrive_expect_tx(&x_full[s], uint32_t(C::kX));
-                tma_load_2d(xring + size_t(s) * C::kX, &tmX, (ks_begin + ks) * kBK, int32_t(m0), &x_full[s]);
+                mbar_arrive_expect_tx(&x_full[s], uint32_t(C::kXT));
+#pragma unroll
+                for (int t = 0; t < TT; t++)   // a tile past the last token reads the zero fill
+                    tma_load_2d(xring + size_t(s) * C::kXT + size_t(t) * C::kX, &tmX, (ks_begin + ks) * kBK,
+                                int32_t(m0 + t * BN), &x_full[s]);
                 issued = ks + 1;
             }
             for (int ks = max(0, issued - XS); ks < issued; ks++)
@@ -487,7 +498,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tc_fence_after();
         const bool skip = __any_sync(0xFFFFFFFFu, !ok || *abort_flag != 0 || nks == 0);
         if (!ok && lane == 0) flag_error(a.status, UW_DEVERR_TIMEOUT);
-        if (!skip) store_accumulator<BN>(tmem, q, grp, kGroups, lane, n0, m0, split, a);
+        if (!skip)
+#pragma unroll 1
+            for (int t = 0; t < TT; t++)
+                if (m0 + t * BN < a.m)
+                    store_accumulator<BN>(tmem + uint32_t(t * BN), q, grp, kGroups, lane, n0, m0 + t * BN, split, a);
     }
 
     tc_fence_before();
@@ -603,21 +618,21 @@ cudaError_t launch_plain(const TcLaunch &p, cudaStream_t stream) {
     return cudaSuccess;
 }
 
-template <int BN>
+template <int BN, int TT>
 cudaError_t launch_fused(const TcLaunch &p, cudaStream_t stream) {
-    using C = FusedCfg<BN>;
+    using C = FusedCfg<BN, TT>;
     TcArgs a{};
     a.m = p.m;
     a.n = p.n;
     a.k = p.k;
     split_k_slices(p, a);
     const int bw = (a.ks_per_split + 31) / 32;     // raw bitmap words per row
-    const int fixed = C::kWS * C::kW + C::kXS * C::kX + 1024 + fused_tail(8, C::kWS, C::kXS, bw);
+    const int fixed = C::kWS * C::kW + C::kXS * C::kXT + 1024 + fused_tail(8, C::kWS, C::kXS, bw);
     int max_cs = (kMaxSmem - fixed) / C::kCStage;
     max_cs = std::min(8, max_cs) & ~1;      // even: each rebuild group owns every other stage
     int cs = (p.stages <= 0 || p.stages > max_cs) ? max_cs : (p.stages & ~1);
     if (cs < 2) return cudaErrorInvalidValue;
-    const size_t smem = size_t(C::kWS) * C::kW + size_t(C::kXS) * C::kX + size_t(cs) * C::kCStage + 1024 +
+    const size_t smem = size_t(C::kWS) * C::kW + size_t(C::kXS) * C::kXT + size_t(cs) * C::kCStage + 1024 +
                         fused_tail(cs, C::kWS, C::kXS, bw);
     CUtensorMap mx, msm, mpl;
     if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2,
@@ -639,10 +654,10 @@ cudaError_t launch_fused(const TcLaunch &p, cudaStream_t stream) {
     a.pal = make_palette16(p.w->palette);
     if (a.split_k > 1 && !p.partial) return cudaErrorInvalidValue;
     static thread_local int ready[16] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
-    cudaError_t err = prepare(k_gemm_tc_fused<BN>, kFusedThreads, smem, C::kTmemCols, cs, ready);
+    cudaError_t err = prepare(k_gemm_tc_fused<BN, TT>, kFusedThreads, smem, C::kTmemCols, cs, ready);
     if (err != cudaSuccess) return err;
-    dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN - 1) / BN), unsigned(a.split_k));
-    k_gemm_tc_fused<BN><<<grid, kFusedThreads, smem, stream>>>(mx, msm, mpl, a, bw);
+    dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN * TT - 1) / (BN * TT)), unsigned(a.split_k));
+    k_gemm_tc_fused<BN, TT><<<grid, kFusedThreads, smem, stream>>>(mx, msm, mpl, a, bw);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (a.split_k > 1) return launch_splitk_reduce(p.partial, a.split_k, p.m * p.n, p.y, stream);
@@ -651,7 +666,12 @@ cudaError_t launch_fused(const TcLaunch &p, cudaStream_t stream) {
 
 template <int BN>
 cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
-    return p.w_bf16 ? launch_plain<BN>(p, stream) : launch_fused<BN>(p, stream);
+    if (p.w_bf16) return launch_plain<BN>(p, stream);
+    // more than one 256-token tile: two tiles per CTA share each rebuilt W
+    // tile (the two accumulators fill TMEM), halving the rebuild work; every
+    // accumulator sees the same MMA sequence, so the result bits do not change
+    if (BN == 256 && p.m > BN) return launch_fused<BN, 2>(p, stream);
+    return launch_fused<BN, 1>(p, stream);
 }
 
 }  // namespace
