@@ -281,12 +281,17 @@ __device__ __forceinline__ uint4 join8(uint32_t r0, uint32_t r1, uint32_t s0, ui
 }
 
 // 8 palette indices in natural order -> the stored 4-bit-palette word layout.
+// Low three bits stay in place; bit 3 of index j moves to bit 8j+7 (j < 4) or
+// 8(j-4)+3 (j >= 4).  Sign-replicating byte permutes turn bit 3 of the even
+// indices (top bit of each byte of x << 4) and of the odd indices (top bit of
+// each byte of x) into byte masks, and two interleaving permutes place index
+// j's mask in byte j (for bit 7) and index j+4's in byte j (for bit 3).
 __device__ __forceinline__ uint32_t natural_to_pal(uint32_t x) {
-    const uint32_t low3 = x & 0x77777777u;
-    const uint32_t b = (x >> 3) & 0x11111111u;                              // bit 3 of j at bit 4j
-    const uint32_t vlo = (((b & 0x1111u) * 0x1248u) >> 12) & 0xFu;          // j = 0..3 -> bits 0..3
-    const uint32_t vhi = ((((b >> 16) & 0x1111u) * 0x1248u) >> 12) & 0xFu;  // j = 4..7
-    return low3 | ((vlo * 0x10204080u) & 0x80808080u) | ((vhi * 0x01020408u) & 0x08080808u);
+    const uint32_t even = prmt(x << 4, 0u, 0xBA98u);   // byte k: bit 3 of index 2k
+    const uint32_t odd = prmt(x, 0u, 0xBA98u);         // byte k: bit 3 of index 2k+1
+    const uint32_t hi = prmt(even, odd, 0x5140u);      // byte j: index j        (j < 4)
+    const uint32_t lo = prmt(even, odd, 0x7362u);      // byte j: index j + 4
+    return (x & 0x77777777u) | (hi & 0x80808080u) | (lo & 0x08080808u);
 }
 
 // acc += a * b over the two BF16 halves of each operand (exact products,
