@@ -213,9 +213,9 @@ def run_reference(args, rank):
 # the figure is reported only while those sources are unchanged.
 MEASURED_TRAFFIC = {
     "fused/mma_gemv_s4_w2": {
-        "bytes": 92491520, "alg_bytes": 89956928,
+        "bytes": 93808128, "alg_bytes": 89956928,
         "files": ("decode_gemm_exponent_b200/csrc/gemv_mma.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
-        "sha256": "df094ee9d9d6c79e12b1b3523a46faa5d9680990a4707e53ffe7ac5d0ec21fc2",
+        "sha256": "93917f7df6283c37da2919c71b54180147b326a961d8a73e983c92e65cf3187a",
     },
 }
 
