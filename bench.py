@@ -15,7 +15,8 @@ each read comes from HBM, not from the 126 MB L2.
 value  = sum over the step's matmuls of 2*N*K (uncompressed BF16 weight bytes)
          / step time  [GB/s], inputs resident in HBM, CUDA events, max over ranks.
 e2e    = the same, with X copied from pinned host memory and Y read back to
-         pinned host memory inside the timed region, through the C ABI.
+         pinned host memory inside the timed region, through the C ABI (copies
+         on their own streams, ordered by events, overlapping the matmuls).
 roofline: the kernel group with the largest share of the step; achieved =
          its algorithmic bytes (compressed planes + X + Y) / its event-timed
          duration, against the measured HBM copy bandwidth.
@@ -357,21 +358,46 @@ def run_gpu(args, rank, world):
     achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
     peak = float(peaks["hbm_gbs"])
 
-    # ---- end-to-end through the C ABI with pinned host buffers
+    # ---- end-to-end through the C ABI with pinned host buffers.  As a
+    # serving loop would, the copies run on their own streams ordered by
+    # events: a step's inputs go up on one copy stream into one of two device
+    # input sets (so they can be sent while the previous step still reads the
+    # other set), every result comes down on another copy stream as soon as
+    # its matmul ends, and the step's matmuls wait only for their inputs.
     hx = {(c["m"], c["mat"].k): c["x"].cpu().pin_memory() for c in calls}
     hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
     h2d = sum(t.numel() * 2 for t in hx.values())
     d2h = sum(t.numel() * 4 for t in hy)
+    xsets = [{key: xs[key[0]][key[1]] for key in hx}, {key: xs[key[0]][key[1]].clone() for key in hx}]
+    copy_in, copy_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()
+    x_ready = [ev() for _ in range(args.steps)]
+    x_free = [ev() for _ in range(args.steps)]
+    y_ready = [[ev() for _ in calls] for _ in range(args.steps)]
+    y_free = [[ev() for _ in calls] for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.steps):
-        for key, t in hx.items():
-            xs[key[0]][key[1]].copy_(t, non_blocking=True)
-        for c, h in zip(calls, hy):
-            issue(c)
-            h.copy_(c["y"], non_blocking=True)
+    for s in range(args.steps):
+        xset = xsets[s & 1]
+        copy_in.wait_event(e0 if s < 2 else x_free[s - 2])     # matmuls of step s-2 read this set
+        with torch.cuda.stream(copy_in):
+            for key, t in hx.items():
+                xset[key].copy_(t, non_blocking=True)
+        x_ready[s].record(copy_in)
+        stream.wait_event(x_ready[s])
+        for i, (c, h) in enumerate(zip(calls, hy)):
+            if s > 0:
+                stream.wait_event(y_free[s - 1][i])              # last step's result is on the host
+            c["mat"].matmul(xset[(c["m"], c["mat"].k)], c["plan"], y=c["y"], ws=c["ws"])
+            y_ready[s][i].record(stream)
+            copy_out.wait_event(y_ready[s][i])
+            with torch.cuda.stream(copy_out):
+                h.copy_(c["y"], non_blocking=True)
+            y_free[s][i].record(copy_out)
+        x_free[s].record(stream)
+    stream.wait_stream(copy_out)                                # every result is on the host
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
