@@ -83,19 +83,19 @@ def load_peaks():
 
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons through NVML (read-only)
-    from a background thread every ~1 ms while the timed region runs, and
-    keeps a CSV of the samples under gpurun_out/."""
+    from a background thread every ~1 ms while the timed region runs; with a
+    `csv_path` the samples are also written there."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, csv_path=None):
         self.gpu = gpu_index
         self.samples = []
         self.error = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
+        self.path = csv_path
 
     def _run(self):
         import pynvml as N
@@ -129,8 +129,9 @@ class ClockSampler:
         if self.thread is not None:
             self.stop.set()
             self.thread.join(timeout=2)
+        if self.thread is not None and self.path:
             try:
-                os.makedirs(os.path.dirname(self.path), exist_ok=True)
+                os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
                 with open(self.path, "w") as f:
                     f.write("time,sm_mhz,power_w,reasons\n")
                     for t, sm, pw, rs in self.samples:
@@ -331,7 +332,8 @@ def run_gpu(args, rank, world):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    clocks_csv = args.clocks_csv.replace("{rank}", str(rank)) if args.clocks_csv else None
+    with ClockSampler(local, clocks_csv) as clk:
         t_start.record(stream)
         for s in range(args.steps):
             for c, (e0, e1) in zip(calls, ev[s]):
@@ -455,6 +457,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write the clock samples of the timed region to this CSV ({rank} = rank)")
     ap.add_argument("--plan-json", default=None, help="write the autotuner's plan file here")
     ap.add_argument("--plans-in", default=None, help="use this plan file instead of autotuning")
     args = ap.parse_args()
