@@ -71,6 +71,10 @@ struct Half {
     uint4 b[Q];
 };
 
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -223,6 +227,9 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
                                   ga + i * Q + coff, goff, sflags, srb, wbase);
         hb[s] = load_half<PAL, Q>(a, smb + int64_t(i) * kCh, palb + i * (kCh / 8), wb + int64_t(i) * kCh, fb[s],
                                   gb + i * Q + coff, goff, sflags, srb, wbase);
+        // the chunk's X rows into L1 now, so that the MMA steps do not wait on L2
+        prefetch_l1(x0 + int64_t(i) * kCh);
+        if (NT == 2) prefetch_l1(x1 + int64_t(i) * kCh);
     };
     auto mma_tile = [&](int t, const uint32_t (&wA)[8 * Q], const uint32_t (&wB)[8 * Q], const uint16_t *xrow) {
         uint32_t xw[8 * Q];
