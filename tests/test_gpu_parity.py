@@ -206,6 +206,56 @@ def test_full_size_8b_sampled(uw, m, plan_kw):
     check_bound(yf[ri, rj], y_ref, a_ref)
 
 
+@pytest.mark.parametrize("frac", [0.0, 0.001, 0.01, 0.05])
+@pytest.mark.parametrize("sigma", [0.005, 0.015, 0.05])
+def test_70b_k_outlier_and_sigma_sweep(uw, frac, sigma):
+    """The 70B configuration's sweep (outlier fraction and per-matrix sigma)
+    at the 70B gate's K = 8192 on 256 rows: decode bit-exact, transcode equal
+    to the oracle's plane, and the warp-MMA (M = 1) and tcgen05 (M = 256)
+    fused kernels equal to their plain twins and within the oracle bound."""
+    n, k = 256, 8192
+    w = synth.weights_bf16(n, k, sigma, frac, 1.0, seed=int(1000 * sigma) + int(1e4 * frac))
+    mat = uw.Matrix(uw.encode(w))
+    assert np.array_equal(host16(mat.decode()), w)
+    assert np.array_equal(mat.transcode().cpu().numpy(), O.encode(w).pal_plane)
+    wd = dev16(w)
+    for m, kw in ((1, dict(kernel=uw.KERNEL_MMA, bn=4, split_k=1)), (256, dict(kernel=uw.KERNEL_TC, bn=256, split_k=1))):
+        x = synth.activations_bf16(m, k, seed=m)
+        xd = dev16(x)
+        plan = uw.make_plan(pipeline=4, **kw)
+        yf = mat.matmul(xd, plan).cpu().numpy()
+        yp = uw.matmul_bf16(xd, wd, plan).cpu().numpy()
+        assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32))
+        y_ref, a_ref = O.gemm(x, w)
+        check_bound(yf, y_ref, a_ref)
+    assert mat.device_status() == 0
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("m,plan_kw", [(1, dict(kernel=3, bn=4, split_k=1, stages=2)),
+                                       (1024, dict(kernel=2, bn=256, split_k=1))])
+def test_full_size_70b_gate_sampled(uw, m, plan_kw):
+    """70B gate shape [28672, 8192], sigma 0.015: fused == plain bit for bit
+    over the whole output, and 512 sampled outputs within the oracle bound
+    (M = 1024 runs two 256-token tiles per CTA)."""
+    n, k = 28672, 8192
+    w = synth.weights_bf16(n, k, 0.015, 0.0005, 1.0, seed=1)
+    x = synth.activations_bf16(m, k, seed=2)
+    mat = uw.Matrix(uw.encode(w))
+    xd, wd = dev16(x), dev16(w)
+    plan = uw.make_plan(pipeline=4, **plan_kw)
+    yf = mat.matmul(xd, plan).cpu().numpy()
+    yp = uw.matmul_bf16(xd, wd, plan).cpu().numpy()
+    assert mat.device_status() == 0
+    assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32))
+    rng = np.random.default_rng(1)
+    ri = rng.integers(0, m, 512)
+    rj = rng.integers(0, n, 512)
+    ri[:2], rj[:2] = [0, m - 1], [0, n - 1]
+    y_ref, a_ref = O.gemm_sampled(x, w, ri, rj)
+    check_bound(yf[ri, rj], y_ref, a_ref)
+
+
 # ---------------------------------------------------------------- failure paths
 
 def test_bounded_wait_times_out_and_context_survives(uw):
