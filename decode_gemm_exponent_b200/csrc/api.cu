@@ -177,10 +177,11 @@ extern "C" uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pi
     if (!plan || m <= 0 || n <= 0 || k <= 0) return UW_ERR_INVALID_ARG;
     std::memset(plan, 0, sizeof(*plan));
     plan->pipeline = pipeline ? pipeline : UW_PIPE_DIRECT_PALETTE;
-    if (m <= 4) {
-        plan->kernel = UW_KERNEL_FMA;
-        plan->bn = 1;
+    if (m <= 8) {
+        plan->kernel = UW_KERNEL_MMA;
+        plan->bn = 4;            // 4 warps per 16-row tile
         plan->split_k = 1;
+        plan->stages = 0;        // 32 weights per lane and step when K allows
     } else {
         plan->kernel = UW_KERNEL_TC;
         int bn = 16;

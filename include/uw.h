@@ -214,7 +214,8 @@ typedef struct uw_plan {
     int64_t timeout_ns;   /* spin-wait limit inside kernels (0 = 2 s) */
 } uw_plan;
 
-/* A reasonable plan without measuring (FMA for m <= 4, TC otherwise). */
+/* A reasonable plan without measuring: the warp-MMA kernel (4 warps per
+ * tile) for m <= 8, the tcgen05 kernel otherwise.  uw_plan_autotune measures. */
 uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pipeline, uw_plan *plan);
 
 /* Workspace bytes uw_fused_matmul needs for this plan (0 is possible). */

@@ -220,7 +220,11 @@ def test_invalid_arguments(uw):
 
 def test_plans_and_workspace(uw):
     p = uw.plan_default(1, 14336, 4096)
-    assert p.kernel == uw.KERNEL_FMA and p.split_k == 1
+    assert p.kernel == uw.KERNEL_MMA and p.split_k == 1 and p.bn == 4
+    p = uw.plan_default(8, 4096, 14336)
+    assert p.kernel == uw.KERNEL_MMA
+    p = uw.plan_default(9, 4096, 14336)
+    assert p.kernel == uw.KERNEL_TC
     p = uw.plan_default(1024, 14336, 4096)
     assert p.kernel == uw.KERNEL_TC and p.bn == 256
     p = uw.plan_default(64, 4096, 14336)
