@@ -212,39 +212,54 @@ def run_reference(args, rank):
 # DRAM traffic of a kernel group's launch on the 8B gate projection, from one
 # ncu capture each (profiles/k_gemv_mma_traffic_8b_gate_m1.md and
 # profiles/k_gemm_tc_traffic_8b_gate.md): bytes per launch, the algorithmic
-# bytes of that launch, and a SHA-256 over the kernel's sources; a figure is
-# reported (scaled to the group's mean algorithmic bytes per launch) only
-# while those sources are unchanged.
+# bytes of that launch, and a SHA-256 over the kernel's sources with comments
+# and whitespace removed (source_digest); a figure is reported (scaled to the
+# group's mean algorithmic bytes per launch) only while that code is unchanged.
 MEASURED_TRAFFIC = {
     "fused/tcgen05_bn64": {
         "bytes": 93612544, "alg_bytes": 94085696,
         "files": ("decode_gemm_exponent_b200/csrc/gemm_tc.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
-        "sha256": "a38dbfe44d97793da096817bfb57bfe6752dafcf2a929c5125416f4414a674f3",
+        "sha256": "278497e4e28f6a45f07770995e5484802aa2dbe40c47ac44886b387b4c4c694c",
     },
     "fused/tcgen05_bn16": {
         "bytes": 93028864, "alg_bytes": 90939968,
         "files": ("decode_gemm_exponent_b200/csrc/gemm_tc.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
-        "sha256": "a38dbfe44d97793da096817bfb57bfe6752dafcf2a929c5125416f4414a674f3",
+        "sha256": "278497e4e28f6a45f07770995e5484802aa2dbe40c47ac44886b387b4c4c694c",
     },
     "fused/mma_gemv_s4_w2": {
         "bytes": 92293888, "alg_bytes": 89956928,
         "files": ("decode_gemm_exponent_b200/csrc/gemv_mma.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
-        "sha256": "9889e4f20a5f1e4bab36c5340a2b8778dadd1f35be305a9d08eaaf4262d762cd",
+        "sha256": "d7bf659f5a3bcaa34626548b4f4cb8c0f4afbd4ff09d140765941b6a8f6d69f1",
     },
 }
 
 
+def source_digest(texts) -> str:
+    """SHA-256 over C/CUDA source texts with comments removed and every run of
+    whitespace reduced to one space, so that an edit of a comment leaves it
+    unchanged and an edit of the code does not.  String and character
+    literals are kept as written."""
+    import hashlib
+    import re
+    tok = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
+    h = hashlib.sha256()
+    for text in texts:
+        code = tok.sub(lambda mt: mt.group(0) if mt.group(0)[0] in "\"'" else " ", text)
+        h.update(" ".join(code.split()).encode())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
 def measured_traffic(group: str, alg_bytes_per_launch: float):
     """ncu DRAM bytes per launch of `group`, scaled by algorithmic bytes, or None."""
-    import hashlib
     rec = MEASURED_TRAFFIC.get(group)
     if rec is None:
         return None
-    h = hashlib.sha256()
+    texts = []
     for f in rec["files"]:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest() != rec["sha256"]:
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            texts.append(fh.read())
+    if source_digest(texts) != rec["sha256"]:
         return None
     return rec["bytes"] * alg_bytes_per_launch / rec["alg_bytes"]
 

@@ -14,22 +14,24 @@
 // without a shared-memory round trip.
 //
 // Work split: a warp tile is 16 consecutive rows of W; a CTA of S warps owns
-// one tile and splits its K into S contiguous slices of 64-weight chunks.
-// Lane (g, c) = (lane / 4, lane % 4) loads weights [16c, 16c + 16) of every
-// chunk of rows g and g + 8 (4 lanes cover a row's 64 sign/mantissa bytes).
-// A chunk's 64 K positions map onto the MMA's four K = 16 steps as: step j,
-// thread c, MMA K slots {2c, 2c+1, 2c+8, 2c+9} <- weights 16c + 4j + {0, 1,
-// 2, 3}; the X fragment uses the same map, so every product is formed exactly
-// once.  Lanes whose token is >= m load a valid X row anyway: it only feeds
-// output columns that are not stored.  Each warp keeps kStages chunks of
-// loads in flight in a register ring.  The raw-group bitmap words of the
+// one tile and splits its K into S contiguous slices of steps.  A step covers
+// 64*Q weights along K (Q = 1 or 2, the plan's width): lane (g, c) = (lane / 4,
+// lane % 4) loads weights [16Qc, 16Qc + 16Q) of the step for rows g and g + 8
+// (4 lanes cover a row's 64*Q sign/mantissa bytes).  The step's K positions
+// map onto 4*Q MMA K-steps of 16 as: K-step j, thread c, MMA K slots {2c,
+// 2c+1, 2c+8, 2c+9} <- weights 16Qc + 4j + {0, 1, 2, 3}; the X fragment uses
+// the same map, so every product is formed exactly once.  Lanes whose token
+// is >= m load a valid X row anyway: it only feeds output columns that are not
+// stored.  Each warp keeps the loads of the next steps in flight in a register
+// ring (3 steps for Q = 1, 2 for Q = 2), and prefetches each ring slot's X rows
+// into L1 when it issues the slot's loads.  The raw-group bitmap words of the
 // tile's rows and their prefix counts are staged in shared memory; each lane
-// keeps a 64-chunk window of its two rows' raw bits in registers, so a raw
-// group's exponents are fetched together with the chunk's other loads.
-// The K steps alternate between two accumulators (independent MMA chains),
-// added at the end, and the S slice results are summed in ascending slice
-// order through shared memory.  The fused and plain variants share all of
-// this but the loader, so their outputs are bit-identical.
+// keeps a 64-group window of its two rows' raw bits in registers, so a raw
+// group's exponents are fetched together with the step's other loads.
+// The MMA K-steps alternate between two accumulators (independent MMA
+// chains), added at the end, and the S slice results are summed in ascending
+// slice order through shared memory.  The fused and plain variants share all
+// of this but the loader, so their outputs are bit-identical.
 #include <algorithm>
 
 #include "device_common.cuh"

@@ -1,5 +1,5 @@
 """Host-side logic of bench.py that needs no GPU: the measured-traffic
-lookup and the plan-file round trip."""
+lookup, the source digest that keys it, and the plan-file round trip."""
 import json
 import os
 import sys
@@ -26,6 +26,16 @@ def test_measured_traffic_lookup():
     finally:
         bench.MEASURED_TRAFFIC.clear()
         bench.MEASURED_TRAFFIC.update(saved)
+
+
+def test_source_digest_ignores_comments_only():
+    src = 'int f(int a) {  // add one\n  return a + 1; /* "x" */\n}\nconst char* s = "// kept";\n'
+    d = bench.source_digest([src])
+    assert bench.source_digest([src.replace("add one", "increment")]) == d
+    assert bench.source_digest([src.replace("  return", "\n\n    return")]) == d
+    assert bench.source_digest([src.replace("a + 1", "a + 2")]) != d
+    assert bench.source_digest([src.replace('"// kept"', '"// gone"')]) != d   # literal, not a comment
+    assert bench.source_digest([src, ""]) != d                                  # file boundaries count
 
 
 def test_plans_from_json_round_trip():
