@@ -275,13 +275,17 @@ def alg_bytes(mat, m, plan):
     huff_in = common + (info.stream_bits + 7) // 8 + (info.n_chunks + 1) * 4
     if plan.pipeline == 1:
         return {"decode": huff_in + 2 * n * k, "plain": 2 * n * k + xy}
+    if plan.pipeline == 2:
+        # exponent plane + all-raw bitmap and rank words written, then read with the sm plane
+        idx = (n * k // 64) // 8 * 2
+        return {"exp_decode": huff_in + n * k + idx, "fused": 2 * n * k + idx + xy}
     return {"transcode": huff_in + n * k // 2, "fused": common + n * k // 2 + xy}
 
 
 def plans_from_json(text, n_mats, uw):
     """Plans from a plan file written by the autotuner (--plan-json)."""
     doc = json.loads(text)
-    pipes = {"decode_gemm": 1, "transcode_fused": 3, "direct_palette": 4}
+    pipes = {"decode_gemm": 1, "decode_exp_fused": 2, "transcode_fused": 3, "direct_palette": 4}
     plans = [[None] * len(MS) for _ in range(n_mats)]
     for e in doc["plans"]:
         b = e["best"]
@@ -292,7 +296,7 @@ def plans_from_json(text, n_mats, uw):
 
 
 def launches_per_call(plan):
-    n = 1 + (1 if plan.pipeline in (1, 3) else 0)
+    n = 1 + (1 if plan.pipeline in (1, 2, 3) else 0)
     if plan.kernel == 2 and plan.split_k > 1:
         n += 1
     return n
@@ -300,7 +304,7 @@ def launches_per_call(plan):
 
 def kernel_group(plan):
     kern = {1: "fma_gemv", 3: "mma_gemv_s%d_w%d" % (plan.bn, plan.stages)}.get(plan.kernel, "tcgen05_bn%d" % plan.bn)
-    pipe = {1: "decode+plain", 3: "transcode+fused", 4: "fused"}[plan.pipeline]
+    pipe = {1: "decode+plain", 2: "exp_decode+fused", 3: "transcode+fused", 4: "fused"}[plan.pipeline]
     return "%s/%s" % (pipe, kern)
 
 

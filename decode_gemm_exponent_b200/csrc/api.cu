@@ -1,5 +1,5 @@
 // api.cu -- the C ABI of libuw (declared in include/uw.h): binding a device
-// copy of a blob, kernel status, the preprocessing kernels and the matmul
+// copy of a blob, kernel status, the preprocessing kernels and the four matmul
 // pipelines of the Unweight page (§六).
 #include <algorithm>
 #include <cstring>
@@ -22,8 +22,8 @@ bool valid_bn_tc(int bn) { return bn == 16 || bn == 32 || bn == 64 || bn == 128 
 
 uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
     if (!p || k <= 0) return UW_ERR_INVALID_ARG;
-    if (p->pipeline != UW_PIPE_DECODE_GEMM && p->pipeline != UW_PIPE_TRANSCODE_FUSED &&
-        p->pipeline != UW_PIPE_DIRECT_PALETTE)
+    if (p->pipeline != UW_PIPE_DECODE_GEMM && p->pipeline != UW_PIPE_DECODE_EXP_FUSED &&
+        p->pipeline != UW_PIPE_TRANSCODE_FUSED && p->pipeline != UW_PIPE_DIRECT_PALETTE)
         return UW_ERR_INVALID_ARG;
     if (p->kernel == UW_KERNEL_FMA) {
         if (m > 8 || (p->bn != 1 && p->bn != 2) || p->split_k != 1) return UW_ERR_INVALID_ARG;
@@ -45,11 +45,7 @@ uint64_t partial_bytes(int64_t m, int64_t n, const uw_plan *p) {
     return align_up(uint64_t(p->split_k) * uint64_t(m) * uint64_t(n) * 4, 256);
 }
 
-uint64_t prep_bytes(int64_t n, int64_t k, const uw_plan *p) {
-    if (p->pipeline == UW_PIPE_DECODE_GEMM) return align_up(uint64_t(n) * uint64_t(k) * 2, 256);
-    if (p->pipeline == UW_PIPE_TRANSCODE_FUSED) return align_up(uint64_t(n) * uint64_t(k) / 2, 256);
-    return 0;
-}
+uint64_t prep_bytes(int64_t n, int64_t k, const uw_plan *p) { return prep_workspace_bytes(n, k, p->pipeline); }
 
 // Run one matmul kernel on prepared weights: w_bf16 (plain) or pal (fused).
 uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const uw_dmat *w,
@@ -165,6 +161,14 @@ extern "C" uw_status uw_decode_to_bf16(const uw_dmat *w, uint16_t *out_dev, void
     return cuda_status(launch_huff_decode(*w, out_dev, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
+extern "C" uw_status uw_decode_exponents(const uw_dmat *w, uint8_t *exp_dev, void *stream) {
+    uw_status st = check_dmat(w);
+    if (st != UW_OK) return st;
+    if (!exp_dev || !aligned(exp_dev, 16)) return UW_ERR_INVALID_ARG;
+    if (!(w->flags & UW_EMIT_HUFFMAN) || !w->stream) return UW_ERR_INVALID_ARG;
+    return cuda_status(launch_exp_decode(*w, exp_dev, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
 extern "C" uw_status uw_transcode_palette(const uw_dmat *w, uint8_t *pal_dev, void *stream) {
     uw_status st = check_dmat(w);
     if (st != UW_OK) return st;
@@ -227,6 +231,15 @@ extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_
         if (st != UW_OK) return st;
         return run_kernel(x_dev, m, wd, nullptr, nullptr, w->n, w->k, y_dev, plan, partial,
                           w->dev_status, s);
+    }
+    if (plan->pipeline == UW_PIPE_DECODE_EXP_FUSED) {
+        if (!(w->flags & UW_EMIT_HUFFMAN)) return UW_ERR_INVALID_ARG;
+        const ExpPlaneLayout L = exp_plane_layout(w->n, w->k);
+        st = cuda_status(launch_exp_decode(*w, wsb, reinterpret_cast<uint32_t *>(wsb + L.flags_off),
+                                           reinterpret_cast<uint32_t *>(wsb + L.rank_off), s));
+        if (st != UW_OK) return st;
+        const uw_dmat v = exp_plane_view(*w, wsb);
+        return run_kernel(x_dev, m, nullptr, &v, v.pal, w->n, w->k, y_dev, plan, partial, w->dev_status, s);
     }
     const uint8_t *pal = nullptr;
     if (plan->pipeline == UW_PIPE_TRANSCODE_FUSED) {

@@ -3,8 +3,9 @@
 // GPU for every projection and batch size and writes a per-model plan file).
 //
 // For each matrix and each batch size m the candidates are the pipelines the
-// blob supports (decode + plain kernel, runtime transcode + fused kernel,
-// direct palette + fused kernel) crossed with the kernel variants: the
+// blob supports (decode + plain kernel, exponent decode + fused kernel,
+// runtime transcode + fused kernel, direct palette + fused kernel) crossed
+// with the kernel variants: the
 // warp-MMA kernel (m <= 16, 2-8 K slices per tile, 16 or 32 weights per lane
 // and step), the FMA GEMV (m <= 8, 1 or 2 rows per warp) and the tcgen05
 // kernel with token tiles around m and split-K factors 1-8 (so that some
@@ -43,6 +44,7 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
     std::vector<int> pipes;
     if (w.flags & UW_EMIT_HUFFMAN) {
         pipes.push_back(UW_PIPE_DECODE_GEMM);
+        pipes.push_back(UW_PIPE_DECODE_EXP_FUSED);
         pipes.push_back(UW_PIPE_TRANSCODE_FUSED);
     }
     if ((w.flags & UW_EMIT_PALETTE) && w.pal) pipes.push_back(UW_PIPE_DIRECT_PALETTE);
@@ -92,8 +94,12 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
 }
 
 const char *pipe_name(int p) {
-    return p == UW_PIPE_DECODE_GEMM ? "decode_gemm" : p == UW_PIPE_TRANSCODE_FUSED ? "transcode_fused"
-                                                                                 : "direct_palette";
+    switch (p) {
+        case UW_PIPE_DECODE_GEMM: return "decode_gemm";
+        case UW_PIPE_DECODE_EXP_FUSED: return "decode_exp_fused";
+        case UW_PIPE_TRANSCODE_FUSED: return "transcode_fused";
+        default: return "direct_palette";
+    }
 }
 
 std::string plan_json(const uw_plan &p, double us) {

@@ -1,6 +1,7 @@
 // decode.cu -- Huffman exponent decoding on sm_100a (Unweight page §六:
-// pipeline 1 rebuilds full BF16 weights in HBM; pipeline 3 transcodes the
-// Huffman stream to 4-bit palette indices at run time).
+// pipeline 1 rebuilds full BF16 weights in HBM; pipeline 2 writes only the
+// exponent bytes; pipeline 3 transcodes the Huffman stream to 4-bit palette
+// indices at run time).
 //
 // One CTA of 256 threads owns a tile of 256 chunks (1024 groups, 65536
 // weights); three CTAs fit on an SM.
@@ -19,8 +20,9 @@
 //      exactly where the next one starts and must not touch a window with no
 //      valid code, otherwise the corrupt bit is raised.
 //   3. The tile is written with coalesced 16-byte accesses: palette words in
-//      the stored 4-bit layout (transcode), or BF16 = palette exponent (or
-//      raw-plane exponent) joined with the sign/mantissa byte (decode).
+//      the stored 4-bit layout (transcode), exponent bytes (exponent decode),
+//      or BF16 = palette exponent (or raw-plane exponent) joined with the
+//      sign/mantissa byte (decode).
 #include "device_common.cuh"
 #include "kernels.h"
 #include "uw_format.h"
@@ -39,6 +41,11 @@ constexpr int kChunkWords = kChunkGroups * kGroup / 8;    // 32 symbol words per
 constexpr int kPrefetch = 8;                              // sm vectors in flight per thread
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
+// what the write phase produces
+constexpr int kOutBf16 = 0;   // BF16 weights [n*k]
+constexpr int kOutPal = 1;    // 4-bit palette plane [n*k/2]
+constexpr int kOutExp = 2;    // exponent bytes [n*k]
+
 struct DecodeArgs {
     const uint32_t *stream;
     const uint32_t *chunk_off;
@@ -51,9 +58,13 @@ struct DecodeArgs {
     uint64_t stream_bits;
     uint64_t code_len;          // code length of palette index s in bits 4s..4s+3
     int64_t n_groups, n_chunks;
-    Palette16 pal;
+    Palette16 pal;              // rotr8 of the palette exponents (BF16 rebuild)
+    Palette16 pal_nat;          // the palette exponents themselves
     uint16_t *out_bf16;
     uint32_t *out_pal;
+    uint8_t *out_exp;
+    uint32_t *out_flags;        // exponent decode: all-raw bitmap (may be null)
+    uint32_t *out_rank;         // exponent decode: its rank bases (with out_flags)
     uint32_t *status;
 };
 
@@ -180,7 +191,7 @@ __device__ __forceinline__ bool decode_chunk(const Src src, uint32_t p, uint32_t
     return rem4 == 0 && p == end && !(err & kLutInvalid);
 }
 
-template <bool TO_PAL>
+template <int OUT>
 __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(smem_raw);
@@ -194,6 +205,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
     if (tid < kFlagWords) {
         const int64_t wi = g_begin / 32 + tid;
         S.flags[tid] = (wi * 32 < g_end) ? a.flagbits[wi] : 0u;
+        if (OUT == kOutExp && a.out_flags && wi * 32 < g_end) {
+            const int64_t left = g_end - wi * 32;
+            a.out_flags[wi] = left >= 32 ? ~0u : (1u << left) - 1u;
+            a.out_rank[wi] = uint32_t(wi * 32);
+        }
     }
     if (tid == 0) {
         const bool bad = b_end < b_begin || uint64_t(b_end) > a.stream_bits;
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
     const uint32_t start = has_chunk ? a.chunk_off[c] : 0u;
     const uint32_t end = has_chunk ? a.chunk_off[c + 1] : 0u;
     uint4 smv[kPrefetch];
-    if (!TO_PAL) {
+    if (OUT == kOutBf16) {
 #pragma unroll
         for (int u = 0; u < kPrefetch; u++) {
             const int i = u * kThreads + tid;   // same item numbering as the write phase
@@ -265,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
     // the group's position inside its flag word and chunk, and its chunk's
     // rotation, are the same for all of a thread's items.  Group lg's symbols
     // follow the chunk's non-raw groups below it.
-    if (TO_PAL) {
+    if (OUT == kOutPal) {
         // item = half a group (32 weights, 4 palette words): group it*128 + tid/2
         constexpr int kItems = kTileGroups * 2 / kThreads;
         const int half = tid & 1, lg0 = tid >> 1;
@@ -288,6 +304,36 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
                                natural_to_pal(n1.y));
             }
             __stcs(out4 + int64_t(it) * kThreads, v);
+        }
+    } else if (OUT == kOutExp) {
+        // item = a quarter group (16 exponent bytes): group it * 64 + tid/4,
+        // numbered as in the BF16 layout below
+        constexpr int kItems = kTileGroups * 4 / kThreads;
+        constexpr int kGroupsPerStep = kThreads / 4;
+        const int q = tid & 3, lg0 = tid >> 2;
+        const uint32_t bit = uint32_t(lg0 & 31), in_chunk = uint32_t(lg0 & 3);
+        const uint32_t below = ((1u << bit) - 1u) & ~((1u << (bit & 28u)) - 1u);
+        const uint32_t sym0 = smem_addr(S.sym) + 4u * uint32_t((lg0 >> 2) * kChunkWords);
+        const uint32_t rot = sym_rot(uint32_t(lg0 >> 2)) + uint32_t(q) * 2u;
+        const int64_t e0 = (g_begin + lg0) * kGroup + q * 16;   // first byte of the first item
+        const int64_t live = g_end - g_begin - lg0;             // items it with it * 64 < live exist
+#pragma unroll 4
+        for (int it = 0; it < kItems; it++) {
+            if (it * kGroupsPerStep >= live) break;
+            const int lg = it * kGroupsPerStep + lg0;
+            const uint32_t fw = S.flags[lg >> 5];
+            uint4 v;
+            if ((fw >> bit) & 1u) {
+                const int64_t g = g_begin + lg;
+                const uint32_t rank = a.rawbase[g >> 5] + __popc(fw & ((1u << bit) - 1u));
+                v = __ldcs(reinterpret_cast<const uint4 *>(a.rawexp + uint64_t(rank) * kGroup + q * 16));
+            } else {
+                const uint32_t k = ((in_chunk - __popc(fw & below)) * 8u + rot) & 31u;
+                const uint2 nw = lds64(sym0 + uint32_t(it) * (kGroupsPerStep / 4) * kChunkWords * 4u + 4u * k);
+                nat_rot(nw.x, a.pal_nat, v.x, v.y);
+                nat_rot(nw.y, a.pal_nat, v.z, v.w);
+            }
+            __stcs(reinterpret_cast<uint4 *>(a.out_exp + e0 + int64_t(it) * kGroupsPerStep * kGroup), v);
         }
     } else {
         // item = a quarter group (16 weights): group (it0 + u) * 64 + tid/4.
@@ -338,9 +384,20 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
 
 }  // namespace
 
-cudaError_t launch_huff_decode(const uw_dmat &w, uint16_t *out_bf16, uint8_t *out_pal,
-                               cudaStream_t stream) {
-    DecodeArgs a;
+namespace {
+
+// The palette exponents as bytes, 4 per word (the lookup table of the
+// exponent decode; the BF16 decode uses their rotr8 form, make_palette16).
+Palette16 make_palette16_natural(const uint8_t palette[16]) {
+    auto word = [&](int i) {
+        return uint32_t(palette[i]) | uint32_t(palette[i + 1]) << 8 | uint32_t(palette[i + 2]) << 16 |
+               uint32_t(palette[i + 3]) << 24;
+    };
+    return Palette16{word(0), word(4), word(8), word(12)};
+}
+
+DecodeArgs decode_args(const uw_dmat &w) {
+    DecodeArgs a{};
     a.stream = w.stream;
     a.stream_words = w.stream_words;
     a.stream_bits = w.stream_bits;
@@ -355,27 +412,45 @@ cudaError_t launch_huff_decode(const uw_dmat &w, uint16_t *out_bf16, uint8_t *ou
     a.n_groups = w.n_groups;
     a.n_chunks = w.n_chunks;
     a.pal = make_palette16(w.palette);
-    a.out_bf16 = out_bf16;
-    a.out_pal = reinterpret_cast<uint32_t *>(out_pal);
+    a.pal_nat = make_palette16_natural(w.palette);
     a.status = w.dev_status;
-    const unsigned grid = unsigned((w.n_chunks + kTileChunks - 1) / kTileChunks);
+    return a;
+}
+
+template <int OUT>
+cudaError_t launch_mode(const DecodeArgs &a, cudaStream_t stream) {
+    const unsigned grid = unsigned((a.n_chunks + kTileChunks - 1) / kTileChunks);
     const size_t smem = sizeof(DecodeSmem);
-    static thread_local int ready_dev[2] = {-1, -1};   // shared-memory opt-in done on device
+    static thread_local int ready_dev = -1;   // shared-memory opt-in done on this device
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    const int which = out_pal ? 1 : 0;
-    if (ready_dev[which] != dev) {
-        err = out_pal ? cudaFuncSetAttribute(k_huff_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem))
-                      : cudaFuncSetAttribute(k_huff_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem));
+    if (ready_dev != dev) {
+        err = cudaFuncSetAttribute(k_huff_decode<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (err != cudaSuccess) return err;
-        ready_dev[which] = dev;
+        ready_dev = dev;
     }
-    if (out_pal) k_huff_decode<true><<<grid, kThreads, smem, stream>>>(a);
-    else k_huff_decode<false><<<grid, kThreads, smem, stream>>>(a);
+    k_huff_decode<OUT><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_huff_decode(const uw_dmat &w, uint16_t *out_bf16, uint8_t *out_pal,
+                               cudaStream_t stream) {
+    DecodeArgs a = decode_args(w);
+    a.out_bf16 = out_bf16;
+    a.out_pal = reinterpret_cast<uint32_t *>(out_pal);
+    return out_pal ? launch_mode<kOutPal>(a, stream) : launch_mode<kOutBf16>(a, stream);
+}
+
+cudaError_t launch_exp_decode(const uw_dmat &w, uint8_t *out_exp, uint32_t *all_raw_flags,
+                              uint32_t *all_raw_rank, cudaStream_t stream) {
+    DecodeArgs a = decode_args(w);
+    a.out_exp = out_exp;
+    a.out_flags = all_raw_rank ? all_raw_flags : nullptr;
+    a.out_rank = all_raw_rank;
+    return launch_mode<kOutExp>(a, stream);
 }
 
 }  // namespace uw

@@ -14,6 +14,57 @@ namespace uw {
 cudaError_t launch_huff_decode(const uw_dmat &w, uint16_t *out_bf16, uint8_t *out_pal,
                                cudaStream_t stream);
 
+// Exponent-only Huffman decode (Unweight page §六, pipeline 2): every
+// weight's exponent byte, uint8 [n*k] in weight order.  When all_raw_flags and
+// all_raw_rank are non-null (n*k/2048 words each) the kernel also writes the
+// raw-group bitmap and per-word rank bases of a layout in which every group is
+// raw: all bits set, word i's base 32*i.  With those, group g's raw rank is g,
+// and the raw plane at byte 64*rank is exactly the exponent plane, so the
+// fused kernels read it through their raw-group path (exp_plane_view).
+cudaError_t launch_exp_decode(const uw_dmat &w, uint8_t *out_exp, uint32_t *all_raw_flags,
+                              uint32_t *all_raw_rank, cudaStream_t stream);
+
+// Pipeline 2's workspace: the exponent plane, then the all-raw bitmap and
+// rank bases, each 256-byte aligned.
+struct ExpPlaneLayout {
+    uint64_t flags_off, rank_off, bytes;
+};
+inline ExpPlaneLayout exp_plane_layout(int64_t n, int64_t k) {
+    const auto up = [](uint64_t x) { return (x + 255u) / 256u * 256u; };
+    const uint64_t plane = uint64_t(n) * uint64_t(k);
+    const uint64_t words = (plane / 64 + 31) / 32;
+    ExpPlaneLayout L;
+    L.flags_off = up(plane);
+    L.rank_off = L.flags_off + up(words * 4);
+    L.bytes = L.rank_off + up(words * 4);
+    return L;
+}
+
+// The matrix as pipeline 2's fused matmul sees it: sign/mantissa plane of
+// `w`, every group raw, the exponent plane in `slot` (laid out as above) as
+// the raw plane.  The palette plane pointer is set to the exponent plane too:
+// kernels that stage the palette plane unconditionally then read n*k/2 valid
+// bytes whose values no raw group uses.
+inline uw_dmat exp_plane_view(const uw_dmat &w, uint8_t *slot) {
+    const ExpPlaneLayout L = exp_plane_layout(w.n, w.k);
+    uw_dmat v = w;
+    v.rawexp = slot;
+    v.flagbits = reinterpret_cast<const uint32_t *>(slot + L.flags_off);
+    v.rawbase = reinterpret_cast<const uint32_t *>(slot + L.rank_off);
+    v.n_raw = w.n_groups;
+    v.pal = slot;
+    return v;
+}
+
+// Workspace bytes of a pipeline's preprocessing output (0 for pipeline 4).
+inline uint64_t prep_workspace_bytes(int64_t n, int64_t k, int32_t pipeline) {
+    const uint64_t nk = uint64_t(n) * uint64_t(k);
+    if (pipeline == UW_PIPE_DECODE_GEMM) return (nk * 2 + 255u) / 256u * 256u;
+    if (pipeline == UW_PIPE_DECODE_EXP_FUSED) return exp_plane_layout(n, k).bytes;
+    if (pipeline == UW_PIPE_TRANSCODE_FUSED) return (nk / 2 + 255u) / 256u * 256u;
+    return 0;
+}
+
 // CUDA-core FMA GEMV, m <= 8 (Unweight page §七, small-batch case).
 // pal_plane == nullptr: plain BF16 weights `w_bf16`; otherwise the fused
 // palette path using `w` (sm/raw planes) and `pal_plane`.  One warp per

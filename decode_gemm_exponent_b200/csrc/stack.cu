@@ -5,8 +5,9 @@
 //
 // Every step's matmul runs on the main stream, in step order, so a step may
 // read what an earlier step wrote.  A step whose plan needs preprocessing
-// (pipeline 1: full decode to BF16; pipeline 3: transcode to the 4-bit
-// plane) has it issued on the side stream into one of two workspace slots,
+// (pipeline 1: full decode to BF16; pipeline 2: exponent-only decode;
+// pipeline 3: transcode to the 4-bit plane) has it issued on the side stream
+// into one of two workspace slots,
 // as soon as the slot's previous user has finished; its matmul then waits for
 // that preprocessing.  So the decode of step i+1 (or i+2) runs while the main
 // stream is still busy with step i.  Preprocessing reads only the weights,
@@ -29,7 +30,8 @@ namespace uw {
 namespace {
 
 inline bool needs_prep(const uw_plan &p) {
-    return p.pipeline == UW_PIPE_DECODE_GEMM || p.pipeline == UW_PIPE_TRANSCODE_FUSED;
+    return p.pipeline == UW_PIPE_DECODE_GEMM || p.pipeline == UW_PIPE_DECODE_EXP_FUSED ||
+           p.pipeline == UW_PIPE_TRANSCODE_FUSED;
 }
 
 struct StackLayout {
@@ -47,9 +49,7 @@ uw_status layout(const uw_stack_step *steps, int n_steps, StackLayout &L) {
         size_t all = 0;
         uw_status st = uw_workspace_size(s.m, s.w->n, s.w->k, &s.plan, &all);
         if (st != UW_OK) return st;
-        uint64_t prep = 0;
-        if (s.plan.pipeline == UW_PIPE_DECODE_GEMM) prep = align_up(uint64_t(s.w->n) * uint64_t(s.w->k) * 2, 256);
-        if (s.plan.pipeline == UW_PIPE_TRANSCODE_FUSED) prep = align_up(uint64_t(s.w->n) * uint64_t(s.w->k) / 2, 256);
+        const uint64_t prep = prep_workspace_bytes(s.w->n, s.w->k, s.plan.pipeline);
         L.slot_bytes = std::max(L.slot_bytes, prep);
         L.partial_bytes = std::max(L.partial_bytes, uint64_t(all) - prep);
     }
@@ -134,10 +134,17 @@ extern "C" uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void 
             st = UW_ERR_CUDA;
             break;
         }
-        if (s.plan.pipeline == UW_PIPE_DECODE_GEMM)
+        if (s.plan.pipeline == UW_PIPE_DECODE_GEMM) {
             st = uw_decode_to_bf16(w, reinterpret_cast<uint16_t *>(slot[b]), prep_s);
-        else
+        } else if (s.plan.pipeline == UW_PIPE_DECODE_EXP_FUSED) {
+            const ExpPlaneLayout EL = exp_plane_layout(w->n, w->k);
+            st = launch_exp_decode(*w, slot[b], reinterpret_cast<uint32_t *>(slot[b] + EL.flags_off),
+                                   reinterpret_cast<uint32_t *>(slot[b] + EL.rank_off), prep_s) == cudaSuccess
+                     ? UW_OK
+                     : UW_ERR_CUDA;
+        } else {
             st = uw_transcode_palette(w, slot[b], prep_s);
+        }
         if (st != UW_OK) break;
         if (overlap && (cudaEventRecord(E.ev[b], side_s) != cudaSuccess ||
                         cudaStreamWaitEvent(main_s, E.ev[b], 0) != cudaSuccess)) {
@@ -148,9 +155,12 @@ extern "C" uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void 
             st = uw_matmul_bf16(s.x_dev, s.m, reinterpret_cast<const uint16_t *>(slot[b]), w->n, w->k, s.y_dev,
                                 &s.plan, partial, L.partial_bytes, w->dev_status, main_s);
         } else {
+            // pipeline 3: the fused kernel on the transcoded plane; pipeline 2:
+            // on the all-raw view whose raw plane is the decoded exponents
             uw_plan p = s.plan;
             p.pipeline = UW_PIPE_DIRECT_PALETTE;
-            st = uw_fused_matmul(s.x_dev, s.m, w, slot[b], s.y_dev, &p, partial, L.partial_bytes, main_s);
+            const uw_dmat v = s.plan.pipeline == UW_PIPE_DECODE_EXP_FUSED ? exp_plane_view(*w, slot[b]) : *w;
+            st = uw_fused_matmul(s.x_dev, s.m, &v, slot[b], s.y_dev, &p, partial, L.partial_bytes, main_s);
         }
         if (st == UW_OK && overlap && cudaEventRecord(E.ev[2 + b], main_s) != cudaSuccess) st = UW_ERR_CUDA;
         n_prep++;

@@ -2,7 +2,8 @@
 
     python -m decode_gemm_exponent_b200.profile_case --kernel fma --n 28672 --k 8192 --m 1
 
-kernels: decode, transcode (Huffman stream -> BF16 / 4-bit palette),
+kernels: decode, exp_decode, transcode (Huffman stream -> BF16 / exponent
+bytes / 4-bit palette),
 fma, tc (fused palette matmul, CUDA-core GEMV or tcgen05), plain_fma,
 plain_tc (the same kernels on BF16 weights).  One warm-up launch is followed
 by --reps timed launches (CUDA events); the per-launch time and the
@@ -22,7 +23,7 @@ from . import synth, uw
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", required=True,
-                    choices=["decode", "transcode", "fma", "tc", "mma", "plain_fma", "plain_tc", "plain_mma"])
+                    choices=["decode", "exp_decode", "transcode", "fma", "tc", "mma", "plain_fma", "plain_tc", "plain_mma"])
     ap.add_argument("--n", type=int, default=28672)
     ap.add_argument("--k", type=int, default=8192)
     ap.add_argument("--m", type=int, default=1)
@@ -55,13 +56,18 @@ def main(argv=None):
         plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, a.bn or 2, 1, a.stages)
     else:
         plan = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, a.bn or 16, a.split, a.stages)
-    ws_bytes = uw.workspace_size(a.m, a.n, a.k, plan) if a.kernel not in ("decode", "transcode") else 0
+    preprocessing = a.kernel in ("decode", "exp_decode", "transcode")
+    ws_bytes = 0 if preprocessing else uw.workspace_size(a.m, a.n, a.k, plan)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
     wd = None
     if a.kernel == "decode":
         out = torch.empty(a.n, a.k, dtype=torch.int16, device="cuda")
         run = lambda: mat.decode(out)
         alg = huff_in + 2 * nk
+    elif a.kernel == "exp_decode":
+        out = torch.empty(a.n, a.k, dtype=torch.uint8, device="cuda")
+        run = lambda: mat.decode_exponents(out)
+        alg = huff_in + nk
     elif a.kernel == "transcode":
         out = torch.empty(nk // 2, dtype=torch.uint8, device="cuda")
         run = lambda: mat.transcode(out)
@@ -97,8 +103,7 @@ def main(argv=None):
         us = 1e3 * e0.elapsed_time(e1) / a.reps
     print(json.dumps({"kernel": a.kernel, "n": a.n, "k": a.k, "m": a.m, "bn": plan.bn,
                       "split": plan.split_k, "us": us, "alg_bytes": int(alg),
-                      "gbs": alg / us / 1e3, "tflops": flops / us / 1e6 if "decode" not in a.kernel
-                      and "transcode" not in a.kernel else None,
+                      "gbs": alg / us / 1e3, "tflops": None if preprocessing else flops / us / 1e6,
                       "l2": "flushed before each call" if a.flush else
                       "not flushed (a matrix under 126 MB stays in L2 between calls)"}))
 

@@ -29,14 +29,14 @@ EMIT_HUFFMAN = 1
 EMIT_PALETTE = 2
 SEC_SM, SEC_RAWEXP, SEC_FLAGS, SEC_RAWBASE, SEC_STREAM, SEC_CHUNKOFF, SEC_DLUT, SEC_PAL = range(8)
 NUM_SECTIONS = 8
-PIPE_DECODE_GEMM, PIPE_TRANSCODE_FUSED, PIPE_DIRECT_PALETTE = 1, 3, 4
+PIPE_DECODE_GEMM, PIPE_DECODE_EXP_FUSED, PIPE_TRANSCODE_FUSED, PIPE_DIRECT_PALETTE = 1, 2, 3, 4
 KERNEL_FMA, KERNEL_TC, KERNEL_MMA = 1, 2, 3
 DEBUG_NEVER_ARRIVE = 1
 
 # every symbol include/uw.h declares
 EXPORTS = ("uw_status_str", "uw_version", "uw_encode", "uw_blob_data", "uw_blob_free",
            "uw_blob_info_get", "uw_matrix_bind", "uw_device_status", "uw_decode_to_bf16",
-           "uw_transcode_palette", "uw_plan_default", "uw_workspace_size", "uw_fused_matmul",
+           "uw_decode_exponents", "uw_transcode_palette", "uw_plan_default", "uw_workspace_size", "uw_fused_matmul",
            "uw_matmul_bf16", "uw_autotune_workspace_size", "uw_plan_autotune",
            "uw_fused_matmul_noalloc", "uw_stack_workspace_size", "uw_stack_run")
 
@@ -116,6 +116,7 @@ def lib() -> ctypes.CDLL:
         "uw_matrix_bind": (ctypes.c_int, [P, SZ, P, P, ctypes.c_int, ctypes.POINTER(DMat)]),
         "uw_device_status": (ctypes.c_int, [ctypes.POINTER(DMat), P]),
         "uw_decode_to_bf16": (ctypes.c_int, [ctypes.POINTER(DMat), P, P]),
+        "uw_decode_exponents": (ctypes.c_int, [ctypes.POINTER(DMat), P, P]),
         "uw_transcode_palette": (ctypes.c_int, [ctypes.POINTER(DMat), P, P]),
         "uw_plan_default": (ctypes.c_int, [I64, I64, I64, I32, ctypes.POINTER(Plan)]),
         "uw_workspace_size": (ctypes.c_int, [I64, I64, I64, ctypes.POINTER(Plan), ctypes.POINTER(SZ)]),
@@ -221,6 +222,15 @@ class Matrix:
               "uw_decode_to_bf16")
         return out
 
+    def decode_exponents(self, out=None, stream=None):
+        """Exponent byte of every weight, uint8 [n, k]."""
+        import torch
+        if out is None:
+            out = torch.empty(self.n, self.k, dtype=torch.uint8, device=self.dev.device)
+        check(lib().uw_decode_exponents(ctypes.byref(self.dmat), _ptr(out), _stream_handle(stream)),
+              "uw_decode_exponents")
+        return out
+
     def transcode(self, out=None, stream=None):
         import torch
         if out is None:
@@ -266,8 +276,8 @@ def fused_matmul_noalloc(mat: "Matrix", x, plan: Plan, y=None, stream=None):
 
 class Stack:
     """A fixed sequence of matmuls run by uw_stack_run: matmuls in order on the
-    main stream, decodes / transcodes of pipeline-1 / pipeline-3 steps on a
-    side stream ahead of their matmuls (cross-layer overlap).
+    main stream, the decodes / transcodes of pipeline 1-3 steps on a side
+    stream ahead of their matmuls (cross-layer overlap).
 
     steps: (Matrix, x, y, plan) tuples, or (Matrix, x, y, plan, pal) for a
     pipeline-4 step with its own palette plane.  The tensors are kept alive

@@ -166,11 +166,17 @@ uw_status uw_matrix_bind(const void *host_blob, size_t bytes, const void *dev_bl
 uw_status uw_device_status(const uw_dmat *w, void *stream);
 
 /* ------------------------------------------------------------------------ */
-/* Preprocessing kernels (Unweight page §六, pipelines 1 and 3).              */
+/* Preprocessing kernels (Unweight page §六, pipelines 1, 2 and 3).           */
 
 /* Full Huffman decode to BF16: out_dev is uint16[n*k] (caller-owned, device,
  * 16-byte aligned).  Needs UW_EMIT_HUFFMAN.  Bit-exact inverse of uw_encode. */
 uw_status uw_decode_to_bf16(const uw_dmat *w, uint16_t *out_dev, void *stream);
+
+/* Exponent-only Huffman decode: exp_dev is uint8[n*k] (device, 16-byte
+ * aligned) and receives every weight's exponent byte, (bits >> 7) & 0xFF, in
+ * weight order (raw groups included), i.e. half the bytes of a full decode.
+ * Needs UW_EMIT_HUFFMAN.                                                      */
+uw_status uw_decode_exponents(const uw_dmat *w, uint8_t *exp_dev, void *stream);
 
 /* Runtime transcode of the Huffman stream to the 4-bit palette plane:
  * pal_dev is uint8[n*k/2] (device, 16-byte aligned), byte-identical to the
@@ -182,6 +188,9 @@ uw_status uw_transcode_palette(const uw_dmat *w, uint8_t *pal_dev, void *stream)
 
 typedef enum uw_pipeline {
     UW_PIPE_DECODE_GEMM = 1,      /* decode to BF16 in the workspace, then the plain kernel */
+    UW_PIPE_DECODE_EXP_FUSED = 2, /* decode only the exponents (n*k bytes) into the
+                                     workspace, then the fused kernel rebuilding BF16
+                                     from the sign/mantissa and exponent bytes      */
     UW_PIPE_TRANSCODE_FUSED = 3,  /* transcode to the palette plane in the workspace, then
                                      the fused kernel                                    */
     UW_PIPE_DIRECT_PALETTE = 4    /* fused kernel on the blob's (or a given) palette plane */
@@ -218,7 +227,11 @@ typedef struct uw_plan {
  * tile) for m <= 8, the tcgen05 kernel otherwise.  uw_plan_autotune measures. */
 uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pipeline, uw_plan *plan);
 
-/* Workspace bytes uw_fused_matmul needs for this plan (0 is possible). */
+/* Workspace bytes uw_fused_matmul needs for this plan (0 is possible): the
+ * preprocessing output (pipeline 1: 2nk bytes of BF16; pipeline 2: the nk-byte
+ * exponent plane plus two nk/2048-word index arrays; pipeline 3: nk/2 bytes;
+ * pipeline 4: none), each part rounded up to 256 bytes, plus split_k*m*n
+ * floats of partial sums for a TC plan with split_k > 1.                     */
 uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw_plan *plan,
                             size_t *bytes);
 
@@ -301,12 +314,12 @@ typedef struct uw_stack_step {
 } uw_stack_step;
 
 /* Workspace of uw_stack_run: two preprocessing slots, each the largest
- * decode (2nk bytes) or transcode (nk/2 bytes) buffer of the stack, plus the
- * largest split-K scratch of any step.                                       */
+ * preprocessing buffer of the stack (decode 2nk bytes, exponent decode a bit
+ * over nk, transcode nk/2), plus the largest split-K scratch of any step.    */
 uw_status uw_stack_workspace_size(const uw_stack_step *steps, int n_steps, size_t *bytes);
 
-/* Run the steps in order on `stream`.  The decode (pipeline 1) or transcode
- * (pipeline 3) of a step is issued on `side_stream` into one of the two
+/* Run the steps in order on `stream`.  The decode (pipelines 1 and 2) or
+ * transcode (pipeline 3) of a step is issued on `side_stream` into one of the two
  * workspace slots as soon as that slot is free, so it overlaps the matmuls
  * of the steps before it; the step's matmul waits for it.  Each step's result
  * is bit-identical to uw_fused_matmul with the same plan.  A step may read

@@ -42,10 +42,12 @@ def test_plans_from_json_round_trip():
     from decode_gemm_exponent_b200 import uw
     doc = {"plans": []}
     kinds = [("fma", 1, 1, 0), ("tc", 64, 4, 0), ("mma", 4, 1, 2)]
+    pipes = [("decode_gemm", uw.PIPE_DECODE_GEMM), ("decode_exp_fused", uw.PIPE_DECODE_EXP_FUSED),
+             ("transcode_fused", uw.PIPE_TRANSCODE_FUSED), ("direct_palette", uw.PIPE_DIRECT_PALETTE)]
     for i in range(3):
         for j, m in enumerate(bench.MS):
             kern, bn, split, stages = kinds[(i + j) % 3]
-            doc["plans"].append({"matrix": i, "m": m, "best": {"pipeline": "direct_palette", "kernel": kern,
+            doc["plans"].append({"matrix": i, "m": m, "best": {"pipeline": pipes[(i + 2 * j) % 4][0], "kernel": kern,
                                                                 "bn": bn, "split_k": split, "stages": stages}})
     plans = bench.plans_from_json(json.dumps(doc), 3, uw)
     for i in range(3):
@@ -53,4 +55,7 @@ def test_plans_from_json_round_trip():
             kern, bn, split, stages = kinds[(i + j) % 3]
             p = plans[i][j]
             assert p.kernel == {"fma": 1, "tc": 2, "mma": 3}[kern] and p.bn == bn and p.split_k == split
-            assert p.stages == stages and p.pipeline == uw.PIPE_DIRECT_PALETTE
+            assert p.stages == stages and p.pipeline == pipes[(i + 2 * j) % 4][1]
+            # every plan has a kernel group and a launch count; pipelines 1-3 add a preprocessing launch
+            assert bench.kernel_group(p).split("/")[0]
+            assert bench.launches_per_call(p) >= (2 if p.pipeline != uw.PIPE_DIRECT_PALETTE else 1)

@@ -61,14 +61,21 @@ DECODE_CASES = {
 }
 
 
+def exponents(w: np.ndarray) -> np.ndarray:
+    # the exponent field of BF16 bit patterns (1 sign, 8 exponent, 7 mantissa bits)
+    return ((w.astype(np.uint16) >> 7) & 0xFF).astype(np.uint8)
+
+
 @pytest.mark.parametrize("case", list(DECODE_CASES))
 def test_decode_and_transcode_bit_exact(uw, case):
     w = DECODE_CASES[case]()
     m = uw.Matrix(uw.encode(w), verify_payload=True)
     d = m.decode()
     p = m.transcode()
+    e = m.decode_exponents()
     assert m.device_status() == 0
     assert np.array_equal(host16(d), w)
+    assert np.array_equal(e.cpu().numpy(), exponents(w))
     ref = O.encode(w)
     assert np.array_equal(p.cpu().numpy(), ref.pal_plane)
     assert np.array_equal(O.decode(ref), w)
@@ -79,6 +86,7 @@ def test_decode_transcode_full_size_8b_gate(uw):
     w = synth.weights_bf16(14336, 4096, 0.02, 0.0005, 1.0, seed=1)
     m = uw.Matrix(uw.encode(w))
     assert np.array_equal(host16(m.decode()), w)
+    assert np.array_equal(m.decode_exponents().cpu().numpy(), exponents(w))
     ref = O.encode(w)
     assert np.array_equal(m.transcode().cpu().numpy(), ref.pal_plane)
     assert m.device_status() == 0
@@ -94,6 +102,8 @@ def test_corrupt_device_stream_is_reported(uw):
     m.dev[off:off + 8] ^= 0x5A
     m.decode()
     assert m.device_status() == 3          # UW_ERR_CORRUPT
+    m.decode_exponents()
+    assert m.device_status() == 3
     # the context stays usable and a clean matrix still decodes
     m2 = uw.Matrix(blob)
     assert np.array_equal(host16(m2.decode()), w) and m2.device_status() == 0
@@ -101,7 +111,7 @@ def test_corrupt_device_stream_is_reported(uw):
 
 # ---------------------------------------------------------------- matmul
 
-def _matmul_case(uw, n, k, m, plan_kw, seed=0, frac=0.002, pipelines=(1, 3, 4)):
+def _matmul_case(uw, n, k, m, plan_kw, seed=0, frac=0.002, pipelines=(1, 2, 3, 4)):
     w = synth.weights_bf16(n, k, 0.02, frac, 1.0, seed=seed)
     x = synth.activations_bf16(m, k, seed=seed)
     mat = uw.Matrix(uw.encode(w))
@@ -186,8 +196,9 @@ def test_tc_stage_depth_does_not_change_bits(uw):
                                        (64, dict(kernel=2, bn=64, split_k=2)),
                                        (1024, dict(kernel=2, bn=256, split_k=1))])
 def test_full_size_8b_sampled(uw, m, plan_kw):
-    """8B gate shape at the bench's launch configurations: fused == plain bit
-    for bit, and 512 sampled outputs within the bound of the oracle."""
+    """8B gate shape at the bench's launch configurations: fused (palette and
+    exponent-plane pipelines) == plain bit for bit, and 512 sampled outputs
+    within the bound of the oracle."""
     n, k = 14336, 4096
     w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1)
     x = synth.activations_bf16(m, k, seed=1)
@@ -196,8 +207,10 @@ def test_full_size_8b_sampled(uw, m, plan_kw):
     plan = uw.make_plan(pipeline=4, **plan_kw)
     yf = mat.matmul(xd, plan).cpu().numpy()
     yp = uw.matmul_bf16(xd, wd, plan).cpu().numpy()
+    ye = mat.matmul(xd, uw.make_plan(pipeline=uw.PIPE_DECODE_EXP_FUSED, **plan_kw)).cpu().numpy()
     assert mat.device_status() == 0
     assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32))
+    assert np.array_equal(ye.view(np.uint32), yp.view(np.uint32))
     rng = np.random.default_rng(0)
     ri = rng.integers(0, m, 512)
     rj = rng.integers(0, n, 512)
@@ -217,6 +230,7 @@ def test_70b_k_outlier_and_sigma_sweep(uw, frac, sigma):
     w = synth.weights_bf16(n, k, sigma, frac, 1.0, seed=int(1000 * sigma) + int(1e4 * frac))
     mat = uw.Matrix(uw.encode(w))
     assert np.array_equal(host16(mat.decode()), w)
+    assert np.array_equal(mat.decode_exponents().cpu().numpy(), exponents(w))
     assert np.array_equal(mat.transcode().cpu().numpy(), O.encode(w).pal_plane)
     wd = dev16(w)
     for m, kw in ((1, dict(kernel=uw.KERNEL_MMA, bn=4, split_k=1)), (256, dict(kernel=uw.KERNEL_TC, bn=256, split_k=1))):
@@ -226,6 +240,8 @@ def test_70b_k_outlier_and_sigma_sweep(uw, frac, sigma):
         yf = mat.matmul(xd, plan).cpu().numpy()
         yp = uw.matmul_bf16(xd, wd, plan).cpu().numpy()
         assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32))
+        ye = mat.matmul(xd, uw.make_plan(pipeline=uw.PIPE_DECODE_EXP_FUSED, **kw)).cpu().numpy()
+        assert np.array_equal(ye.view(np.uint32), yp.view(np.uint32))
         y_ref, a_ref = O.gemm(x, w)
         check_bound(yf, y_ref, a_ref)
     assert mat.device_status() == 0

@@ -2,7 +2,7 @@
 
 Each step of a stack must give exactly what uw_fused_matmul gives for the
 same matrix, input and plan, whichever stream the preprocessing ran on, and
-the fused results must lie within the oracle's bound.  Steps mix all three
+the fused results must lie within the oracle's bound.  Steps mix all four
 pipelines and both kernels, and more preprocessing steps than slots, so that
 slots are reused while earlier matmuls may still read them.
 """
@@ -36,7 +36,8 @@ def make_stack(uw, layers=3, m_list=(1, 64)):
             w = synth.weights_bf16(n, k, 0.02, 0.002, 1.0, seed=100 * layer + i)
             ws.append(w)
             mats.append(uw.Matrix(uw.encode(w)))
-    pipes = (uw.PIPE_DECODE_GEMM, uw.PIPE_TRANSCODE_FUSED, uw.PIPE_DIRECT_PALETTE, uw.PIPE_DECODE_GEMM)
+    pipes = (uw.PIPE_DECODE_GEMM, uw.PIPE_TRANSCODE_FUSED, uw.PIPE_DIRECT_PALETTE, uw.PIPE_DECODE_EXP_FUSED,
+             uw.PIPE_DECODE_GEMM)
     steps = []
     for j, m in enumerate(m_list):
         for i, mat in enumerate(mats):

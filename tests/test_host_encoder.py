@@ -209,6 +209,8 @@ def test_invalid_arguments(uw):
     dm = uw.DMat()
     assert lib.uw_decode_to_bf16(None, None, None) == 1
     assert lib.uw_decode_to_bf16(ctypes.byref(dm), None, None) == 1
+    assert lib.uw_decode_exponents(None, None, None) == 1
+    assert lib.uw_decode_exponents(ctypes.byref(dm), None, None) == 1
     p = uw.make_plan()
     assert lib.uw_fused_matmul(None, 1, ctypes.byref(dm), None, None, ctypes.byref(p), None, 0, None) == 1
     assert lib.uw_matmul_bf16(None, 1, None, 64, 64, None, ctypes.byref(p), None, 0, None, None) == 1
@@ -233,8 +235,13 @@ def test_plans_and_workspace(uw):
     assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_FMA, 1)) == 0
     assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_DECODE_GEMM, uw.KERNEL_FMA, 1)) == n * k * 2
     assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_TRANSCODE_FUSED, uw.KERNEL_FMA, 1)) == n * k // 2
+    # pipeline 2: exponent plane + all-raw bitmap + rank bases (one word per 32 groups each)
+    assert uw.workspace_size(1, n, k, uw.make_plan(uw.PIPE_DECODE_EXP_FUSED, uw.KERNEL_MMA, 4)) == \
+        n * k + 2 * (n * k // 64 // 32) * 4
+    assert uw.workspace_size(64, n, k, uw.make_plan(uw.PIPE_DECODE_EXP_FUSED, uw.KERNEL_TC, 64, 2)) == \
+        n * k + 2 * (n * k // 64 // 32) * 4 + 2 * 64 * n * 4
     assert uw.workspace_size(16, n, k, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 16, 4)) == 4 * 16 * n * 4
-    for bad in (uw.make_plan(kernel=9), uw.make_plan(bn=48), uw.make_plan(pipeline=2),
+    for bad in (uw.make_plan(kernel=9), uw.make_plan(bn=48), uw.make_plan(pipeline=0), uw.make_plan(pipeline=5),
                 uw.make_plan(kernel=uw.KERNEL_FMA, bn=1, split_k=2), uw.make_plan(split_k=0)):
         with pytest.raises(uw.UwError):
             uw.workspace_size(4, n, k, bad)
@@ -285,6 +292,14 @@ def test_stack_workspace_and_argument_checks(uw):
     bad = (uw.StackStep * 3)(*steps)
     bad[1].x_dev = None
     assert run(bad, 3, fake, size.value, None, None) == uw.ERR_INVALID_ARG
+    # a pipeline-2 step: its slot holds the exponent plane and two small index
+    # arrays (16 words each here, each padded to 256 bytes)
+    one = (uw.StackStep * 1)(uw.StackStep(ctypes.pointer(dm), fake, 4, fake,
+                                          uw.make_plan(uw.PIPE_DECODE_EXP_FUSED, uw.KERNEL_MMA, 2), None))
+    assert uw.lib().uw_stack_workspace_size(one, 1, ctypes.byref(size)) == 0
+    assert size.value == 2 * (n * k + 2 * 256)
+    one[0].y_dev = None
+    assert run(one, 1, fake, size.value, None, None) == uw.ERR_INVALID_ARG
     bad = (uw.StackStep * 3)(*steps)
     bad[2].plan.bn = 24                                   # not a tcgen05 token tile
     assert uw.lib().uw_stack_workspace_size(bad, 3, ctypes.byref(size)) == uw.ERR_INVALID_ARG
