@@ -265,21 +265,25 @@ def measured_traffic(group: str, alg_bytes_per_launch: float):
 
 
 def alg_bytes(mat, m, plan):
-    """Algorithmic HBM bytes of the kernels one matmul call launches."""
+    """Algorithmic HBM bytes of the kernels one matmul call launches: what
+    each kernel must read of the compressed forms and write."""
     info = mat.info
     n, k = mat.n, mat.k
-    common = info.section_bytes[0] + info.section_bytes[1] + (n * k // 64) // 8 * 2   # sm + raw + flags/base
+    nk = n * k
+    flags = nk // 64 // 8                                   # raw bitmap (rank bases: as many)
+    sm = info.section_bytes[0]                              # sign/mantissa plane
+    raw = info.section_bytes[1] + flags                     # raw plane + rank bases
+    stream = (info.stream_bits + 7) // 8 + (info.n_chunks + 1) * 4
     xy = m * k * 2 + m * n * 4
+    fused_in = sm + raw + flags + nk // 2                   # palette form
     if plan.pipeline == 4:
-        return {"fused": common + n * k // 2 + xy}
-    huff_in = common + (info.stream_bits + 7) // 8 + (info.n_chunks + 1) * 4
+        return {"fused": fused_in + xy}
     if plan.pipeline == 1:
-        return {"decode": huff_in + 2 * n * k, "plain": 2 * n * k + xy}
+        return {"decode": stream + flags + raw + sm + 2 * nk, "plain": 2 * nk + xy}
     if plan.pipeline == 2:
         # exponent plane + all-raw bitmap and rank words written, then read with the sm plane
-        idx = (n * k // 64) // 8 * 2
-        return {"exp_decode": huff_in + n * k + idx, "fused": 2 * n * k + idx + xy}
-    return {"transcode": huff_in + n * k // 2, "fused": common + n * k // 2 + xy}
+        return {"exp_decode": stream + flags + raw + nk + 2 * flags, "fused": sm + nk + 2 * flags + xy}
+    return {"transcode": stream + flags + nk // 2, "fused": fused_in + xy}
 
 
 def plans_from_json(text, n_mats, uw):

@@ -46,8 +46,16 @@ def main(argv=None):
     x = torch.from_numpy(synth.activations_bf16(a.m, a.k, a.seed).view(np.int16)).cuda()
     y = torch.empty(a.m, a.n, dtype=torch.float32, device="cuda")
     nk = a.n * a.k
-    common = info.section_bytes[uw.SEC_SM] + info.section_bytes[uw.SEC_RAWEXP] + nk // 64 // 4
-    huff_in = common + (info.stream_bits + 7) // 8 + (info.n_chunks + 1) * 4
+    # bytes each kernel reads of the compressed forms: the raw bitmap (nk/512)
+    # and its rank bases (nk/512); the Huffman stream and chunk offsets; the
+    # raw plane; the sign/mantissa plane (the transcode needs only the stream
+    # and the bitmap, the exponent decode no sign/mantissa bytes)
+    flags = nk // 64 // 8
+    stream = (info.stream_bits + 7) // 8 + (info.n_chunks + 1) * 4
+    raw = info.section_bytes[uw.SEC_RAWEXP] + flags
+    sm = info.section_bytes[uw.SEC_SM]
+    common = sm + raw + flags
+    huff_in = common + stream
     xy = a.m * a.k * 2 + a.m * a.n * 4
     flops = 2.0 * a.m * nk
     if a.kernel in ("fma", "plain_fma"):
@@ -67,11 +75,11 @@ def main(argv=None):
     elif a.kernel == "exp_decode":
         out = torch.empty(a.n, a.k, dtype=torch.uint8, device="cuda")
         run = lambda: mat.decode_exponents(out)
-        alg = huff_in + nk
+        alg = stream + flags + raw + nk
     elif a.kernel == "transcode":
         out = torch.empty(nk // 2, dtype=torch.uint8, device="cuda")
         run = lambda: mat.transcode(out)
-        alg = huff_in + nk // 2
+        alg = stream + flags + nk // 2
     elif a.kernel in ("fma", "tc", "mma"):
         run = lambda: mat.matmul(x, plan, y=y, ws=ws)
         alg = common + nk // 2 + xy

@@ -38,6 +38,28 @@ def test_source_digest_ignores_comments_only():
     assert bench.source_digest([src, ""]) != d                                  # file boundaries count
 
 
+def test_alg_bytes_per_pipeline():
+    """Each kernel is charged for what it must read and write: the decode
+    kernels never read the sign/mantissa plane unless they write BF16."""
+    from types import SimpleNamespace as NS
+    from decode_gemm_exponent_b200 import uw
+    n, k, m = 256, 1024, 4
+    nk = n * k
+    sec = [nk, 4096, 0, 0, 0, 0, 0, nk // 2]            # sm, raw plane, ...
+    mat = NS(n=n, k=k, info=NS(section_bytes=sec, stream_bits=8 * 70000, n_chunks=nk // 256))
+    stream = 70000 + (nk // 256 + 1) * 4
+    flags = nk // 512
+    xy = m * k * 2 + m * n * 4
+    plan = lambda p: uw.make_plan(p, uw.KERNEL_MMA, 4)
+    assert bench.alg_bytes(mat, m, plan(4)) == {"fused": nk + 4096 + 2 * flags + nk // 2 + xy}
+    assert bench.alg_bytes(mat, m, plan(1)) == {"decode": stream + nk + 4096 + 2 * flags + 2 * nk,
+                                                 "plain": 2 * nk + xy}
+    assert bench.alg_bytes(mat, m, plan(2)) == {"exp_decode": stream + 4096 + 4 * flags + nk,
+                                                 "fused": 2 * nk + 2 * flags + xy}
+    assert bench.alg_bytes(mat, m, plan(3)) == {"transcode": stream + flags + nk // 2,
+                                                 "fused": nk + 4096 + 2 * flags + nk // 2 + xy}
+
+
 def test_plans_from_json_round_trip():
     from decode_gemm_exponent_b200 import uw
     doc = {"plans": []}
