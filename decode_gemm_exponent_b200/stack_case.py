@@ -14,8 +14,11 @@ with 0.05% N(0, 1) outliers, seed 3*layer + projection + 1.  Activations per
     describes (a Huffman layer decoded while a palette layer computes); the
     kernel choice (FMA or tcgen05, token tile, split) is the autotuned one.
 Each line reports the stack's time with and without the side stream and the
-effective weight bandwidth (uncompressed BF16 bytes / time).  The host
-encode runs in a spawn process pool before any CUDA call.
+effective weight bandwidth (uncompressed BF16 bytes / time), and the
+decode/compute SM split chosen by uw_stack_tune_split among --splits
+(preprocessing SMs in a green-context partition of their own; 0 = the side
+stream shares all SMs) with each candidate's time.  The host encode runs in a
+spawn process pool before any CUDA call.
 """
 from __future__ import annotations
 
@@ -44,6 +47,8 @@ def main(argv=None):
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--workers", type=int, default=min(16, os.cpu_count() or 1))
+    ap.add_argument("--splits", type=int, nargs="+", default=[0, 16, 32, 48],
+                    help="preprocessing SM counts tried by the split tuner (0 = no split)")
     a = ap.parse_args(argv)
 
     jobs = [(layer, i, n, k) for layer in range(a.layers) for i, (_, n, k) in enumerate(SHAPES)]
@@ -91,6 +96,10 @@ def main(argv=None):
             for mat in mats[:3]:
                 if mat.device_status() != 0:
                     raise RuntimeError("kernel status during the stack run")
+            best_split, split_us = stack.tune_split(a.splits, reps=a.reps)
+            for mat in mats[:3]:
+                if mat.device_status() != 0:
+                    raise RuntimeError("kernel status during the split tuning")
             n_prep = sum(1 for s in steps if s[3].pipeline != uw.PIPE_DIRECT_PALETTE)
             print(json.dumps({
                 "workload": "llama-3.1-8b MLP stack", "layers": a.layers, "m": m, "plans": kind,
@@ -99,6 +108,8 @@ def main(argv=None):
                 "speedup": round(us_serial / us_overlap, 4),
                 "weight_gbs_overlap": round(weight_bytes / us_overlap / 1e3, 1),
                 "weight_gbs_one_stream": round(weight_bytes / us_serial / 1e3, 1),
+                "split_best_prep_sms": best_split,
+                "split_us": {str(c): round(u, 1) for c, u in zip(a.splits, split_us)},
                 "plan_per_projection": [str(plans[p][j].as_dict()) for p in range(3)],
             }), flush=True)
         del stack, steps

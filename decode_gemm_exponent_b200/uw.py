@@ -38,7 +38,8 @@ EXPORTS = ("uw_status_str", "uw_version", "uw_encode", "uw_blob_data", "uw_blob_
            "uw_blob_info_get", "uw_matrix_bind", "uw_device_status", "uw_decode_to_bf16",
            "uw_decode_exponents", "uw_transcode_palette", "uw_plan_default", "uw_workspace_size", "uw_fused_matmul",
            "uw_matmul_bf16", "uw_autotune_workspace_size", "uw_plan_autotune",
-           "uw_fused_matmul_noalloc", "uw_stack_workspace_size", "uw_stack_run")
+           "uw_fused_matmul_noalloc", "uw_stack_workspace_size", "uw_stack_run",
+           "uw_sm_split_create", "uw_sm_split_get", "uw_sm_split_destroy", "uw_stack_tune_split")
 
 
 class UwError(RuntimeError):
@@ -126,6 +127,13 @@ def lib() -> ctypes.CDLL:
         "uw_fused_matmul_noalloc": (ctypes.c_int, [P, I64, ctypes.POINTER(DMat), P, ctypes.POINTER(Plan), P]),
         "uw_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, ctypes.POINTER(SZ)]),
         "uw_stack_run": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, P, SZ, P, P]),
+        "uw_sm_split_create": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.POINTER(P)]),
+        "uw_sm_split_get": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(ctypes.c_int),
+                                           ctypes.POINTER(ctypes.c_int)]),
+        "uw_sm_split_destroy": (None, [P]),
+        "uw_stack_tune_split": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, P, SZ, ctypes.c_int,
+                                               ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int,
+                                               ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), P]),
         "uw_autotune_workspace_size": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(DMat)), ctypes.c_int,
                                                       ctypes.POINTER(I64), ctypes.c_int,
                                                       ctypes.POINTER(SZ)]),
@@ -306,6 +314,53 @@ class Stack:
         side = ctypes.c_void_p(side_stream.cuda_stream) if side_stream is not None else ctypes.c_void_p(0)
         check(lib().uw_stack_run(self.steps, len(self.steps), _ptr(self.ws), self.ws.numel(),
                                  _stream_handle(stream), side), "uw_stack_run")
+
+    def tune_split(self, candidates, reps: int = 5, stream=None):
+        """uw_stack_tune_split: the fastest preprocessing SM count among
+        `candidates` (0 = no split) and each candidate's microseconds per run."""
+        import torch
+        cand = (ctypes.c_int * len(candidates))(*candidates)
+        us = (ctypes.c_float * len(candidates))()
+        best = ctypes.c_int()
+        dev = self.ws.device.index if self.ws.device.index is not None else torch.cuda.current_device()
+        check(lib().uw_stack_tune_split(self.steps, len(self.steps), _ptr(self.ws), self.ws.numel(), dev, cand,
+                                        len(candidates), reps, ctypes.byref(best), us, _stream_handle(stream)),
+              "uw_stack_tune_split")
+        return best.value, [float(u) for u in us]
+
+
+class SmSplit:
+    """uw_sm_split: the device's SMs split into a preprocessing and a compute
+    partition (green contexts), each with a stream, wrapped as torch external
+    streams (`prep_stream`, `compute_stream`) for Stack.run and the matmuls.
+    Call close() (or leave a `with` block) once their work has completed."""
+
+    def __init__(self, prep_sms: int, device=None):
+        import torch
+        dev = torch.cuda.current_device() if device is None else int(device)
+        h = ctypes.c_void_p()
+        check(lib().uw_sm_split_create(dev, prep_sms, ctypes.byref(h)), "uw_sm_split_create")
+        self.handle = h
+        ps, cs = ctypes.c_void_p(), ctypes.c_void_p()
+        pn, cn = ctypes.c_int(), ctypes.c_int()
+        check(lib().uw_sm_split_get(h, ctypes.byref(ps), ctypes.byref(cs), ctypes.byref(pn), ctypes.byref(cn)),
+              "uw_sm_split_get")
+        self.prep_sms, self.compute_sms = pn.value, cn.value
+        self.prep_stream = torch.cuda.ExternalStream(ps.value, device=dev)
+        self.compute_stream = torch.cuda.ExternalStream(cs.value, device=dev)
+
+    def close(self):
+        if self.handle:
+            self.prep_stream.synchronize()
+            self.compute_stream.synchronize()
+            lib().uw_sm_split_destroy(self.handle)
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
 
 
 def workspace_size(m: int, n: int, k: int, plan: Plan) -> int:

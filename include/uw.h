@@ -332,6 +332,48 @@ uw_status uw_stack_workspace_size(const uw_stack_step *steps, int n_steps, size_
 uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void *ws, size_t ws_bytes,
                        void *stream, void *side_stream);
 
+/* ------------------------------------------------------------------------ */
+/* Decode/compute SM split (Unweight page §九: the autotuner also measures how */
+/* the SMs are divided between decoding and compute).                         */
+
+/* A split of one device's SMs into two green contexts with one stream each:
+ * a preprocessing partition and a compute partition.  Work on a partition's
+ * stream runs only on its SMs.  Both streams belong to the device's primary
+ * context, so every entry point of this library (and the caller's device
+ * memory and events) works on them.                                          */
+typedef struct uw_sm_split uw_sm_split;
+
+/* Split device `device`: at least prep_sms SMs (rounded up by the driver to
+ * whole granules, 8 SMs on this GPU) for preprocessing, the rest for compute.
+ * prep_sms <= 0, or a split that leaves the compute partition empty, gives
+ * UW_ERR_INVALID_ARG; a driver without green contexts (or no driver) gives
+ * UW_ERR_CUDA.  Typical use: uw_stack_run(..., compute_stream, prep_stream). */
+uw_status uw_sm_split_create(int device, int prep_sms, uw_sm_split **out);
+
+/* The split's streams (cudaStream_t as void*) and actual SM counts; any
+ * output pointer may be NULL.                                                */
+uw_status uw_sm_split_get(const uw_sm_split *s, void **prep_stream, void **compute_stream,
+                          int *prep_sms, int *compute_sms);
+
+/* Destroy the streams and green contexts.  All work queued on the split's
+ * streams must have completed.  NULL is ignored.                             */
+void uw_sm_split_destroy(uw_sm_split *s);
+
+/* Choose the split for a stack: for every candidate cand[c] (preprocessing
+ * SMs; 0 = no split, the two streams share all SMs) run the stack once to
+ * warm up and then `reps` times (0 = 5) with the matmuls on the compute
+ * stream and the preprocessing on the other, timed with CUDA events, and
+ * return the fastest candidate in *best and every candidate's microseconds
+ * per run in us_out[c] (may be NULL).  The caller's `stream` is synchronized
+ * first (the steps' inputs may be produced there); all candidates run on
+ * streams created and destroyed here, and no work is left in flight on
+ * return.  The stack's weights are re-read every run: a stack larger than
+ * the 126 MB L2 times as in a model's layer sequence.  ws as in uw_stack_run.
+ * Errors as in uw_stack_run and uw_sm_split_create.                          */
+uw_status uw_stack_tune_split(const uw_stack_step *steps, int n_steps, void *ws, size_t ws_bytes,
+                              int device, const int *cand, int n_cand, int reps, int *best,
+                              float *us_out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -103,3 +103,50 @@ def test_stack_slot_reuse_on_one_matrix(uw):
     for x, y in zip(xs, ys):
         assert np.array_equal(y.cpu().numpy(), mat.matmul(x, plan).cpu().numpy())
     assert mat.device_status() == 0
+
+
+# ---------------------------------------------------------------- decode/compute SM split
+
+def test_sm_split_partitions(uw):
+    total = torch.cuda.get_device_properties(0).multi_processor_count
+    with uw.SmSplit(20) as sp:
+        assert sp.prep_sms >= 20 and sp.prep_sms % 8 == 0       # whole 8-SM granules
+        assert 0 < sp.compute_sms and sp.prep_sms + sp.compute_sms <= total
+    for bad in (0, total):
+        with pytest.raises(uw.UwError):
+            uw.SmSplit(bad)
+
+
+def test_stack_on_split_streams_matches_single_calls(uw):
+    """The matmuls on the compute partition's stream, the decodes and
+    transcodes on the preprocessing partition's: every step bit-identical to
+    the single call."""
+    mats, ws, steps = make_stack(uw)
+    want = reference_outputs(uw, steps)
+    stack = uw.Stack(steps)
+    with uw.SmSplit(24) as sp:
+        for rep in range(2):
+            for _, _, y, _ in steps:
+                y.fill_(float("nan"))
+            torch.cuda.synchronize()
+            stack.run(stream=sp.compute_stream, side_stream=sp.prep_stream)
+            sp.compute_stream.synchronize()
+            for s, (st, w_ref) in enumerate(zip(steps, want)):
+                got = st[2].cpu().numpy()
+                assert np.array_equal(got.view(np.uint32), w_ref.view(np.uint32)), "step %d rep %d" % (s, rep)
+    for mat in mats:
+        assert mat.device_status() == 0
+
+
+def test_tune_split_picks_a_candidate(uw):
+    mats, ws, steps = make_stack(uw, layers=2, m_list=(1,))
+    want = reference_outputs(uw, steps)
+    stack = uw.Stack(steps)
+    cands = [0, 16, 32]
+    best, us = stack.tune_split(cands, reps=2)
+    assert best in cands and len(us) == 3 and all(u > 0 for u in us)
+    assert us[cands.index(best)] == min(us)
+    for (_, _, y, _), w_ref in zip(steps, want):          # the last timed run's outputs
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), w_ref.view(np.uint32))
+    for mat in mats:
+        assert mat.device_status() == 0

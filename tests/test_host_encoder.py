@@ -303,3 +303,41 @@ def test_stack_workspace_and_argument_checks(uw):
     bad = (uw.StackStep * 3)(*steps)
     bad[2].plan.bn = 24                                   # not a tcgen05 token tile
     assert uw.lib().uw_stack_workspace_size(bad, 3, ctypes.byref(size)) == uw.ERR_INVALID_ARG
+
+
+def test_sm_split_argument_checks(uw):
+    """uw_sm_split_* and uw_stack_tune_split reject bad arguments before any
+    CUDA call; with no driver (this host) a valid split request fails with
+    UW_ERR_CUDA instead of crashing."""
+    lib = uw.lib()
+    h = ctypes.c_void_p()
+    assert lib.uw_sm_split_create(0, 0, ctypes.byref(h)) == uw.ERR_INVALID_ARG
+    assert lib.uw_sm_split_create(-1, 16, ctypes.byref(h)) == uw.ERR_INVALID_ARG
+    assert lib.uw_sm_split_create(0, 16, None) == uw.ERR_INVALID_ARG
+    st = lib.uw_sm_split_create(0, 16, ctypes.byref(h))
+    assert st in (uw.UW_OK, uw.ERR_CUDA)
+    if st == uw.UW_OK:                     # a machine with a GPU
+        lib.uw_sm_split_destroy(h)
+    assert lib.uw_sm_split_get(None, None, None, None, None) == uw.ERR_INVALID_ARG
+    lib.uw_sm_split_destroy(None)
+    # the tuner: argument and workspace checks on a bound-but-never-read matrix
+    w = synth.weights_bf16(128, 256, 0.02, 0.002, 1.0, seed=3)
+    host = np.frombuffer(uw.encode(w), np.uint8)
+    fake = 1 << 40
+    dm = uw.DMat()
+    uw.check(lib.uw_matrix_bind(host.ctypes.data, host.size, fake, fake, 0, ctypes.byref(dm)), "uw_matrix_bind")
+    steps = (uw.StackStep * 1)(uw.StackStep(ctypes.pointer(dm), fake, 4, fake,
+                                            uw.make_plan(uw.PIPE_DECODE_GEMM, uw.KERNEL_MMA, 2), None))
+    size = ctypes.c_size_t()
+    assert lib.uw_stack_workspace_size(steps, 1, ctypes.byref(size)) == 0
+    cand = (ctypes.c_int * 2)(0, 16)
+    best = ctypes.c_int()
+    tune = lib.uw_stack_tune_split
+    assert tune(None, 1, fake, size.value, 0, cand, 2, 1, ctypes.byref(best), None, None) == uw.ERR_INVALID_ARG
+    assert tune(steps, 1, fake, size.value, 0, cand, 0, 1, ctypes.byref(best), None, None) == uw.ERR_INVALID_ARG
+    assert tune(steps, 1, fake, size.value, 0, cand, 2, 1, None, None, None) == uw.ERR_INVALID_ARG
+    assert tune(steps, 1, fake, size.value, -1, cand, 2, 1, ctypes.byref(best), None, None) == uw.ERR_INVALID_ARG
+    neg = (ctypes.c_int * 2)(0, -8)
+    assert tune(steps, 1, fake, size.value, 0, neg, 2, 1, ctypes.byref(best), None, None) == uw.ERR_INVALID_ARG
+    assert tune(steps, 1, fake, size.value - 1, 0, cand, 2, 1, ctypes.byref(best), None, None) == uw.ERR_WORKSPACE
+    assert tune(steps, 1, fake + 16, size.value, 0, cand, 2, 1, ctypes.byref(best), None, None) == uw.ERR_WORKSPACE
