@@ -3,6 +3,7 @@
 // pipelines of the Unweight page (§六).
 #include <algorithm>
 #include <cstring>
+#include <vector>
 
 #include "kernels.h"
 #include "uw_format.h"
@@ -252,6 +253,28 @@ extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_
         if (!pal || !aligned(pal, 16)) return UW_ERR_INVALID_ARG;
     }
     return run_kernel(x_dev, m, nullptr, w, pal, w->n, w->k, y_dev, plan, partial, w->dev_status, s);
+}
+
+extern "C" uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const uw_plan *plan,
+                                             void *stream) {
+    if (!items || n_items <= 0 || !plan) return UW_ERR_INVALID_ARG;
+    if (plan->pipeline != UW_PIPE_DIRECT_PALETTE || plan->kernel != UW_KERNEL_MMA) return UW_ERR_INVALID_ARG;
+    std::vector<MmaItem> v(static_cast<size_t>(n_items));
+    for (int i = 0; i < n_items; i++) {
+        const uw_batch_item &it = items[i];
+        uw_status st = check_dmat(it.w);
+        if (st != UW_OK) return st;
+        if (it.m < 0 || it.m > 16) return UW_ERR_INVALID_ARG;
+        st = check_plan(plan, it.m > 0 ? it.m : 1, it.w->k);
+        if (st != UW_OK) return st;
+        if (it.m > 0) {
+            if (!it.x_dev || !it.y_dev || !aligned(it.x_dev, 16) || !aligned(it.y_dev, 16)) return UW_ERR_INVALID_ARG;
+            if (!it.w->pal || !aligned(it.w->pal, 16)) return UW_ERR_INVALID_ARG;
+        }
+        v[size_t(i)] = MmaItem{it.x_dev, int(it.m), it.w, it.y_dev};
+    }
+    return cuda_status(launch_gemv_mma_batched(v.data(), n_items, plan->bn, plan->stages,
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 extern "C" uw_status uw_matmul_bf16(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev,

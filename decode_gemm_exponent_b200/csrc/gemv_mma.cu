@@ -160,8 +160,9 @@ __device__ __forceinline__ void rebuild(const Half<Q> &h, bool raw, const Palett
     }
 }
 
+// One CTA's work: the 16-row tile `tile` of the matmul `a`.
 template <bool PAL, int NT, int Q>   // NT: 8-token tiles (1: m <= 8, 2: m <= 16); Q: 16*Q weights per lane and row
-__global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
+__device__ __forceinline__ void gemv_mma_tile(const MmaArgs &a, int64_t tile) {
     constexpr int kCh = kChunk * Q;               // weights per chunk along K
     constexpr int kWl = 16 * Q;                   // weights per lane and row in a chunk
     constexpr int kStages = Q == 1 ? 3 : 2;       // chunks of loads in flight per warp
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slices = blockDim.x >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int64_t row0 = int64_t(blockIdx.x) * kTileRows;
+    const int64_t row0 = tile * kTileRows;
     const int64_t ra = row0 + g, rb = ra + 8;       // this lane's two rows
     const int64_t gpr = a.k / kChunk;               // groups per row
     const int64_t cpr = a.k / kCh;                  // chunks per row
@@ -316,6 +317,31 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
     }
 }
 
+template <bool PAL, int NT, int Q>
+__global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma(const MmaArgs a) {
+    gemv_mma_tile<PAL, NT, Q>(a, blockIdx.x);
+}
+
+// Many fused matmuls in one launch (the experts of a mixture-of-experts
+// layer): CTA b runs tile b - tile_end[i-1] of item i, where item i is the
+// first with b < tile_end[i].  Items share the kernel's template arguments
+// (token tiles, step width) and the CTA size; each item's tiles compute
+// exactly what a launch of k_gemv_mma for that item alone computes.
+constexpr int kBatchMax = 32;
+struct MmaBatch {
+    MmaArgs item[kBatchMax];
+    int tile_end[kBatchMax];   // inclusive prefix sums of the items' tile counts
+    int n_items;
+};
+
+template <int NT, int Q>
+__global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma_batched(const __grid_constant__ MmaBatch b) {
+    const int t = int(blockIdx.x);
+    int i = 0;
+    while (i + 1 < b.n_items && t >= b.tile_end[i]) i++;
+    gemv_mma_tile<true, NT, Q>(b.item[i], t - (i ? b.tile_end[i - 1] : 0));
+}
+
 }  // namespace
 
 cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
@@ -358,6 +384,60 @@ cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, co
     }
 #undef UW_MMA_LAUNCH
     return cudaGetLastError();
+}
+
+cudaError_t launch_gemv_mma_batched(const MmaItem *items, int n_items, int slices, int width,
+                                    cudaStream_t stream) {
+    if (n_items < 0 || slices < 1 || slices > kMaxSlices) return cudaErrorInvalidValue;
+    // one step width for all items: 32 weights per lane only if every K allows it
+    bool all128 = true;
+    for (int i = 0; i < n_items; i++) all128 = all128 && items[i].w->k % (2 * kChunk) == 0;
+    if (width == 2 && !all128) return cudaErrorInvalidValue;
+    const int q = width == 1 ? 1 : (all128 ? 2 : 1);
+    int i = 0;
+    while (i < n_items) {
+        MmaBatch b{};
+        int tiles = 0, max_m = 0, max_fw = 0;
+        for (; i < n_items && b.n_items < kBatchMax; i++) {
+            const MmaItem &it = items[i];
+            const uw_dmat &w = *it.w;
+            if (it.m == 0) continue;   // an expert without tokens
+            if (it.m < 0 || it.m > 16 || w.n % kTileRows || w.k % (q * kChunk) || !w.pal) return cudaErrorInvalidValue;
+            MmaArgs &a = b.item[b.n_items];
+            a.x = it.x;
+            a.m = it.m;
+            a.y = it.y;
+            a.n = w.n;
+            a.k = w.k;
+            a.flag_words = int(((kTileRows * (w.k / kChunk)) >> 5) + 2);
+            a.sm = w.sm;
+            a.pal = reinterpret_cast<const uint32_t *>(w.pal);
+            a.flagbits = w.flagbits;
+            a.rawbase = w.rawbase;
+            a.rawexp = w.rawexp;
+            a.palette = make_palette16(w.palette);
+            tiles += int(w.n / kTileRows);
+            b.tile_end[b.n_items] = tiles;
+            max_m = it.m > max_m ? it.m : max_m;
+            max_fw = a.flag_words > max_fw ? a.flag_words : max_fw;
+            b.n_items++;
+        }
+        if (b.n_items == 0) continue;
+        const int nt = max_m > 8 ? 2 : 1;
+        const size_t smem = size_t(2 * max_fw) * 4 + (slices > 1 ? size_t(slices) * 32 * 4 * nt * 4 : 0);
+        if (smem > size_t(kMaxSmem)) return cudaErrorInvalidValue;
+        const unsigned grid = unsigned(tiles), block = unsigned(slices * 32);
+        if (q == 2) {
+            if (nt == 2) k_gemv_mma_batched<2, 2><<<grid, block, smem, stream>>>(b);
+            else k_gemv_mma_batched<1, 2><<<grid, block, smem, stream>>>(b);
+        } else {
+            if (nt == 2) k_gemv_mma_batched<2, 1><<<grid, block, smem, stream>>>(b);
+            else k_gemv_mma_batched<1, 1><<<grid, block, smem, stream>>>(b);
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace uw

@@ -81,6 +81,20 @@ cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, co
                             const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices, int width,
                             cudaStream_t stream);
 
+// The warp-MMA fused kernel over many matrices in as few launches as
+// possible (32 matrices per launch; items with m == 0 are skipped): item i
+// computes y[m, n] = x[m, k] * W^T on its palette-form matrix, bit-identical
+// to launch_gemv_mma for that item alone with the same slices and step
+// width.  width 0 picks 32 weights per lane only if every item's k allows it.
+struct MmaItem {
+    const uint16_t *x;
+    int m;
+    const uw_dmat *w;
+    float *y;
+};
+cudaError_t launch_gemv_mma_batched(const MmaItem *items, int n_items, int slices, int width,
+                                    cudaStream_t stream);
+
 // tcgen05 GEMM (Unweight page §七, reconstructive matmul), token tile `bn`.
 struct TcLaunch {
     const uint16_t *x;         // [m, k] BF16

@@ -39,7 +39,8 @@ EXPORTS = ("uw_status_str", "uw_version", "uw_encode", "uw_blob_data", "uw_blob_
            "uw_decode_exponents", "uw_transcode_palette", "uw_plan_default", "uw_workspace_size", "uw_fused_matmul",
            "uw_matmul_bf16", "uw_autotune_workspace_size", "uw_plan_autotune",
            "uw_fused_matmul_noalloc", "uw_stack_workspace_size", "uw_stack_run",
-           "uw_sm_split_create", "uw_sm_split_get", "uw_sm_split_destroy", "uw_stack_tune_split")
+           "uw_sm_split_create", "uw_sm_split_get", "uw_sm_split_destroy", "uw_stack_tune_split",
+           "uw_fused_matmul_batched")
 
 
 class UwError(RuntimeError):
@@ -89,6 +90,11 @@ class StackStep(ctypes.Structure):
                 ("y_dev", ctypes.c_void_p), ("plan", Plan), ("pal_dev", ctypes.c_void_p)]
 
 
+class BatchItem(ctypes.Structure):
+    _fields_ = [("w", ctypes.POINTER(DMat)), ("x_dev", ctypes.c_void_p), ("m", ctypes.c_int64),
+                ("y_dev", ctypes.c_void_p)]
+
+
 def make_plan(pipeline=PIPE_DIRECT_PALETTE, kernel=KERNEL_TC, bn=16, split_k=1, stages=0,
               debug_flags=0, timeout_ns=0) -> Plan:
     return Plan(pipeline, kernel, bn, split_k, stages, debug_flags, timeout_ns)
@@ -125,6 +131,7 @@ def lib() -> ctypes.CDLL:
                                            P, SZ, P]),
         "uw_matmul_bf16": (ctypes.c_int, [P, I64, P, I64, I64, P, ctypes.POINTER(Plan), P, SZ, P, P]),
         "uw_fused_matmul_noalloc": (ctypes.c_int, [P, I64, ctypes.POINTER(DMat), P, ctypes.POINTER(Plan), P]),
+        "uw_fused_matmul_batched": (ctypes.c_int, [ctypes.POINTER(BatchItem), ctypes.c_int, ctypes.POINTER(Plan), P]),
         "uw_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, ctypes.POINTER(SZ)]),
         "uw_stack_run": (ctypes.c_int, [ctypes.POINTER(StackStep), ctypes.c_int, P, SZ, P, P]),
         "uw_sm_split_create": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.POINTER(P)]),
@@ -280,6 +287,20 @@ def fused_matmul_noalloc(mat: "Matrix", x, plan: Plan, y=None, stream=None):
     check(lib().uw_fused_matmul_noalloc(_ptr(x), m, ctypes.byref(mat.dmat), _ptr(y), ctypes.byref(plan),
                                         _stream_handle(stream)), "uw_fused_matmul_noalloc")
     return y
+
+
+def fused_matmul_batched(items, plan: Plan, stream=None):
+    """uw_fused_matmul_batched: items are (Matrix, x [m, k], y [m, n]) with
+    0 <= m <= 16 (m = 0: skipped); all run with the warp-MMA plan `plan` in
+    as few launches as possible (32 matrices each)."""
+    arr = (BatchItem * len(items))()
+    for i, (mat, x, y) in enumerate(items):
+        m = int(x.shape[0])
+        if x.shape[1] != mat.k or tuple(y.shape) != (m, mat.n):
+            raise ValueError("item %d: shapes do not match the matrix" % i)
+        arr[i] = BatchItem(ctypes.pointer(mat.dmat), x.data_ptr() if m else None, m, y.data_ptr() if m else None)
+    check(lib().uw_fused_matmul_batched(arr, len(items), ctypes.byref(plan), _stream_handle(stream)),
+          "uw_fused_matmul_batched")
 
 
 class Stack:

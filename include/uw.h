@@ -253,6 +253,29 @@ uw_status uw_matmul_bf16(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev
                          void *ws, size_t ws_bytes, uint32_t *dev_status, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Many small matmuls in one launch (the experts of a mixture-of-experts      */
+/* layer, which the Unweight page §十一 names as the next target).            */
+
+/* One matmul of a batch: y_dev[m, w->n] = x_dev[m, w->k] * W^T. */
+typedef struct uw_batch_item {
+    const uw_dmat *w;        /* palette form (UW_EMIT_PALETTE) */
+    const uint16_t *x_dev;   /* [m, k] BF16, 16-byte aligned */
+    int64_t m;               /* 0..16 tokens; 0 = nothing to do (an expert nobody routed to) */
+    float *y_dev;            /* [m, n] float32, 16-byte aligned */
+} uw_batch_item;
+
+/* Run every item with the warp-MMA fused kernel, up to 32 items per launch
+ * instead of one launch per item.  plan: UW_PIPE_DIRECT_PALETTE and
+ * UW_KERNEL_MMA (bn warps per tile, as for uw_fused_matmul); stages 0 takes 32
+ * weights per lane and step only if every item's k is a multiple of 128.
+ * Each item's y is bit-identical to uw_fused_matmul on that item with the
+ * same plan (and stages resolved the same way).  Items may differ in n, k, m
+ * and palette; no workspace.  All arguments are checked before anything is
+ * launched; errors as in uw_fused_matmul.                                    */
+uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const uw_plan *plan,
+                                  void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Matmul without a caller workspace (no counterpart on the Unweight page).   */
 
 /* Bytes of the library-owned scratch array used by uw_fused_matmul_noalloc. */

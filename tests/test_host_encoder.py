@@ -341,3 +341,39 @@ def test_sm_split_argument_checks(uw):
     assert tune(steps, 1, fake, size.value, 0, neg, 2, 1, ctypes.byref(best), None, None) == uw.ERR_INVALID_ARG
     assert tune(steps, 1, fake, size.value - 1, 0, cand, 2, 1, ctypes.byref(best), None, None) == uw.ERR_WORKSPACE
     assert tune(steps, 1, fake + 16, size.value, 0, cand, 2, 1, ctypes.byref(best), None, None) == uw.ERR_WORKSPACE
+
+
+def test_batched_matmul_argument_checks(uw):
+    """uw_fused_matmul_batched checks every item before launching anything
+    (the matrices are bound to device addresses that are never read)."""
+    lib = uw.lib()
+    fake = 1 << 40
+    dms = []
+    for n, k in ((128, 256), (64, 192)):
+        w = synth.weights_bf16(n, k, 0.02, 0.002, 1.0, seed=n + k)
+        host = np.frombuffer(uw.encode(w, uw.EMIT_HUFFMAN | uw.EMIT_PALETTE), np.uint8)
+        dm = uw.DMat()
+        uw.check(lib.uw_matrix_bind(host.ctypes.data, host.size, fake, fake, 0, ctypes.byref(dm)), "uw_matrix_bind")
+        dms.append(dm)
+
+    def items(*spec):
+        arr = (uw.BatchItem * len(spec))()
+        for i, (j, m, x, y) in enumerate(spec):
+            arr[i] = uw.BatchItem(ctypes.pointer(dms[j]), x, m, y)
+        return arr
+
+    ok = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, 2, 1, 0)
+    run = lambda arr, plan: lib.uw_fused_matmul_batched(arr, len(arr), ctypes.byref(plan), None)
+    good = items((0, 4, fake, fake), (1, 1, fake, fake))
+    assert lib.uw_fused_matmul_batched(good, 0, ctypes.byref(ok), None) == uw.ERR_INVALID_ARG
+    assert lib.uw_fused_matmul_batched(None, 2, ctypes.byref(ok), None) == uw.ERR_INVALID_ARG
+    assert run(good, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 16, 1)) == uw.ERR_INVALID_ARG
+    assert run(good, uw.make_plan(uw.PIPE_DECODE_GEMM, uw.KERNEL_MMA, 2, 1)) == uw.ERR_INVALID_ARG
+    assert run(good, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, 9, 1)) == uw.ERR_INVALID_ARG
+    # 32 weights per lane need every k to be a multiple of 128 (k = 192 is not)
+    assert run(good, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA, 2, 1, 2)) == uw.ERR_INVALID_ARG
+    assert run(items((0, 17, fake, fake)), ok) == uw.ERR_INVALID_ARG
+    assert run(items((0, -1, fake, fake)), ok) == uw.ERR_INVALID_ARG
+    assert run(items((0, 4, fake + 8, fake)), ok) == uw.ERR_INVALID_ARG      # misaligned x
+    assert run(items((0, 4, fake, None)), ok) == uw.ERR_INVALID_ARG          # no y
+    assert run(items((0, 4, fake, fake), (1, 2, None, fake)), ok) == uw.ERR_INVALID_ARG
