@@ -32,6 +32,9 @@
 // chains), added at the end, and the S slice results are summed in ascending
 // slice order through shared memory.  The fused and plain variants share all
 // of this but the loader, so their outputs are bit-identical.
+// The batched kernel runs the same tile body for many matrices in one launch
+// (the routed experts of a mixture-of-experts layer, Unweight page §十一),
+// so each matrix's output is the single kernel's, bit for bit.
 #include <algorithm>
 
 #include "device_common.cuh"
