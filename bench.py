@@ -264,6 +264,22 @@ def measured_traffic(group: str, alg_bytes_per_launch: float):
     return rec["bytes"] * alg_bytes_per_launch / rec["alg_bytes"]
 
 
+def compression_stats(infos):
+    """Size and exponent statistics of the layer's matrices (weighted by
+    their weight counts): compressed size of each form as a fraction of BF16,
+    Shannon entropy of the exponent byte, top-16 palette coverage and the
+    fraction of 64-weight groups stored raw."""
+    w = [i.n * i.k for i in infos]
+    tot = sum(w)
+    return {
+        "compressed_fraction_huffman": round(sum(i.huffman_bytes for i in infos) / (2 * tot), 4),
+        "compressed_fraction_palette": round(sum(i.palette_bytes for i in infos) / (2 * tot), 4),
+        "exponent_entropy_bits": round(sum(i.entropy_bits * x for i, x in zip(infos, w)) / tot, 4),
+        "top16_coverage": round(sum(i.top16_coverage * x for i, x in zip(infos, w)) / tot, 6),
+        "raw_group_fraction": round(sum(i.n_raw for i in infos) / sum(i.n_groups for i in infos), 5),
+    }
+
+
 def alg_bytes(mat, m, plan):
     """Algorithmic HBM bytes of the kernels one matmul call launches: what
     each kernel must read of the compressed forms and write."""
@@ -467,10 +483,7 @@ def run_gpu(args, rank, world):
         "config": {
             "workload": WORKLOAD,
             "l2": "no flush: each matrix is re-read after >= 160 MB of other matrices (inputs larger than L2)",
-            "compressed_fraction_huffman": round(sum(i.huffman_bytes for i in infos) /
-                                                 sum(2 * i.n * i.k for i in infos), 4),
-            "compressed_fraction_palette": round(sum(i.palette_bytes for i in infos) /
-                                                 sum(2 * i.n * i.k for i in infos), 4),
+            **compression_stats(infos),
             "plans": {"%s@M=%d" % (c["name"], c["m"]): kernel_group(c["plan"]) +
                       ("/split%d" % c["plan"].split_k if c["plan"].kernel == 2 else "") for c in calls},
             "per_call_us": {"%s@M=%d" % (c["name"], c["m"]): round(1e3 * t, 2) for c, t in zip(calls, per_call)},

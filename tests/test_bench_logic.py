@@ -60,6 +60,34 @@ def test_alg_bytes_per_pipeline():
                                                  "fused": nk + 4096 + 2 * flags + nk // 2 + xy}
 
 
+def test_compression_stats_on_real_blobs():
+    """The bench line's size and exponent statistics come from the blob
+    headers; checked against the oracle's own histogram on two small
+    matrices of different sizes (weights-weighted means)."""
+    import numpy as np
+    from decode_gemm_exponent_b200 import synth, uw
+    from oracle import oracle as O
+    ws = [synth.weights_bf16(128, 512, 0.02, 0.001, 1.0, seed=1), synth.weights_bf16(64, 256, 0.05, 0.01, 1.0, seed=2)]
+    infos = [uw.blob_info(uw.encode(w)) for w in ws]
+    st = bench.compression_stats(infos)
+    n_w = [w.size for w in ws]
+    ent, cov, raw, groups = 0.0, 0.0, 0, 0
+    for w in ws:
+        e = ((w >> 7) & 0xFF).astype(np.int64)
+        p = np.bincount(e.ravel(), minlength=256) / e.size
+        nz = p[p > 0]
+        ent += float(-(nz * np.log2(nz)).sum()) * w.size
+        cov += float(np.sort(p)[::-1][:16].sum()) * w.size
+        ref = O.encode(w)
+        raw += ref.n_raw
+        groups += ref.raw.size
+    assert abs(st["exponent_entropy_bits"] - ent / sum(n_w)) < 1e-3
+    assert abs(st["top16_coverage"] - cov / sum(n_w)) < 1e-5
+    assert abs(st["raw_group_fraction"] - raw / groups) < 1e-5
+    # (on matrices this small the Huffman form's fixed 16 KB decode table outweighs its saving)
+    assert 0 < st["compressed_fraction_huffman"] < 1 and 0 < st["compressed_fraction_palette"] < 1
+
+
 def test_plans_from_json_round_trip():
     from decode_gemm_exponent_b200 import uw
     doc = {"plans": []}
