@@ -14,8 +14,11 @@
  *        Huffman -> 4-bit palette transcode, and pre-transcoded palette.
  *   §七  reconstructive matmul: compressed tiles are staged into shared memory,
  *        rebuilt to BF16 there and fed straight to the tensor cores.
- *   §九  an autotuner measures the pipelines and kernel variants per
- *        projection and batch size and writes a per-model plan.
+ *   §九  an autotuner measures the pipelines, the kernel variants and the
+ *        decode/compute SM split per projection and batch size and writes a
+ *        per-model plan.
+ *   §十一 mixture-of-experts models are the next target (many small
+ *        expert matrices).
  *
  * Conventions for every entry point:
  *   - Returns a uw_status; nothing throws across the ABI.

@@ -377,3 +377,6 @@ def test_batched_matmul_argument_checks(uw):
     assert run(items((0, 4, fake + 8, fake)), ok) == uw.ERR_INVALID_ARG      # misaligned x
     assert run(items((0, 4, fake, None)), ok) == uw.ERR_INVALID_ARG          # no y
     assert run(items((0, 4, fake, fake), (1, 2, None, fake)), ok) == uw.ERR_INVALID_ARG
+    # experts that nobody routed to are skipped: a batch of them launches nothing and succeeds
+    # (this host has no GPU, so any launch would fail)
+    assert run(items((0, 0, None, None), (1, 0, None, None)), ok) == uw.UW_OK
