@@ -68,7 +68,7 @@ const char *uw_version(void);
 /* ------------------------------------------------------------------------ */
 /* Host encoder (Unweight page §三, §四, §六).                                */
 
-#define UW_EMIT_HUFFMAN 1u   /* Huffman exponent stream (pipelines 1 and 3)    */
+#define UW_EMIT_HUFFMAN 1u   /* Huffman exponent stream (pipelines 1, 2, 3)    */
 #define UW_EMIT_PALETTE 2u   /* pre-transcoded 4-bit palette plane (pipeline 4) */
 
 /* Sections of a blob (each 256-byte aligned inside the blob). */
