@@ -304,14 +304,9 @@ def alg_bytes(mat, m, plan):
 
 def plans_from_json(text, n_mats, uw):
     """Plans from a plan file written by the autotuner (--plan-json)."""
-    doc = json.loads(text)
-    pipes = {"decode_gemm": 1, "decode_exp_fused": 2, "transcode_fused": 3, "direct_palette": 4}
-    plans = [[None] * len(MS) for _ in range(n_mats)]
-    for e in doc["plans"]:
-        b = e["best"]
-        plans[e["matrix"]][MS.index(e["m"])] = uw.make_plan(
-            pipes[b["pipeline"]], {"fma": 1, "tc": 2, "mma": 3}[b["kernel"]], b["bn"], b["split_k"],
-            b.get("stages", 0))
+    plans = uw.plans_from_json(text, MS)
+    if len(plans) != n_mats:
+        raise ValueError("plan file holds %d matrices, the layer has %d" % (len(plans), n_mats))
     return plans
 
 

@@ -11,6 +11,7 @@ the host, torch ``int16`` (same bits) on the device.
 from __future__ import annotations
 
 import ctypes
+import json
 import os
 from typing import Optional, Sequence
 
@@ -434,6 +435,36 @@ def autotune(mats: Sequence[Matrix], ms: Sequence[int], reps: int = 5, stream=No
                                  reps, plans, js, cap, _stream_handle(stream)), "uw_plan_autotune")
     out = [[plans[i * len(ms) + j] for j in range(len(ms))] for i in range(len(mats))]
     return out, js.value.decode()
+
+
+PIPELINE_NAMES = {PIPE_DECODE_GEMM: "decode_gemm", PIPE_DECODE_EXP_FUSED: "decode_exp_fused",
+                  PIPE_TRANSCODE_FUSED: "transcode_fused", PIPE_DIRECT_PALETTE: "direct_palette"}
+KERNEL_NAMES = {KERNEL_FMA: "fma", KERNEL_TC: "tc", KERNEL_MMA: "mma"}
+
+
+def plans_from_json(text: str, ms: Sequence[int]):
+    """Reload a plan file written by uw_plan_autotune (the per-model plan of
+    Unweight page §九): plans[i][j] for matrix i and batch size ms[j].  Raises
+    ValueError when the file lacks a (matrix, m) pair or names an unknown
+    pipeline or kernel."""
+    doc = json.loads(text)
+    pipes = {v: k for k, v in PIPELINE_NAMES.items()}
+    kerns = {v: k for k, v in KERNEL_NAMES.items()}
+    ms = list(ms)
+    n_mats = 1 + max((e["matrix"] for e in doc["plans"]), default=-1)
+    plans = [[None] * len(ms) for _ in range(n_mats)]
+    for e in doc["plans"]:
+        if e["m"] not in ms:
+            continue
+        b = e["best"]
+        if b["pipeline"] not in pipes or b["kernel"] not in kerns:
+            raise ValueError("plan file: unknown pipeline or kernel in %r" % (b,))
+        plans[e["matrix"]][ms.index(e["m"])] = make_plan(pipes[b["pipeline"]], kerns[b["kernel"]], b["bn"],
+                                                         b["split_k"], b.get("stages", 0))
+    missing = [(i, ms[j]) for i in range(n_mats) for j in range(len(ms)) if plans[i][j] is None]
+    if missing:
+        raise ValueError("plan file has no plan for (matrix, m) %s" % missing[:4])
+    return plans
 
 
 lib()   # fail loudly at import when the library is missing

@@ -109,3 +109,21 @@ def test_plans_from_json_round_trip():
             # every plan has a kernel group and a launch count; pipelines 1-3 add a preprocessing launch
             assert bench.kernel_group(p).split("/")[0]
             assert bench.launches_per_call(p) >= (2 if p.pipeline != uw.PIPE_DIRECT_PALETTE else 1)
+
+
+def test_plan_file_reader_rejects_incomplete_or_unknown_plans():
+    import pytest
+    from decode_gemm_exponent_b200 import uw
+    best = {"pipeline": "direct_palette", "kernel": "mma", "bn": 4, "split_k": 1, "stages": 2, "us": 1.0}
+    doc = {"plans": [{"matrix": 0, "n": 64, "k": 64, "m": 1, "best": best, "candidates": [best]},
+                     {"matrix": 1, "n": 64, "k": 64, "m": 1, "best": best, "candidates": [best]}]}
+    plans = uw.plans_from_json(json.dumps(doc), [1])
+    assert len(plans) == 2 and plans[1][0].kernel == uw.KERNEL_MMA and plans[1][0].stages == 2
+    with pytest.raises(ValueError):                       # no plan for m = 4
+        uw.plans_from_json(json.dumps(doc), [1, 4])
+    bad = json.loads(json.dumps(doc))
+    bad["plans"][1]["best"]["kernel"] = "wgmma"
+    with pytest.raises(ValueError):
+        uw.plans_from_json(json.dumps(bad), [1])
+    with pytest.raises(ValueError):                       # the bench's layer has three matrices
+        bench.plans_from_json(json.dumps(doc), 3, uw)
