@@ -57,6 +57,8 @@ def _cases():
         "one_exponent": one_exp.astype(np.uint16).reshape(64, 128),
         "heavy_outliers": synth.weights_bf16(64, 512, 0.015, 0.05, 1.0, seed=5),
         "wide_sigma": synth.weights_bf16(64, 256, 0.05, 0.0, 1.0, seed=6),
+        # a mixture-of-experts expert's gate shape, as the batched matmul runs it
+        "moe_expert_768x2048": synth.weights_bf16(768, 2048, 0.02, 0.0005, 1.0, seed=1),
     }
 
 
