@@ -382,3 +382,28 @@ def test_batched_matmul_argument_checks(uw):
     # experts that nobody routed to are skipped: a batch of them launches nothing and succeeds
     # (this host has no GPU, so any launch would fail)
     assert run(items((0, 0, None, None), (1, 0, None, None)), ok) == uw.UW_OK
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/uw.h is a C interface: it compiles as pedantic C99 and every
+    declared entry point links against the library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_uw.c"
+    src.write_text('#include "uw.h"\n'
+                   'int main(void) {\n'
+                   '    uw_batch_item it = {0}; uw_stack_step st = {0}; uw_plan p = {0}; uw_sm_split *s = 0;\n'
+                   '    (void)it; (void)st; (void)p; (void)s;\n'
+                   '    return uw_status_str(UW_OK)[0] == 0;\n'
+                   '}\n')
+    cuda_inc = "/usr/local/cuda/include"
+    lib_dir = os.path.join(root, "decode_gemm_exponent_b200")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(root, "include"), "-I", cuda_inc, str(src),
+                        "-L", lib_dir, "-l:libuw.so", "-o", str(tmp_path / "use_uw")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
