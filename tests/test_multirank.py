@@ -43,9 +43,9 @@ def _worker(rank, world, port, out):
 def test_two_rank_weak_scaling_logic():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    ctx = mp.get_context("spawn")     # no fork anywhere: the parent may hold threads (or a CUDA context)
+    mgr = ctx.Manager()
     out = mgr.dict()
-    ctx = mp.get_context("spawn")
     procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
     for p in procs:
         p.start()
