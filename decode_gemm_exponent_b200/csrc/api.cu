@@ -34,6 +34,8 @@ uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
     } else if (p->kernel == UW_KERNEL_TC) {
         if (!valid_bn_tc(p->bn) || p->split_k < 1 || p->split_k > 64 || p->stages < 0 || p->stages > 8)
             return UW_ERR_INVALID_ARG;
+    } else if (p->kernel == UW_KERNEL_TC_SK) {
+        if (!valid_bn_tc(p->bn) || p->split_k != 1 || p->stages < 0 || p->stages > 8) return UW_ERR_INVALID_ARG;
     } else {
         return UW_ERR_INVALID_ARG;
     }
@@ -41,7 +43,14 @@ uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
     return UW_OK;
 }
 
-uint64_t partial_bytes(int64_t m, int64_t n, const uw_plan *p) {
+// Scratch after the preprocessing output: split-K partial sums, or for the
+// stream-K kernel its tile counters (unless the caller keeps them apart,
+// `own_counters`) followed by its partial tiles.
+uint64_t partial_bytes(int64_t m, int64_t n, int64_t k, const uw_plan *p, bool own_counters = false) {
+    if (p->kernel == UW_KERNEL_TC_SK) {
+        const SkGeometry g = sk_geometry(m, n, k, p->bn);
+        return (own_counters ? 0 : g.counter_bytes) + g.partial_bytes;
+    }
     if (p->kernel != UW_KERNEL_TC || p->split_k <= 1) return 0;
     return align_up(uint64_t(p->split_k) * uint64_t(m) * uint64_t(n) * 4, 256);
 }
@@ -51,7 +60,7 @@ uint64_t prep_bytes(int64_t n, int64_t k, const uw_plan *p) { return prep_worksp
 // Run one matmul kernel on prepared weights: w_bf16 (plain) or pal (fused).
 uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const uw_dmat *w,
                      const uint8_t *pal, int64_t n, int64_t k, float *y, const uw_plan *plan,
-                     float *partial, uint32_t *status, cudaStream_t stream) {
+                     float *partial, uint32_t *status, uint32_t *sk_counters, cudaStream_t stream) {
     if (plan->kernel == UW_KERNEL_FMA)
         return cuda_status(launch_gemv_fma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, status, stream));
     if (plan->kernel == UW_KERNEL_MMA)
@@ -72,6 +81,17 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
     t.debug_flags = plan->debug_flags;
     t.timeout_ns = plan->timeout_ns > 0 ? uint64_t(plan->timeout_ns) : kDefaultTimeoutNs;
     t.dev_status = status;
+    if (plan->kernel == UW_KERNEL_TC_SK) {
+        uint8_t *base = reinterpret_cast<uint8_t *>(partial);
+        if (!base) return UW_ERR_WORKSPACE;
+        if (sk_counters) {
+            t.sk_counters = sk_counters;
+        } else {
+            t.sk_counters = reinterpret_cast<uint32_t *>(base);
+            t.partial = reinterpret_cast<float *>(base + sk_geometry(m, n, k, plan->bn).counter_bytes);
+        }
+        return cuda_status(launch_gemm_sk(t, stream));
+    }
     return cuda_status(launch_gemm_tc(t, stream));
 }
 
@@ -205,23 +225,29 @@ extern "C" uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw
     if (!bytes || m <= 0 || n <= 0 || k <= 0) return UW_ERR_INVALID_ARG;
     uw_status st = check_plan(plan, m, k);
     if (st != UW_OK) return st;
-    *bytes = size_t(prep_bytes(n, k, plan) + partial_bytes(m, n, plan));
+    *bytes = size_t(prep_bytes(n, k, plan) + partial_bytes(m, n, k, plan));
     return UW_OK;
 }
 
-extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_dmat *w,
-                                     const uint8_t *pal_dev, float *y_dev, const uw_plan *plan,
-                                     void *ws, size_t ws_bytes, void *stream) {
+namespace uw {
+
+uint64_t sk_counter_bytes(int64_t m, int64_t n, int64_t k, const uw_plan *plan) {
+    if (!plan || plan->kernel != UW_KERNEL_TC_SK || m <= 0) return 0;
+    return sk_geometry(m, n, k, plan->bn).counter_bytes;
+}
+
+uw_status fused_matmul_ex(const uint16_t *x_dev, int64_t m, const uw_dmat *w, const uint8_t *pal_dev, float *y_dev,
+                          const uw_plan *plan, void *ws, size_t ws_bytes, uint32_t *sk_counters, cudaStream_t s) {
     uw_status st = check_dmat(w);
     if (st != UW_OK) return st;
     if (!x_dev || !y_dev || m <= 0) return UW_ERR_INVALID_ARG;
     if (!aligned(x_dev, 16) || !aligned(y_dev, 16)) return UW_ERR_INVALID_ARG;
     st = check_plan(plan, m, w->k);
     if (st != UW_OK) return st;
-    const uint64_t need_prep = prep_bytes(w->n, w->k, plan), need_part = partial_bytes(m, w->n, plan);
+    const uint64_t need_prep = prep_bytes(w->n, w->k, plan),
+                   need_part = partial_bytes(m, w->n, w->k, plan, sk_counters != nullptr);
     if (need_prep + need_part > 0 && (!ws || ws_bytes < need_prep + need_part || !aligned(ws, 256)))
         return UW_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     float *partial = need_part ? reinterpret_cast<float *>(wsb + need_prep) : nullptr;
 
@@ -231,7 +257,7 @@ extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_
         st = cuda_status(launch_huff_decode(*w, wd, nullptr, s));
         if (st != UW_OK) return st;
         return run_kernel(x_dev, m, wd, nullptr, nullptr, w->n, w->k, y_dev, plan, partial,
-                          w->dev_status, s);
+                          w->dev_status, sk_counters, s);
     }
     if (plan->pipeline == UW_PIPE_DECODE_EXP_FUSED) {
         if (!(w->flags & UW_EMIT_HUFFMAN)) return UW_ERR_INVALID_ARG;
@@ -240,7 +266,8 @@ extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_
                                            reinterpret_cast<uint32_t *>(wsb + L.rank_off), s));
         if (st != UW_OK) return st;
         const uw_dmat v = exp_plane_view(*w, wsb);
-        return run_kernel(x_dev, m, nullptr, &v, v.pal, w->n, w->k, y_dev, plan, partial, w->dev_status, s);
+        return run_kernel(x_dev, m, nullptr, &v, v.pal, w->n, w->k, y_dev, plan, partial, w->dev_status,
+                          sk_counters, s);
     }
     const uint8_t *pal = nullptr;
     if (plan->pipeline == UW_PIPE_TRANSCODE_FUSED) {
@@ -252,7 +279,30 @@ extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_
         pal = pal_dev ? pal_dev : w->pal;
         if (!pal || !aligned(pal, 16)) return UW_ERR_INVALID_ARG;
     }
-    return run_kernel(x_dev, m, nullptr, w, pal, w->n, w->k, y_dev, plan, partial, w->dev_status, s);
+    return run_kernel(x_dev, m, nullptr, w, pal, w->n, w->k, y_dev, plan, partial, w->dev_status, sk_counters, s);
+}
+
+uw_status matmul_bf16_ex(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev, int64_t n, int64_t k, float *y_dev,
+                         const uw_plan *plan, void *ws, size_t ws_bytes, uint32_t *dev_status, uint32_t *sk_counters,
+                         cudaStream_t s) {
+    if (!x_dev || !w_dev || !y_dev || m <= 0 || n <= 0 || k <= 0) return UW_ERR_INVALID_ARG;
+    if (n % 64 || k % 64) return UW_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(x_dev, 16) || !aligned(w_dev, 16) || !aligned(y_dev, 16)) return UW_ERR_INVALID_ARG;
+    uw_status st = check_plan(plan, m, k);
+    if (st != UW_OK) return st;
+    const uint64_t need = partial_bytes(m, n, k, plan, sk_counters != nullptr);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 256))) return UW_ERR_WORKSPACE;
+    return run_kernel(x_dev, m, w_dev, nullptr, nullptr, n, k, y_dev, plan, need ? static_cast<float *>(ws) : nullptr,
+                      dev_status, sk_counters, s);
+}
+
+}  // namespace uw
+
+extern "C" uw_status uw_fused_matmul(const uint16_t *x_dev, int64_t m, const uw_dmat *w,
+                                     const uint8_t *pal_dev, float *y_dev, const uw_plan *plan,
+                                     void *ws, size_t ws_bytes, void *stream) {
+    return fused_matmul_ex(x_dev, m, w, pal_dev, y_dev, plan, ws, ws_bytes, nullptr,
+                           static_cast<cudaStream_t>(stream));
 }
 
 extern "C" uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const uw_plan *plan,
@@ -280,14 +330,6 @@ extern "C" uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_i
 extern "C" uw_status uw_matmul_bf16(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev,
                                     int64_t n, int64_t k, float *y_dev, const uw_plan *plan,
                                     void *ws, size_t ws_bytes, uint32_t *dev_status, void *stream) {
-    if (!x_dev || !w_dev || !y_dev || m <= 0 || n <= 0 || k <= 0) return UW_ERR_INVALID_ARG;
-    if (n % 64 || k % 64) return UW_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned(x_dev, 16) || !aligned(w_dev, 16) || !aligned(y_dev, 16)) return UW_ERR_INVALID_ARG;
-    uw_status st = check_plan(plan, m, k);
-    if (st != UW_OK) return st;
-    const uint64_t need = partial_bytes(m, n, plan);
-    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 256))) return UW_ERR_WORKSPACE;
-    return run_kernel(x_dev, m, w_dev, nullptr, nullptr, n, k, y_dev, plan,
-                      need ? static_cast<float *>(ws) : nullptr, dev_status,
-                      static_cast<cudaStream_t>(stream));
+    return matmul_bf16_ex(x_dev, m, w_dev, n, k, y_dev, plan, ws, ws_bytes, dev_status, nullptr,
+                          static_cast<cudaStream_t>(stream));
 }

@@ -74,6 +74,15 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
             }
         int bn_hi = 16;
         while (bn_hi < m && bn_hi < 256) bn_hi *= 2;
+        for (int bn : {bn_hi / 2, bn_hi}) {   // persistent stream-K kernel
+            if (bn < 16) continue;
+            uw_plan p{};
+            p.pipeline = pipe;
+            p.kernel = UW_KERNEL_TC_SK;
+            p.bn = bn;
+            p.split_k = 1;
+            out.push_back(p);
+        }
         for (int bn : {bn_hi / 2, bn_hi}) {
             if (bn < 16) continue;
             const int64_t tiles = ((w.n + 127) / 128) * ((m + bn - 1) / bn);
@@ -102,12 +111,21 @@ const char *pipe_name(int p) {
     }
 }
 
+const char *kernel_name(int k) {
+    switch (k) {
+        case UW_KERNEL_FMA: return "fma";
+        case UW_KERNEL_MMA: return "mma";
+        case UW_KERNEL_TC_SK: return "tc_sk";
+        default: return "tc";
+    }
+}
+
 std::string plan_json(const uw_plan &p, double us) {
     char buf[256];
     std::snprintf(buf, sizeof buf,
                   "{\"pipeline\": \"%s\", \"kernel\": \"%s\", \"bn\": %d, \"split_k\": %d, \"stages\": %d, "
                   "\"us\": %.3f}",
-                  pipe_name(p.pipeline), p.kernel == UW_KERNEL_FMA ? "fma" : p.kernel == UW_KERNEL_MMA ? "mma" : "tc",
+                  pipe_name(p.pipeline), kernel_name(p.kernel),
                   p.bn, p.split_k, p.stages, us);
     return buf;
 }
@@ -163,6 +181,15 @@ extern "C" uw_status uw_plan_autotune(const uw_dmat *const *mats, int n_mats, co
             uw_plan best{};
             std::string cand_json;
             for (const uw_plan &p : candidates(w, m)) {
+                // other candidates' partial sums share the front of the
+                // workspace: a stream-K candidate starts from zeroed counters
+                // (each completed call leaves them zero for its repetitions)
+                const uint64_t cnt = uw::sk_counter_bytes(m, w.n, w.k, &p);
+                if (cnt && cudaMemsetAsync(static_cast<uint8_t *>(ws) + uw::prep_workspace_bytes(w.n, w.k, p.pipeline),
+                                           0, cnt, s) != cudaSuccess) {
+                    result = UW_ERR_CUDA;
+                    break;
+                }
                 uw_status st = uw_fused_matmul(x_dev, m, &w, nullptr, y_dev, &p, ws, cand_bytes, stream);
                 if (st == UW_OK) st = w.dev_status ? uw_device_status(&w, stream)
                                                    : (cudaStreamSynchronize(s) == cudaSuccess ? UW_OK : UW_ERR_CUDA);

@@ -85,6 +85,50 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     return true;
 }
 
+// Potentially blocking test: the thread may be suspended in hardware until
+// the phase completes or a system-defined time slice ends, so waiting warps
+// take few issue slots from the working ones.
+__device__ __forceinline__ bool mbar_try_wait_susp(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait that also gives up as soon as *abort is set by another role of
+// the CTA (so one time-out ends every wait of the CTA quickly).  Returns
+// false on time-out or abort.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                                   const volatile int *abort) {
+    if (mbar_try_wait_susp(bar, parity)) return true;
+    const long long limit = (long long)(timeout_ns * 2);
+    const long long t0 = clock64();
+    while (!mbar_try_wait_susp(bar, parity)) {
+        if (*abort || clock64() - t0 > limit) return false;
+    }
+    return true;
+}
+
+// Named barrier over `threads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also ORs a predicate over its threads: every thread
+// gets the same answer, so the threads can take one branch together.
+__device__ __forceinline__ bool named_bar_any(uint32_t id, uint32_t threads, bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, q; }"
+        : "=r"(out)
+        : "r"(uint32_t(pred)), "r"(id), "r"(threads)
+        : "memory");
+    return out != 0;
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes and

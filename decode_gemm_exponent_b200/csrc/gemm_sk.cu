@@ -1,0 +1,673 @@
+// gemm_sk.cu -- persistent stream-K tensor-core matmul Y = X * W^T on sm_100a
+// (tcgen05 MMA, TMEM accumulators), in a fused flavour that rebuilds W from
+// its compressed planes in shared memory (Unweight page §七, reconstructive
+// matmul; §五, decompressed weights never go back to HBM) and a plain flavour
+// that loads BF16 W (the uncompressed baseline and the bit-exactness twin).
+//
+// Work decomposition.  A tile is 128 rows of W (the MMA's M) by BN tokens
+// (the MMA's N); a unit is one 64-wide K-step of one tile.  Tiles are ordered
+// row block major (the token blocks of one row block are neighbours, so a
+// compressed W tile read by one CTA is still in L2 for the next).  The grid
+// has one CTA per SM (G = min(SMs, units)), and CTA c owns the contiguous unit
+// range [c*U/G, (c+1)*U/G), so every SM gets the same number of K-steps
+// whatever the shape (no partial last wave).  A tile whose K range is cut
+// between CTAs ("split") is summed by a fix-up: every CTA holding a piece
+// writes its fp32 partial tile to the workspace and bumps the tile's counter;
+// the CTA that brings the counter to the number of pieces adds all pieces in
+// CTA order (= K order) and writes Y, then zeroes the counter.  No CTA waits
+// for another, and the sum order is fixed by the schedule alone, so the plain
+// and fused flavours (same schedule, same MMA sequence) give identical bits.
+//
+// Roles (warps):
+//   0      producer: fused -- per K-step the sign/mantissa tile (TMA, 64-byte
+//          swizzle) and the 4-bit palette tile (TMA, 32-byte swizzle), and
+//          for each raw (row, group) its 64 exponents by a 64-byte bulk copy,
+//          all counted on one barrier; the 32 lanes share the 128 rows' raw
+//          bits and write the step's 128-bit raw mask next to the stage.
+//          plain -- the BF16 W tile (TMA, 128-byte swizzle) into the W ring.
+//   1      MMA issuer and TMEM owner: 4 x tcgen05.mma (K = 16) per K-step into
+//          one of two accumulators (double-buffered, so the epilogue of one
+//          tile overlaps the MMAs of the next).
+//   2      X producer (TMA, 128-byte swizzle).
+//   3-6    epilogue: TMEM -> registers -> Y (or a partial tile + fix-up).
+//   7-14   (fused) rebuild: all 8 warps work on the same K-step; thread t
+//          rebuilds 32 weights (half h = t & 1) of tile row r = t >> 1 into
+//          the 128-byte-swizzled K-major BF16 W tile.  The thread-to-data map
+//          keeps every 16-byte shared-memory access of a quarter warp on
+//          distinct bank groups (sign/mantissa, palette words and W stores).
+// Every wait is bounded; on time-out a role raises UW_DEVERR_TIMEOUT and sets
+// the CTA's abort flag, which ends every other wait of the CTA; TMA copies
+// and MMAs in flight are waited for (bounded) before TMEM is freed.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "device_common.cuh"
+#include "kernels.h"
+#include "uw_format.h"
+
+namespace uw {
+namespace {
+
+using namespace dev;
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kMaxSmem = 232448;        // 227 KB opt-in per CTA
+constexpr int kFixedWarps = 7;          // producer, MMA, X producer, 4 epilogue warps
+constexpr int kRebuildWarps = 8;
+constexpr int kEpiWarp0 = 3;
+constexpr int kFirstRebuildWarp = kFixedWarps;
+constexpr int kFusedThreads = (kFixedWarps + kRebuildWarps) * 32;
+constexpr int kPlainThreads = kFixedWarps * 32;
+
+constexpr int kTileW = kBM * kBK * 2;            // BF16 W tile
+constexpr int kTileSM = kBM * kBK;               // sign/mantissa tile
+constexpr int kTilePL = kBM * kBK / 2;           // 4-bit palette tile
+constexpr int kTileRAW = kBM * kGroup;           // one 64-byte exponent slot per row
+constexpr int kCStage = kTileSM + kTilePL + kTileRAW;
+constexpr int kOffPL = kTileSM, kOffRAW = kTileSM + kTilePL;
+
+struct SkArgs {
+    int64_t m, n, k;
+    int64_t units;            // tiles * S
+    int S;                    // K-steps per tile
+    int TB;                   // token blocks
+    int G;                    // CTAs
+    int dc, dw, dx;           // ring depths: compressed, W, X
+    uint32_t debug_flags;
+    uint64_t timeout_ns;
+    float *y;
+    uint32_t *counters;       // [tiles], zero between calls
+    float *partial;           // [2G][BN][128]
+    const uint32_t *flagbits;
+    const uint32_t *rawbase;
+    const uint8_t *rawexp;
+    int64_t nflag;            // words of flagbits
+    Palette16 pal;
+    uint32_t *status;
+};
+
+// first unit of CTA c; the CTA holding unit u
+__host__ __device__ __forceinline__ int64_t sk_unit0(int64_t c, int64_t units, int G) { return c * units / G; }
+__host__ __device__ __forceinline__ int sk_cta_of(int64_t u, int64_t units, int G) {
+    return int(((u + 1) * G - 1) / units);
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+template <int BN>
+struct SkCfg {
+    static constexpr int kX = BN * kBK * 2;
+    static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32u : uint32_t(2 * BN);   // two accumulators
+    static_assert(kX % 1024 == 0, "X stage keeps 1024-byte alignment");
+    static_assert(2 * BN <= 512, "accumulators exceed TMEM");
+};
+
+// shared-memory bytes after the rings: raw masks, barriers, TMEM slot, flags
+__host__ __device__ constexpr int sk_tail(int dc, int dw, int dx) {
+    return dc * 16 + (2 * dc + 2 * dw + 2 * dx + 4 + 2) * 8 + 16;
+}
+
+template <bool FUSED, int BN>
+__device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMap *tmA, const CUtensorMap *tmB,
+                                        const SkArgs &a) {
+    using C = SkCfg<BN>;
+    extern __shared__ uint8_t smem_dyn[];
+    const int dc = FUSED ? a.dc : 0, dw = a.dw, dx = a.dx;
+    uint8_t *wring = align1024(smem_dyn);
+    uint8_t *xring = wring + size_t(dw) * kTileW;
+    uint8_t *cring = xring + size_t(dx) * C::kX;
+    uint32_t *masks = reinterpret_cast<uint32_t *>(cring + size_t(dc) * kCStage);   // [dc][4]
+    uint64_t *c_full = reinterpret_cast<uint64_t *>(masks + 4 * dc);
+    uint64_t *c_empty = c_full + dc;
+    uint64_t *w_full = c_empty + dc;
+    uint64_t *w_empty = w_full + dw;
+    uint64_t *x_full = w_empty + dw;
+    uint64_t *x_empty = x_full + dx;
+    uint64_t *acc_full = x_empty + dx;      // [2]
+    uint64_t *acc_empty = acc_full + 2;     // [2]
+    uint64_t *never = acc_empty + 2;
+    uint64_t *mma_done = never + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *last_flag = abort_flag + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t T = a.timeout_ns;
+    const int64_t u0 = sk_unit0(blockIdx.x, a.units, a.G), u1 = sk_unit0(int64_t(blockIdx.x) + 1, a.units, a.G);
+    const int nu = int(u1 - u0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < dc; s++) {
+            mbar_init(&c_full[s], 1);
+            mbar_init(&c_empty[s], kRebuildWarps);
+        }
+        for (int s = 0; s < dw; s++) {
+            mbar_init(&w_full[s], FUSED ? kRebuildWarps : 1);
+            mbar_init(&w_empty[s], 1);
+        }
+        for (int s = 0; s < dx; s++) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(never, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(tmX);
+        prefetch_tensormap(tmA);
+        if (FUSED) prefetch_tensormap(tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto fail = [&](bool timed_out) {
+        if (timed_out) flag_error(a.status, UW_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int issued = 0;
+        if constexpr (FUSED) {
+            const int64_t G64 = a.k / kGroup;     // groups per row
+            int64_t wcur[4] = {-1, -1, -1, -1};
+            uint32_t bm[4] = {0u, 0u, 0u, 0u}, rb[4] = {0u, 0u, 0u, 0u};
+            for (int i = 0; i < nu; i++) {
+                const int64_t u = u0 + i;
+                const int64_t t = u / a.S;
+                const int ks = int(u - t * a.S);
+                const int64_t n0 = (t / a.TB) * kBM;
+                const int s = i % dc;
+                // raw bits and ranks of this lane's rows r = lane + 32 j
+                uint32_t rawbits = 0u, rank[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int64_t row = n0 + lane + 32 * j;
+                    if (row < a.n) {
+                        const int64_t g = row * G64 + ks;
+                        const int64_t w = g >> 5;
+                        if (w != wcur[j]) {
+                            bm[j] = __ldg(a.flagbits + w);
+                            rb[j] = __ldg(a.rawbase + w);
+                            wcur[j] = w;
+                            if (w + 1 < a.nflag) {   // the next word into L1 before it is needed
+                                prefetch_l1(a.flagbits + w + 1);
+                                prefetch_l1(a.rawbase + w + 1);
+                            }
+                        }
+                        const uint32_t bit = uint32_t(g) & 31u;
+                        if ((bm[j] >> bit) & 1u) {
+                            rawbits |= 1u << j;
+                            rank[j] = rb[j] + __popc(bm[j] & ((1u << bit) - 1u));
+                        }
+                    }
+                }
+                const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, rawbits & 1u);
+                const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, rawbits & 2u);
+                const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, rawbits & 4u);
+                const uint32_t m3 = __ballot_sync(0xFFFFFFFFu, rawbits & 8u);
+                const uint32_t nraw = __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
+                int ok = 1, stop = 0;
+                if (lane == 0) {
+                    if (i >= dc) ok = mbar_wait_or_abort(&c_empty[s], (uint32_t(i / dc) & 1u) ^ 1u, T, abort_flag);
+                    if (!ok) fail(!*abort_flag);
+                    stop = !ok || *abort_flag;
+                }
+                if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
+                uint8_t *st = cring + size_t(s) * kCStage;
+                if (lane == 0) {
+                    masks[4 * s + 0] = m0;
+                    masks[4 * s + 1] = m1;
+                    masks[4 * s + 2] = m2;
+                    masks[4 * s + 3] = m3;
+                    mbar_arrive_expect_tx(&c_full[s], uint32_t(kTileSM + kTilePL) + uint32_t(kGroup) * nraw);
+                    tma_load_2d(st, tmA, ks * kBK, int32_t(n0), &c_full[s]);
+                    tma_load_2d(st + kOffPL, tmB, ks * (kBK / 2), int32_t(n0), &c_full[s]);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    if ((rawbits >> j) & 1u)
+                        bulk_g2s(st + kOffRAW + (lane + 32 * j) * kGroup, a.rawexp + uint64_t(rank[j]) * kGroup,
+                                 kGroup, &c_full[s]);
+                issued = i + 1;
+            }
+            // no copy may still be landing when the CTA exits
+            if (lane == 0)
+                for (int i = max(0, issued - dc); i < issued; i++)
+                    mbar_wait(&c_full[i % dc], uint32_t(i / dc) & 1u, T);
+        } else if (lane == 0) {
+            for (int i = 0; i < nu; i++) {
+                const int64_t u = u0 + i;
+                const int64_t t = u / a.S;
+                const int ks = int(u - t * a.S);
+                const int64_t n0 = (t / a.TB) * kBM;
+                const int s = i % dw;
+                if (i >= dw && !mbar_wait_or_abort(&w_empty[s], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag)) {
+                    fail(!*abort_flag);
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_arrive_expect_tx(&w_full[s], uint32_t(kTileW));
+                tma_load_2d(wring + size_t(s) * kTileW, tmA, ks * kBK, int32_t(n0), &w_full[s]);
+                issued = i + 1;
+            }
+            for (int i = max(0, issued - dw); i < issued; i++)
+                mbar_wait(&w_full[i % dw], uint32_t(i / dw) & 1u, T);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+            bool ok = true;
+            if (a.debug_flags & UW_DEBUG_NEVER_ARRIVE) ok = mbar_wait_or_abort(never, 0, T, abort_flag);
+            int seg = -1;
+            int64_t tprev = -1;
+            bool first = true;
+            for (int i = 0; i < nu && ok; i++) {
+                const int64_t u = u0 + i;
+                const int64_t t = u / a.S;
+                if (t != tprev) {   // a new tile: close the previous accumulator, claim the next
+                    if (seg >= 0) tc_commit(&acc_full[seg & 1]);
+                    seg++;
+                    tprev = t;
+                    if (seg >= 2)
+                        ok = mbar_wait_or_abort(&acc_empty[seg & 1], (uint32_t(seg >> 1) & 1u) ^ 1u, T, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    first = true;
+                }
+                const int xs = i % dx, ws = i % dw;
+                ok = mbar_wait_or_abort(&x_full[xs], uint32_t(i / dx) & 1u, T, abort_flag) &&
+                     mbar_wait_or_abort(&w_full[ws], uint32_t(i / dw) & 1u, T, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t sa = smem_addr(wring + size_t(ws) * kTileW);
+                const uint32_t sb = smem_addr(xring + size_t(xs) * C::kX);
+                const uint32_t d = tmem + uint32_t((seg & 1) * BN);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; kk++)
+                    tc_mma_bf16(d, smem_desc_k128(sa + 32 * kk), smem_desc_k128(sb + 32 * kk), idesc,
+                                (!first || kk) ? 1u : 0u);
+                first = false;
+                tc_commit(&w_empty[ws]);
+                tc_commit(&x_empty[xs]);
+            }
+            if (ok) {
+                if (seg >= 0) tc_commit(&acc_full[seg & 1]);
+            } else {
+                fail(!*abort_flag);
+                // every MMA issued so far must finish before TMEM is freed
+                tc_commit(mma_done);
+                mbar_wait(mma_done, 0, T);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ X producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nu; i++) {
+                const int64_t u = u0 + i;
+                const int64_t t = u / a.S;
+                const int ks = int(u - t * a.S);
+                const int64_t m0 = (t % a.TB) * BN;
+                const int s = i % dx;
+                if (i >= dx && !mbar_wait_or_abort(&x_empty[s], (uint32_t(i / dx) & 1u) ^ 1u, T, abort_flag)) {
+                    fail(!*abort_flag);
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_arrive_expect_tx(&x_full[s], uint32_t(C::kX));   // rows past m read the zero fill
+                tma_load_2d(xring + size_t(s) * C::kX, tmX, ks * kBK, int32_t(m0), &x_full[s]);
+                issued = i + 1;
+            }
+            for (int i = max(0, issued - dx); i < issued; i++)
+                mbar_wait(&x_full[i % dx], uint32_t(i / dx) & 1u, T);
+        }
+        __syncwarp();
+    } else if (warp < kFirstRebuildWarp) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;               // TMEM lane quarter this warp may read
+        const int r = q * 32 + lane;          // tile row
+        const int64_t t_first = nu > 0 ? u0 / a.S : 0, t_last = nu > 0 ? (u1 - 1) / a.S : -1;
+        int seg = -1;
+        for (int64_t t = t_first; t <= t_last; t++) {
+            seg++;
+            const int b = seg & 1;
+            const int64_t ka = t == t_first ? u0 - t * a.S : 0;
+            const int64_t kb = t == t_last ? u1 - t * a.S : a.S;
+            const bool split = ka != 0 || kb != a.S;
+            const int slot = t == t_first ? 0 : 1;
+            const bool ok = mbar_wait_or_abort(&acc_full[b], uint32_t(seg >> 1) & 1u, T, abort_flag);
+            // the four epilogue warps decide together, so that all of them
+            // meet the same named barriers below
+            if (named_bar_any(1, 128, !ok)) {
+                if (!ok && lane == 0 && !*abort_flag) fail(true);
+                break;
+            }
+            tc_fence_after();
+            const int64_t n0 = (t / a.TB) * kBM, m0 = (t % a.TB) * BN;
+            const int64_t row = n0 + r;
+            float *pout = a.partial + (int64_t(2 * blockIdx.x + slot) * BN) * kBM + r;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(b * BN + c0), v);
+                tmem_ld_wait();
+                if (split) {
+#pragma unroll
+                    for (int j = 0; j < 16; j++) pout[(c0 + j) * kBM] = __uint_as_float(v[j]);
+                } else if (row < a.n) {
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        const int64_t tok = m0 + c0 + j;
+                        if (tok < a.m) a.y[tok * a.n + row] = __uint_as_float(v[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+            if (!split) continue;
+            // fix-up: the last piece of the tile to arrive sums all pieces in CTA order
+            __threadfence();
+            named_bar_sync(1, 128);
+            const int ca = sk_cta_of(t * a.S, a.units, a.G), cb = sk_cta_of(t * a.S + a.S - 1, a.units, a.G);
+            if (warp == kEpiWarp0 && lane == 0) {
+                const uint32_t old = atomicAdd(a.counters + t, 1u);
+                *last_flag = old == uint32_t(cb - ca) ? 1 : 0;
+            }
+            named_bar_sync(1, 128);
+            if (*last_flag) {
+                __threadfence();
+                if (row < a.n) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < BN; c0 += 8) {
+                        float acc[8];
+#pragma unroll
+                        for (int j = 0; j < 8; j++) acc[j] = 0.f;
+                        for (int c = ca; c <= cb; c++) {
+                            const int sl = (t == sk_unit0(c, a.units, a.G) / a.S) ? 0 : 1;
+                            const float *pin = a.partial + (int64_t(2 * c + sl) * BN + c0) * kBM + r;
+                            float v[8];
+#pragma unroll
+                            for (int j = 0; j < 8; j++) v[j] = __ldcg(pin + j * kBM);
+                            if (c == ca) {
+#pragma unroll
+                                for (int j = 0; j < 8; j++) acc[j] = v[j];
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 8; j++) acc[j] += v[j];
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; j++) {
+                            const int64_t tok = m0 + c0 + j;
+                            if (tok < a.m) a.y[tok * a.n + row] = acc[j];
+                        }
+                    }
+                }
+                if (warp == kEpiWarp0 && lane == 0) a.counters[t] = 0u;
+            }
+        }
+    } else if constexpr (FUSED) {
+        // ------------------------------------------------------------ rebuild
+        const int tid = threadIdx.x - 32 * kFirstRebuildWarp;   // 0..255
+        const int r = tid >> 1, h = tid & 1;
+        const int sw64 = (r >> 1) & 3, sw32 = (r >> 2) & 1, sw128 = r & 7;
+        const Palette16 P = a.pal;
+        for (int i = 0; i < nu; i++) {
+            const int cs = i % dc, ws = i % dw;
+            bool ok = mbar_wait_or_abort(&c_full[cs], uint32_t(i / dc) & 1u, T, abort_flag);
+            if (ok && i >= dw) ok = mbar_wait_or_abort(&w_empty[ws], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag);
+            if (__any_sync(0xFFFFFFFFu, !ok)) {
+                if (lane == 0 && !*abort_flag) fail(true);
+                break;
+            }
+            const uint8_t *st = cring + size_t(cs) * kCStage;
+            const bool raw = (masks[4 * cs + (r >> 5)] >> (r & 31)) & 1u;
+            const uint8_t *smrow = st + r * 64;
+            const uint4 s0 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h) ^ sw64) << 4));
+            const uint4 s1 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h + 1) ^ sw64) << 4));
+            uint32_t rv[8];
+            if (raw) {
+                const uint8_t *rp = st + kOffRAW + r * kGroup + h * 32;
+                const uint4 e0 = *reinterpret_cast<const uint4 *>(rp);
+                const uint4 e1 = *reinterpret_cast<const uint4 *>(rp + 16);
+                rv[0] = rot4(e0.x); rv[1] = rot4(e0.y); rv[2] = rot4(e0.z); rv[3] = rot4(e0.w);
+                rv[4] = rot4(e1.x); rv[5] = rot4(e1.y); rv[6] = rot4(e1.z); rv[7] = rot4(e1.w);
+            } else {
+                const uint4 p = *reinterpret_cast<const uint4 *>(st + kOffPL + r * 32 + ((h ^ sw32) << 4));
+                pal_rot(p.x, P, rv[0], rv[1]);
+                pal_rot(p.y, P, rv[2], rv[3]);
+                pal_rot(p.z, P, rv[4], rv[5]);
+                pal_rot(p.w, P, rv[6], rv[7]);
+            }
+            // the stage's bytes are all in registers: hand it back to the producer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c_empty[cs]);
+            uint8_t *wrow = wring + size_t(ws) * kTileW + r * 128;
+            const int c0 = 4 * h;
+            *reinterpret_cast<uint4 *>(wrow + (((c0 + 0) ^ sw128) << 4)) = join8(rv[0], rv[1], s0.x, s0.y);
+            *reinterpret_cast<uint4 *>(wrow + (((c0 + 1) ^ sw128) << 4)) = join8(rv[2], rv[3], s0.z, s0.w);
+            *reinterpret_cast<uint4 *>(wrow + (((c0 + 2) ^ sw128) << 4)) = join8(rv[4], rv[5], s1.x, s1.y);
+            *reinterpret_cast<uint4 *>(wrow + (((c0 + 3) ^ sw128) << 4)) = join8(rv[6], rv[7], s1.z, s1.w);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&w_full[ws]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    k_gemm_sk_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmSM,
+                    const __grid_constant__ CUtensorMap tmPL, const SkArgs a) {
+    sk_body<true, BN>(&tmX, &tmSM, &tmPL, a);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kPlainThreads, 1)
+    k_gemm_sk_plain(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const SkArgs a) {
+    sk_body<false, BN>(&tmX, &tmW, &tmW, a);
+}
+
+// ============================================================== host side
+
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ring depths per token tile (compressed depth for the fused flavour is the
+// largest that fits, at most 6, unless the plan asks for fewer)
+struct Depths {
+    int dc, dw, dx;
+};
+Depths depths(bool fused, int bn, int stages) {
+    const int kx = bn * kBK * 2;
+    Depths d{};
+    if (fused) {
+        d.dw = bn <= 128 ? 3 : 2;
+        d.dx = bn <= 64 ? 4 : (bn == 128 ? 3 : 2);
+        int room = kMaxSmem - 1024 - d.dw * kTileW - d.dx * kx - sk_tail(8, d.dw, d.dx);
+        d.dc = std::min(6, room / kCStage);
+        if (stages > 0) d.dc = std::min(d.dc, stages);
+    } else {
+        d.dc = 0;
+        d.dx = bn <= 64 ? 6 : (bn == 128 ? 4 : 3);
+        int room = kMaxSmem - 1024 - d.dx * kx - sk_tail(0, 8, d.dx);
+        d.dw = std::min(8, room / kTileW);
+        if (stages > 0) d.dw = std::min(d.dw, std::max(2, stages));
+    }
+    return d;
+}
+
+size_t smem_bytes(bool fused, int bn, const Depths &d) {
+    return size_t(d.dw) * kTileW + size_t(d.dx) * bn * kBK * 2 + (fused ? size_t(d.dc) * kCStage : 0) + 1024 +
+           sk_tail(fused ? d.dc : 0, d.dw, d.dx);
+}
+
+int device_sms() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+            cudaGetLastError();
+            return 148;
+        }
+        cache[dev] = sms;
+    }
+    return cache[dev];
+}
+
+template <class K>
+cudaError_t prepare(K kern, int threads, size_t smem, uint32_t tmem_cols, int (&ready)[64]) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!ready[dev]) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        if (err != cudaSuccess) return err;
+        ready[dev] = 1;
+    }
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (err != cudaSuccess) return err;
+    // a second CTA on the SM would block in tcgen05.alloc until the first ends
+    if (per_sm < 1 || per_sm * int(tmem_cols) > 512) return cudaErrorInvalidConfiguration;
+    return cudaSuccess;
+}
+
+template <int BN>
+cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
+    using C = SkCfg<BN>;
+    const bool fused = p.w_bf16 == nullptr;
+    const SkGeometry g = sk_geometry(p.m, p.n, p.k, BN);
+    if (g.G <= 0) return cudaErrorInvalidValue;
+    if (!p.sk_counters || !p.partial) return cudaErrorInvalidValue;
+    const Depths d = depths(fused, BN, p.stages);
+    if ((fused && d.dc < 2) || d.dw < 2 || d.dx < 2) return cudaErrorInvalidValue;
+    size_t smem = smem_bytes(fused, BN, d);
+    smem = std::max(smem, size_t(kMaxSmem / 2 + 1024));   // one CTA per SM
+    if (smem > size_t(kMaxSmem)) return cudaErrorInvalidValue;
+
+    SkArgs a{};
+    a.m = p.m;
+    a.n = p.n;
+    a.k = p.k;
+    a.units = g.units;
+    a.S = g.S;
+    a.TB = g.TB;
+    a.G = g.G;
+    a.dc = d.dc;
+    a.dw = d.dw;
+    a.dx = d.dx;
+    a.debug_flags = p.debug_flags;
+    a.timeout_ns = p.timeout_ns;
+    a.y = p.y;
+    a.counters = p.sk_counters;
+    a.partial = p.partial;
+    a.status = p.dev_status;
+
+    CUtensorMap mx, ma, mb;
+    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2, kBK,
+                  BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    cudaError_t err;
+    if (fused) {
+        a.flagbits = p.w->flagbits;
+        a.rawbase = p.w->rawbase;
+        a.rawexp = p.w->rawexp;
+        a.nflag = (p.n * (p.k / kGroup) + 31) / 32;
+        a.pal = make_palette16(p.w->palette);
+        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k), kBK,
+                      kBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+            !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n), uint64_t(p.k / 2),
+                      kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
+            return cudaErrorInvalidValue;
+        static int ready[64] = {0};
+        err = prepare(k_gemm_sk_fused<BN>, kFusedThreads, smem, C::kTmemCols, ready);
+        if (err != cudaSuccess) return err;
+        k_gemm_sk_fused<BN><<<unsigned(g.G), kFusedThreads, smem, stream>>>(mx, ma, mb, a);
+    } else {
+        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.w_bf16, uint64_t(p.k), uint64_t(p.n),
+                      uint64_t(p.k) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        static int ready[64] = {0};
+        err = prepare(k_gemm_sk_plain<BN>, kPlainThreads, smem, C::kTmemCols, ready);
+        if (err != cudaSuccess) return err;
+        k_gemm_sk_plain<BN><<<unsigned(g.G), kPlainThreads, smem, stream>>>(mx, ma, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+SkGeometry sk_geometry(int64_t m, int64_t n, int64_t k, int bn) {
+    SkGeometry g{};
+    if (m <= 0 || n <= 0 || k <= 0 || bn <= 0) return g;
+    g.S = int(k / kBK);
+    g.TB = int((m + bn - 1) / bn);
+    g.RB = (n + kBM - 1) / kBM;
+    g.tiles = g.RB * g.TB;
+    g.units = g.tiles * g.S;
+    g.G = int(std::min<int64_t>(device_sms(), g.units));
+    g.counter_bytes = align_up(uint64_t(g.tiles) * 4, 256);
+    g.partial_bytes = align_up(uint64_t(2 * g.G) * uint64_t(bn) * kBM * 4, 256);
+    return g;
+}
+
+cudaError_t launch_gemm_sk(const TcLaunch &p, cudaStream_t stream) {
+    switch (p.bn) {
+        case 16: return launch_bn<16>(p, stream);
+        case 32: return launch_bn<32>(p, stream);
+        case 64: return launch_bn<64>(p, stream);
+        case 128: return launch_bn<128>(p, stream);
+        case 256: return launch_bn<256>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace uw

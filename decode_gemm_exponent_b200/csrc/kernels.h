@@ -103,13 +103,42 @@ struct TcLaunch {
     const uw_dmat *w;          // fused path: sm/raw/flag planes
     const uint8_t *pal;        // fused path: palette plane
     float *y;                  // [m, n]
-    float *partial;            // [split_k, m, n] when split_k > 1
+    float *partial;            // [split_k, m, n] when split_k > 1; stream-K: partial tiles
+    uint32_t *sk_counters;     // stream-K: one counter per tile (zero between calls)
     int bn, split_k, stages;
     uint32_t debug_flags;
     uint64_t timeout_ns;
     uint32_t *dev_status;
 };
 cudaError_t launch_gemm_tc(const TcLaunch &p, cudaStream_t stream);
+
+// Persistent stream-K tcgen05 GEMM (same TcLaunch; split_k unused): one CTA
+// per SM, each a contiguous run of (tile, K-step) units; tiles cut between
+// CTAs are summed in CTA order by the last CTA to finish a piece.
+// Workspace: `counters` (one u32 per tile, zero before the first call and
+// left zero by every call that completes) and `partial` (two 128 x bn fp32
+// tiles per CTA).
+struct SkGeometry {
+    int S = 0, TB = 0, G = 0;
+    int64_t RB = 0, tiles = 0, units = 0;
+    uint64_t counter_bytes = 0, partial_bytes = 0;
+};
+SkGeometry sk_geometry(int64_t m, int64_t n, int64_t k, int bn);
+cudaError_t launch_gemm_sk(const TcLaunch &p, cudaStream_t stream);
+
+// uw_fused_matmul / uw_matmul_bf16 with the stream-K tile counters kept
+// apart from the workspace (sk_counters != nullptr: at least
+// sk_counter_bytes, zero at the call; the workspace then holds only the
+// preprocessing output and the partial tiles).  For callers that share one
+// scratch region between plans of different kernels (layer stacks, the
+// autotuner, the no-workspace entry point), where another kernel's partial
+// sums would otherwise land on the counters.
+uint64_t sk_counter_bytes(int64_t m, int64_t n, int64_t k, const uw_plan *plan);
+uw_status fused_matmul_ex(const uint16_t *x_dev, int64_t m, const uw_dmat *w, const uint8_t *pal_dev, float *y_dev,
+                          const uw_plan *plan, void *ws, size_t ws_bytes, uint32_t *sk_counters, cudaStream_t s);
+uw_status matmul_bf16_ex(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev, int64_t n, int64_t k, float *y_dev,
+                         const uw_plan *plan, void *ws, size_t ws_bytes, uint32_t *dev_status, uint32_t *sk_counters,
+                         cudaStream_t s);
 
 // Fixed-order sum of split-K partials: y[i] = sum_s partial[s][i], s ascending.
 cudaError_t launch_splitk_reduce(const float *partial, int split_k, int64_t count, float *y,

@@ -21,9 +21,15 @@ namespace uw {
 namespace {
 
 constexpr size_t kScratchBytes = size_t(16) << 20;   // UW_NOALLOC_SCRATCH_BYTES
+constexpr size_t kCounterBytes = size_t(64) << 10;   // UW_NOALLOC_COUNTER_BYTES
 static_assert(kScratchBytes == UW_NOALLOC_SCRATCH_BYTES, "header and library disagree");
+static_assert(kCounterBytes == UW_NOALLOC_COUNTER_BYTES, "header and library disagree");
 
-// split-K partial sums of uw_fused_matmul_noalloc, shared by every call on a device
+// Scratch of uw_fused_matmul_noalloc, shared by every call on a device: the
+// first kCounterBytes hold the stream-K kernel's tile counters (zero at
+// load, and every completed call leaves them zero), the rest the split-K
+// partial sums or stream-K partial tiles.  Keeping the counters apart means
+// a split-K call's partial sums never land on them.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -34,7 +40,7 @@ std::mutex g_setup_mutex;
 uw_status scratch_address(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return UW_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return UW_ERR_UNSUPPORTED_SHAPE;
+    if (dev < 0 || dev >= kMaxDevices) return UW_ERR_INVALID_ARG;
     void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
     if (!p) {
         std::lock_guard<std::mutex> lock(g_setup_mutex);
@@ -60,9 +66,12 @@ extern "C" uw_status uw_fused_matmul_noalloc(const uint16_t *x_dev, int64_t m, c
     size_t need = 0;
     uw_status st = uw_workspace_size(m, w->n, w->k, plan, &need);
     if (st != UW_OK) return st;
-    if (need > kScratchBytes) return UW_ERR_WORKSPACE;
+    const uint64_t counters = sk_counter_bytes(m, w->n, w->k, plan);
+    if (counters > kCounterBytes || need - counters > kScratchBytes - kCounterBytes) return UW_ERR_WORKSPACE;
     void *scratch = nullptr;
     st = scratch_address(&scratch);
     if (st != UW_OK) return st;
-    return uw_fused_matmul(x_dev, m, w, nullptr, y_dev, plan, scratch, kScratchBytes, stream);
+    uint8_t *base = static_cast<uint8_t *>(scratch);
+    return fused_matmul_ex(x_dev, m, w, nullptr, y_dev, plan, base + kCounterBytes, kScratchBytes - kCounterBytes,
+                           reinterpret_cast<uint32_t *>(base), static_cast<cudaStream_t>(stream));
 }

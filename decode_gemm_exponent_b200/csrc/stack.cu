@@ -36,8 +36,9 @@ inline bool needs_prep(const uw_plan &p) {
 
 struct StackLayout {
     uint64_t slot_bytes = 0;      // one preprocessing slot (2 slots)
-    uint64_t partial_bytes = 0;   // split-K partial sums, reused by every step
-    uint64_t total() const { return 2 * slot_bytes + partial_bytes; }
+    uint64_t partial_bytes = 0;   // split-K partial sums / stream-K partial tiles, reused by every step
+    uint64_t counter_bytes = 0;   // stream-K tile counters, apart from the partial sums
+    uint64_t total() const { return 2 * slot_bytes + partial_bytes + counter_bytes; }
 };
 
 uw_status layout(const uw_stack_step *steps, int n_steps, StackLayout &L) {
@@ -50,8 +51,10 @@ uw_status layout(const uw_stack_step *steps, int n_steps, StackLayout &L) {
         uw_status st = uw_workspace_size(s.m, s.w->n, s.w->k, &s.plan, &all);
         if (st != UW_OK) return st;
         const uint64_t prep = prep_workspace_bytes(s.w->n, s.w->k, s.plan.pipeline);
+        const uint64_t counters = sk_counter_bytes(s.m, s.w->n, s.w->k, &s.plan);
         L.slot_bytes = std::max(L.slot_bytes, prep);
-        L.partial_bytes = std::max(L.partial_bytes, uint64_t(all) - prep);
+        L.partial_bytes = std::max(L.partial_bytes, uint64_t(all) - prep - counters);
+        L.counter_bytes = std::max(L.counter_bytes, counters);
     }
     return UW_OK;
 }
@@ -111,6 +114,9 @@ extern "C" uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void 
     const bool overlap = side_stream != nullptr && side_s != main_s;
     uint8_t *slot[2] = {static_cast<uint8_t *>(ws), static_cast<uint8_t *>(ws) + L.slot_bytes};
     void *partial = L.partial_bytes ? static_cast<uint8_t *>(ws) + 2 * L.slot_bytes : nullptr;
+    uint32_t *counters =
+        L.counter_bytes ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + 2 * L.slot_bytes + L.partial_bytes)
+                        : nullptr;
 
     // ev[0..1]: slot s holds its step's prepared weights; ev[2..3]: slot s is
     // free again; ev[4]: fork / join marker
@@ -125,7 +131,8 @@ extern "C" uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void 
         const uw_stack_step &s = steps[i];
         const uw_dmat *w = s.w;
         if (!needs_prep(s.plan)) {
-            st = uw_fused_matmul(s.x_dev, s.m, w, s.pal_dev, s.y_dev, &s.plan, partial, L.partial_bytes, main_s);
+            st = fused_matmul_ex(s.x_dev, s.m, w, s.pal_dev, s.y_dev, &s.plan, partial, L.partial_bytes, counters,
+                                 main_s);
             continue;
         }
         const int b = n_prep & 1;
@@ -152,15 +159,15 @@ extern "C" uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void 
             break;
         }
         if (s.plan.pipeline == UW_PIPE_DECODE_GEMM) {
-            st = uw_matmul_bf16(s.x_dev, s.m, reinterpret_cast<const uint16_t *>(slot[b]), w->n, w->k, s.y_dev,
-                                &s.plan, partial, L.partial_bytes, w->dev_status, main_s);
+            st = matmul_bf16_ex(s.x_dev, s.m, reinterpret_cast<const uint16_t *>(slot[b]), w->n, w->k, s.y_dev,
+                                &s.plan, partial, L.partial_bytes, w->dev_status, counters, main_s);
         } else {
             // pipeline 3: the fused kernel on the transcoded plane; pipeline 2:
             // on the all-raw view whose raw plane is the decoded exponents
             uw_plan p = s.plan;
             p.pipeline = UW_PIPE_DIRECT_PALETTE;
             const uw_dmat v = s.plan.pipeline == UW_PIPE_DECODE_EXP_FUSED ? exp_plane_view(*w, slot[b]) : *w;
-            st = uw_fused_matmul(s.x_dev, s.m, &v, slot[b], s.y_dev, &p, partial, L.partial_bytes, main_s);
+            st = fused_matmul_ex(s.x_dev, s.m, &v, slot[b], s.y_dev, &p, partial, L.partial_bytes, counters, main_s);
         }
         if (st == UW_OK && overlap && cudaEventRecord(E.ev[2 + b], main_s) != cudaSuccess) st = UW_ERR_CUDA;
         n_prep++;

@@ -31,7 +31,7 @@ EMIT_PALETTE = 2
 SEC_SM, SEC_RAWEXP, SEC_FLAGS, SEC_RAWBASE, SEC_STREAM, SEC_CHUNKOFF, SEC_DLUT, SEC_PAL = range(8)
 NUM_SECTIONS = 8
 PIPE_DECODE_GEMM, PIPE_DECODE_EXP_FUSED, PIPE_TRANSCODE_FUSED, PIPE_DIRECT_PALETTE = 1, 2, 3, 4
-KERNEL_FMA, KERNEL_TC, KERNEL_MMA = 1, 2, 3
+KERNEL_FMA, KERNEL_TC, KERNEL_MMA, KERNEL_TC_SK = 1, 2, 3, 4
 DEBUG_NEVER_ARRIVE = 1
 
 # every symbol include/uw.h declares
@@ -270,8 +270,7 @@ class Matrix:
         if y is None:
             y = torch.empty(m, self.n, dtype=torch.float32, device=x.device)
         if ws is None:
-            nb = self.workspace_bytes(m, plan)
-            ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=x.device) if nb else None
+            ws = new_workspace(self.workspace_bytes(m, plan), x.device)
         check(lib().uw_fused_matmul(_ptr(x), m, ctypes.byref(self.dmat), _ptr(pal), _ptr(y),
                                     ctypes.byref(plan), _ptr(ws), ws.numel() if ws is not None else 0,
                                     _stream_handle(stream)), "uw_fused_matmul")
@@ -329,7 +328,7 @@ class Stack:
         check(lib().uw_stack_workspace_size(arr, len(steps), ctypes.byref(size)), "uw_stack_workspace_size")
         self.ws_bytes = int(size.value)
         dev = steps[0][1].device
-        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
+        self.ws = new_workspace(max(self.ws_bytes, 256), dev)
 
     def run(self, stream=None, side_stream=None):
         """Issue the whole stack; side_stream=None runs everything on `stream`."""
@@ -385,6 +384,14 @@ class SmSplit:
         self.close()
 
 
+def new_workspace(nbytes: int, device):
+    """A zero-filled device workspace of `nbytes` (None for 0).  Zero matters
+    for stream-K plans, whose tile counters must start at zero; every call
+    that completes leaves them zero, so the buffer can be reused as is."""
+    import torch
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device) if nbytes else None
+
+
 def workspace_size(m: int, n: int, k: int, plan: Plan) -> int:
     size = ctypes.c_size_t()
     check(lib().uw_workspace_size(m, n, k, ctypes.byref(plan), ctypes.byref(size)), "uw_workspace_size")
@@ -405,8 +412,7 @@ def matmul_bf16(x, w, plan: Plan, y=None, ws=None, status=None, stream=None):
     if y is None:
         y = torch.empty(m, n, dtype=torch.float32, device=x.device)
     if ws is None:
-        nb = workspace_size(m, n, k, plan)
-        ws = torch.empty(nb, dtype=torch.uint8, device=x.device) if nb else None
+        ws = new_workspace(workspace_size(m, n, k, plan), x.device)
     check(lib().uw_matmul_bf16(_ptr(x), m, _ptr(w), n, k, _ptr(y), ctypes.byref(plan), _ptr(ws),
                                ws.numel() if ws is not None else 0, _ptr(status), _stream_handle(stream)),
           "uw_matmul_bf16")
@@ -439,7 +445,7 @@ def autotune(mats: Sequence[Matrix], ms: Sequence[int], reps: int = 5, stream=No
 
 PIPELINE_NAMES = {PIPE_DECODE_GEMM: "decode_gemm", PIPE_DECODE_EXP_FUSED: "decode_exp_fused",
                   PIPE_TRANSCODE_FUSED: "transcode_fused", PIPE_DIRECT_PALETTE: "direct_palette"}
-KERNEL_NAMES = {KERNEL_FMA: "fma", KERNEL_TC: "tc", KERNEL_MMA: "mma"}
+KERNEL_NAMES = {KERNEL_FMA: "fma", KERNEL_TC: "tc", KERNEL_MMA: "mma", KERNEL_TC_SK: "tc_sk"}
 
 
 def plans_from_json(text: str, ms: Sequence[int]):

@@ -202,9 +202,16 @@ typedef enum uw_pipeline {
 typedef enum uw_kernel {
     UW_KERNEL_FMA = 1,   /* CUDA-core FMA GEMV, one warp per `bn` rows, m <= 8       */
     UW_KERNEL_TC = 2,    /* tcgen05 MMA with a TMEM accumulator, token tile `bn`      */
-    UW_KERNEL_MMA = 3    /* m <= 16: W rebuilt in registers straight into warp-level
+    UW_KERNEL_MMA = 3,   /* m <= 16: W rebuilt in registers straight into warp-level
                             MMA fragments; one CTA per 16-row tile, whose `bn`
                             warps split K (summed in a fixed order)               */
+    UW_KERNEL_TC_SK = 4  /* any m: persistent stream-K tcgen05 kernel, token tile
+                            `bn`, one CTA per SM, each owning an equal contiguous
+                            run of (128-row x bn tile, 64-wide K-step) units; a
+                            tile cut between CTAs is summed in CTA (= K) order by
+                            the CTA that finishes its last piece.  Needs a
+                            workspace whose tile counters are zero (see
+                            uw_workspace_size); split_k must be 1             */
 } uw_kernel;
 
 #define UW_DEBUG_NEVER_ARRIVE 1u   /* TC kernel: wait on a barrier nobody signals, so
@@ -217,9 +224,12 @@ typedef struct uw_plan {
                              FMA: weight rows per warp, 1 or 2;
                              MMA: warps per CTA = K slices per 16-row tile, 1..8 */
     int32_t split_k;      /* TC: K split into this many slices (>= 1), reduced in a
-                             fixed order; FMA, MMA: must be 1 */
+                             fixed order; FMA, MMA, TC_SK: must be 1 */
     int32_t stages;       /* TC: shared-memory ring depth (0 = default: 4 for the plain
                              kernel, the largest that fits for the fused one);
+                             TC_SK: compressed-tile ring depth of the fused kernel
+                             (W-tile ring of the plain one), 0 = the largest that
+                             fits (at most 6 / 8);
                              MMA: weights per lane and row per step, 1 = 16, 2 = 32
                              (K a multiple of 128), 0 = 32 when K allows, else 16 */
     uint32_t debug_flags; /* UW_DEBUG_* (0 in production) */
@@ -234,7 +244,14 @@ uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pipeline, uw_
  * preprocessing output (pipeline 1: 2nk bytes of BF16; pipeline 2: the nk-byte
  * exponent plane plus two nk/2048-word index arrays; pipeline 3: nk/2 bytes;
  * pipeline 4: none), each part rounded up to 256 bytes, plus split_k*m*n
- * floats of partial sums for a TC plan with split_k > 1.                     */
+ * floats of partial sums for a TC plan with split_k > 1, or for a TC_SK plan
+ * one uint32 counter per 128 x bn tile (256-byte rounded) followed by two
+ * 128 x bn float tiles per CTA (one CTA per SM of the current device).
+ * TC_SK: the counters must be zero when a call starts.  Zero the whole
+ * workspace once after allocating it; every call that completes leaves the
+ * counters zero again, so the same workspace serves any later TC_SK call
+ * (any shape) without clearing.  After a call whose uw_device_status reports
+ * an error, zero the workspace again before reusing it.                     */
 uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw_plan *plan,
                             size_t *bytes);
 
@@ -281,8 +298,11 @@ uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const
 /* ------------------------------------------------------------------------ */
 /* Matmul without a caller workspace (no counterpart on the Unweight page).   */
 
-/* Bytes of the library-owned scratch array used by uw_fused_matmul_noalloc. */
+/* Bytes of the library-owned scratch array used by uw_fused_matmul_noalloc,
+ * and how many of them (at its start) hold TC_SK tile counters, one uint32
+ * per 128 x bn tile.                                                        */
 #define UW_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define UW_NOALLOC_COUNTER_BYTES (64u << 10)
 
 /* uw_fused_matmul for callers that cannot give the library device memory
  * (an engine that hands its plug-ins no allocator and forbids cudaMalloc
@@ -293,14 +313,22 @@ uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const
  * every GPU that loads the library holds until the process exits.  Nothing is
  * allocated per call (no cudaMalloc, no allocating library routine).
  *   - plan->pipeline must be UW_PIPE_DIRECT_PALETTE (INVALID_ARG otherwise);
- *     a plan whose uw_workspace_size exceeds UW_NOALLOC_SCRATCH_BYTES is
- *     rejected with UW_ERR_WORKSPACE before anything is launched.
+ *     a plan whose scratch (uw_workspace_size) does not fit is rejected with
+ *     UW_ERR_WORKSPACE before anything is launched: partial sums beyond
+ *     UW_NOALLOC_SCRATCH_BYTES - UW_NOALLOC_COUNTER_BYTES, or (TC_SK) more
+ *     tile counters than UW_NOALLOC_COUNTER_BYTES hold.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: do not call this
+ *     entry point on a device after cudaDeviceReset.  Devices with an
+ *     ordinal of 64 or more are refused (UW_ERR_INVALID_ARG).
  *   - All calls on a device share the one array: calls that may overlap on
  *     the GPU (other streams, other threads) race and must be serialised by
- *     the caller.  No state carries over between calls; every partial sum a
- *     call reads was written by that same call.                             */
+ *     the caller.  Partial sums do not carry over: in a call whose kernels
+ *     complete, every partial sum read was written by that same call.  A
+ *     call whose uw_device_status then reports an error may have left stale
+ *     values in y, and (TC_SK) non-zero tile counters, after which the
+ *     entry point should not be used again in the process.                 */
 uw_status uw_fused_matmul_noalloc(const uint16_t *x_dev, int64_t m, const uw_dmat *w,
                                   float *y_dev, const uw_plan *plan, void *stream);
 
@@ -341,7 +369,10 @@ typedef struct uw_stack_step {
 
 /* Workspace of uw_stack_run: two preprocessing slots, each the largest
  * preprocessing buffer of the stack (decode 2nk bytes, exponent decode a bit
- * over nk, transcode nk/2), plus the largest split-K scratch of any step.    */
+ * over nk, transcode nk/2), plus the largest split-K scratch of any step,
+ * plus (for TC_SK steps) a region of stream-K tile counters kept apart from
+ * the partial sums.  Zero the workspace once after allocating it (the
+ * counters must start at zero; completed runs leave them zero).             */
 uw_status uw_stack_workspace_size(const uw_stack_step *steps, int n_steps, size_t *bytes);
 
 /* Run the steps in order on `stream`.  The decode (pipelines 1 and 2) or

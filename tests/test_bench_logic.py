@@ -20,9 +20,15 @@ def test_measured_traffic_lookup():
         assert got is None or abs(got - 2 * rec["bytes"]) < 1e-6 * rec["bytes"]
     saved = dict(bench.MEASURED_TRAFFIC)
     try:
-        name, rec = next(iter(saved.items()))
-        bench.MEASURED_TRAFFIC[name] = dict(rec, sha256="0" * 64)   # pretend the kernel changed
-        assert bench.measured_traffic(name, rec["alg_bytes"]) is None
+        # a record keyed on the current source of a committed kernel file
+        f = "decode_gemm_exponent_b200/csrc/gemm_sk.cu"
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            digest = bench.source_digest([fh.read()])
+        rec = {"bytes": 1000, "alg_bytes": 800, "files": (f,), "sha256": digest}
+        bench.MEASURED_TRAFFIC["fused/test_kernel"] = rec
+        assert abs(bench.measured_traffic("fused/test_kernel", 1600) - 2000) < 1e-9
+        bench.MEASURED_TRAFFIC["fused/test_kernel"] = dict(rec, sha256="0" * 64)   # pretend the kernel changed
+        assert bench.measured_traffic("fused/test_kernel", 800) is None
     finally:
         bench.MEASURED_TRAFFIC.clear()
         bench.MEASURED_TRAFFIC.update(saved)
@@ -91,20 +97,20 @@ def test_compression_stats_on_real_blobs():
 def test_plans_from_json_round_trip():
     from decode_gemm_exponent_b200 import uw
     doc = {"plans": []}
-    kinds = [("fma", 1, 1, 0), ("tc", 64, 4, 0), ("mma", 4, 1, 2)]
+    kinds = [("fma", 1, 1, 0), ("tc", 64, 4, 0), ("mma", 4, 1, 2), ("tc_sk", 16, 1, 3)]
     pipes = [("decode_gemm", uw.PIPE_DECODE_GEMM), ("decode_exp_fused", uw.PIPE_DECODE_EXP_FUSED),
              ("transcode_fused", uw.PIPE_TRANSCODE_FUSED), ("direct_palette", uw.PIPE_DIRECT_PALETTE)]
     for i in range(3):
         for j, m in enumerate(bench.MS):
-            kern, bn, split, stages = kinds[(i + j) % 3]
+            kern, bn, split, stages = kinds[(i + j) % 4]
             doc["plans"].append({"matrix": i, "m": m, "best": {"pipeline": pipes[(i + 2 * j) % 4][0], "kernel": kern,
                                                                 "bn": bn, "split_k": split, "stages": stages}})
     plans = bench.plans_from_json(json.dumps(doc), 3, uw)
     for i in range(3):
         for j in range(len(bench.MS)):
-            kern, bn, split, stages = kinds[(i + j) % 3]
+            kern, bn, split, stages = kinds[(i + j) % 4]
             p = plans[i][j]
-            assert p.kernel == {"fma": 1, "tc": 2, "mma": 3}[kern] and p.bn == bn and p.split_k == split
+            assert p.kernel == {"fma": 1, "tc": 2, "mma": 3, "tc_sk": 4}[kern] and p.bn == bn and p.split_k == split
             assert p.stages == stages and p.pipeline == pipes[(i + 2 * j) % 4][1]
             # every plan has a kernel group and a launch count; pipelines 1-3 add a preprocessing launch
             assert bench.kernel_group(p).split("/")[0]
@@ -127,3 +133,24 @@ def test_plan_file_reader_rejects_incomplete_or_unknown_plans():
         uw.plans_from_json(json.dumps(bad), [1])
     with pytest.raises(ValueError):                       # the bench's layer has three matrices
         bench.plans_from_json(json.dumps(doc), 3, uw)
+
+
+def test_oracle_sample_is_the_step_on_a_row_sample():
+    """The reference arm and the CPU baseline run the step's 12 calls on the
+    first 1/16 of each matrix's rows; both arms print the same config."""
+    tasks = bench.oracle_tasks()
+    assert sorted(tasks) == sorted((i, m) for m in bench.MS for i in range(len(bench.PROJ)))
+    rows = [bench.oracle_sample_rows(n) for _, n, _ in bench.PROJ]
+    assert rows == [896, 896, 256]
+    assert bench.oracle_step_bytes() == sum(2 * r * k for r, (_, _, k) in zip(rows, bench.PROJ)) * len(bench.MS)
+    assert bench.workload_config() == {"workload": bench.WORKLOAD, "l2": bench.L2_NOTE}
+    assert "12 calls" in bench.oracle_sample_text(4) and "4 worker processes" in bench.oracle_sample_text(4)
+
+
+def test_kernel_names_of_every_plan_kind():
+    from decode_gemm_exponent_b200 import uw
+    assert bench.kernel_group(uw.make_plan(4, uw.KERNEL_TC_SK, 64, 1)) == "fused/tc_sk_bn64"
+    assert bench.plan_label(uw.make_plan(1, uw.KERNEL_TC, 64, 4)) == "decode+plain/tcgen05_bn64/split4"
+    assert bench.launches_per_call(uw.make_plan(4, uw.KERNEL_TC_SK, 16, 1)) == 1
+    assert bench.launches_per_call(uw.make_plan(3, uw.KERNEL_TC_SK, 16, 1)) == 2
+    assert bench.launches_per_call(uw.make_plan(4, uw.KERNEL_TC, 16, 4)) == 2
