@@ -365,6 +365,9 @@ def alg_bytes(mat, m, plan):
     fused_in = sm + raw + flags + nk // 2                   # palette form
     if plan.pipeline == 4:
         return {"fused": fused_in + xy}
+    if plan.pipeline == 5:
+        # the Huffman form (stream, chunk offsets, bitmap, raw plane, sign/mantissa) read by one kernel
+        return {"fused": stream + flags + raw + sm + xy}
     if plan.pipeline == 1:
         return {"decode": stream + flags + raw + sm + 2 * nk, "plain": 2 * nk + xy}
     if plan.pipeline == 2:
@@ -394,7 +397,8 @@ def kernel_name(plan):
 
 
 def kernel_group(plan):
-    pipe = {1: "decode+plain", 2: "exp_decode+fused", 3: "transcode+fused", 4: "fused"}[plan.pipeline]
+    pipe = {1: "decode+plain", 2: "exp_decode+fused", 3: "transcode+fused", 4: "fused",
+            5: "huffman_fused"}[plan.pipeline]
     return "%s/%s" % (pipe, kernel_name(plan))
 
 

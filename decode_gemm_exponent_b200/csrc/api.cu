@@ -24,7 +24,10 @@ bool valid_bn_tc(int bn) { return bn == 16 || bn == 32 || bn == 64 || bn == 128 
 uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
     if (!p || k <= 0) return UW_ERR_INVALID_ARG;
     if (p->pipeline != UW_PIPE_DECODE_GEMM && p->pipeline != UW_PIPE_DECODE_EXP_FUSED &&
-        p->pipeline != UW_PIPE_TRANSCODE_FUSED && p->pipeline != UW_PIPE_DIRECT_PALETTE)
+        p->pipeline != UW_PIPE_TRANSCODE_FUSED && p->pipeline != UW_PIPE_DIRECT_PALETTE &&
+        p->pipeline != UW_PIPE_HUFFMAN_FUSED)
+        return UW_ERR_INVALID_ARG;
+    if (p->pipeline == UW_PIPE_HUFFMAN_FUSED && (p->kernel != UW_KERNEL_TC_SK || p->bn > 128 || k % 256))
         return UW_ERR_INVALID_ARG;
     if (p->kernel == UW_KERNEL_FMA) {
         if (m > 8 || (p->bn != 1 && p->bn != 2) || p->split_k != 1) return UW_ERR_INVALID_ARG;
@@ -60,7 +63,8 @@ uint64_t prep_bytes(int64_t n, int64_t k, const uw_plan *p) { return prep_worksp
 // Run one matmul kernel on prepared weights: w_bf16 (plain) or pal (fused).
 uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const uw_dmat *w,
                      const uint8_t *pal, int64_t n, int64_t k, float *y, const uw_plan *plan,
-                     float *partial, uint32_t *status, uint32_t *sk_counters, cudaStream_t stream) {
+                     float *partial, uint32_t *status, uint32_t *sk_counters, cudaStream_t stream,
+                     bool huffman = false) {
     if (plan->kernel == UW_KERNEL_FMA)
         return cuda_status(launch_gemv_fma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, status, stream));
     if (plan->kernel == UW_KERNEL_MMA)
@@ -81,6 +85,7 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
     t.debug_flags = plan->debug_flags;
     t.timeout_ns = plan->timeout_ns > 0 ? uint64_t(plan->timeout_ns) : kDefaultTimeoutNs;
     t.dev_status = status;
+    t.huffman = huffman;
     if (plan->kernel == UW_KERNEL_TC_SK) {
         uint8_t *base = reinterpret_cast<uint8_t *>(partial);
         if (!base) return UW_ERR_WORKSPACE;
@@ -268,6 +273,11 @@ uw_status fused_matmul_ex(const uint16_t *x_dev, int64_t m, const uw_dmat *w, co
         const uw_dmat v = exp_plane_view(*w, wsb);
         return run_kernel(x_dev, m, nullptr, &v, v.pal, w->n, w->k, y_dev, plan, partial, w->dev_status,
                           sk_counters, s);
+    }
+    if (plan->pipeline == UW_PIPE_HUFFMAN_FUSED) {
+        if (!(w->flags & UW_EMIT_HUFFMAN) || !w->stream || !w->chunk_off || !w->dlut) return UW_ERR_INVALID_ARG;
+        return run_kernel(x_dev, m, nullptr, w, nullptr, w->n, w->k, y_dev, plan, partial, w->dev_status,
+                          sk_counters, s, true);
     }
     const uint8_t *pal = nullptr;
     if (plan->pipeline == UW_PIPE_TRANSCODE_FUSED) {

@@ -82,6 +82,12 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
             p.bn = bn;
             p.split_k = 1;
             out.push_back(p);
+            // the same kernel decoding the Huffman stream itself (pipeline 3's
+            // transcode moved into the matmul)
+            if (pipe == UW_PIPE_TRANSCODE_FUSED && bn <= 128 && w.k % 256 == 0) {
+                p.pipeline = UW_PIPE_HUFFMAN_FUSED;
+                out.push_back(p);
+            }
         }
         for (int bn : {bn_hi / 2, bn_hi}) {
             if (bn < 16) continue;
@@ -107,6 +113,7 @@ const char *pipe_name(int p) {
         case UW_PIPE_DECODE_GEMM: return "decode_gemm";
         case UW_PIPE_DECODE_EXP_FUSED: return "decode_exp_fused";
         case UW_PIPE_TRANSCODE_FUSED: return "transcode_fused";
+        case UW_PIPE_HUFFMAN_FUSED: return "huffman_fused";
         default: return "direct_palette";
     }
 }

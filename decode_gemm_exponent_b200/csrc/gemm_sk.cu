@@ -1,8 +1,16 @@
 // gemm_sk.cu -- persistent stream-K tensor-core matmul Y = X * W^T on sm_100a
-// (tcgen05 MMA, TMEM accumulators), in a fused flavour that rebuilds W from
-// its compressed planes in shared memory (Unweight page §七, reconstructive
-// matmul; §五, decompressed weights never go back to HBM) and a plain flavour
-// that loads BF16 W (the uncompressed baseline and the bit-exactness twin).
+// (tcgen05 MMA, TMEM accumulators), in three flavours that issue the same MMA
+// sequence on the same schedule, so their outputs are bit-identical:
+//   * plain:   W loaded as BF16 (the uncompressed baseline and the twin);
+//   * palette: W rebuilt in shared memory from its sign/mantissa plane, its
+//              4-bit palette plane and its raw groups (Unweight page §七, the
+//              reconstructive matmul; §五, decompressed weights never go back
+//              to HBM);
+//   * Huffman: the same rebuild, but the 4-bit palette indices are decoded
+//              from the Huffman exponent stream inside the kernel (page §六,
+//              pipeline 3's transcode moved into the matmul's producer: the
+//              bytes read are the Huffman form and X, the only bytes written
+//              are Y).
 //
 // Work decomposition.  A tile is 128 rows of W (the MMA's M) by BN tokens
 // (the MMA's N); a unit is one 64-wide K-step of one tile.  Tiles are ordered
@@ -15,26 +23,36 @@
 // writes its fp32 partial tile to the workspace and bumps the tile's counter;
 // the CTA that brings the counter to the number of pieces adds all pieces in
 // CTA order (= K order) and writes Y, then zeroes the counter.  No CTA waits
-// for another, and the sum order is fixed by the schedule alone, so the plain
-// and fused flavours (same schedule, same MMA sequence) give identical bits.
+// for another, and the sum order is fixed by the schedule alone.
 //
 // Roles (warps):
-//   0      producer: fused -- per K-step the sign/mantissa tile (TMA, 64-byte
-//          swizzle) and the 4-bit palette tile (TMA, 32-byte swizzle), and
+//   0      producer: per K-step the sign/mantissa tile (TMA, 64-byte swizzle),
+//          the 4-bit palette tile (TMA, 32-byte swizzle; palette flavour), and
 //          for each raw (row, group) its 64 exponents by a 64-byte bulk copy,
 //          all counted on one barrier; the 32 lanes share the 128 rows' raw
 //          bits and write the step's 128-bit raw mask next to the stage.
-//          plain -- the BF16 W tile (TMA, 128-byte swizzle) into the W ring.
+//          Plain flavour: the BF16 W tile (TMA, 128-byte swizzle).
 //   1      MMA issuer and TMEM owner: 4 x tcgen05.mma (K = 16) per K-step into
 //          one of two accumulators (double-buffered, so the epilogue of one
 //          tile overlaps the MMAs of the next).
 //   2      X producer (TMA, 128-byte swizzle).
 //   3-6    epilogue: TMEM -> registers -> Y (or a partial tile + fix-up).
-//   7-14   (fused) rebuild: all 8 warps work on the same K-step; thread t
-//          rebuilds 32 weights (half h = t & 1) of tile row r = t >> 1 into
-//          the 128-byte-swizzled K-major BF16 W tile.  The thread-to-data map
-//          keeps every 16-byte shared-memory access of a quarter warp on
+//   7-14   rebuild (palette, Huffman): all 8 warps work on the same K-step;
+//          thread t rebuilds 32 weights (half h = t & 1) of tile row r = t >> 1
+//          into the 128-byte-swizzled K-major BF16 W tile.  The thread-to-data
+//          map keeps every 16-byte shared-memory access of a quarter warp on
 //          distinct bank groups (sign/mantissa, palette words and W stores).
+//   15     (Huffman) stream producer: per super-step (the K-steps of one
+//          4-group stream chunk in each of the tile's 128 rows) it reads the
+//          128 chunks' start bits, packs the chunks' stream words into one
+//          slot of a 4-slot shared-memory ring with bulk copies, and writes a
+//          table of where each chunk's words are (a chunk that does not fit
+//          the slot is read from global memory by its decoder instead).
+//   16-23  (Huffman) decoders: two groups of 4 warps take alternate
+//          super-steps, one thread per tile row.  A thread decodes its row's
+//          chunk group by group with the 12-bit multi-symbol table, each
+//          group's 64 indices into a private scratch line, then copies them
+//          into the K-step's compressed stage in the stored 4-bit layout.
 // Every wait is bounded; on time-out a role raises UW_DEVERR_TIMEOUT and sets
 // the CTA's abort flag, which ends every other wait of the CTA; TMA copies
 // and MMAs in flight are waited for (bounded) before TMEM is freed.
@@ -51,6 +69,8 @@ namespace {
 
 using namespace dev;
 
+constexpr int kModePlain = 0, kModePal = 1, kModeHuff = 2;
+
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kMaxSmem = 232448;        // 227 KB opt-in per CTA
@@ -58,8 +78,12 @@ constexpr int kFixedWarps = 7;          // producer, MMA, X producer, 4 epilogue
 constexpr int kRebuildWarps = 8;
 constexpr int kEpiWarp0 = 3;
 constexpr int kFirstRebuildWarp = kFixedWarps;
-constexpr int kFusedThreads = (kFixedWarps + kRebuildWarps) * 32;
+constexpr int kStreamWarp = kFixedWarps + kRebuildWarps;   // Huffman flavour
+constexpr int kFirstDecWarp = kStreamWarp + 1;
+constexpr int kDecWarps = 8;            // two groups of 4
 constexpr int kPlainThreads = kFixedWarps * 32;
+constexpr int kPalThreads = (kFixedWarps + kRebuildWarps) * 32;
+constexpr int kHuffThreads = (kFixedWarps + kRebuildWarps + 1 + kDecWarps) * 32;
 
 constexpr int kTileW = kBM * kBK * 2;            // BF16 W tile
 constexpr int kTileSM = kBM * kBK;               // sign/mantissa tile
@@ -67,6 +91,12 @@ constexpr int kTilePL = kBM * kBK / 2;           // 4-bit palette tile
 constexpr int kTileRAW = kBM * kGroup;           // one 64-byte exponent slot per row
 constexpr int kCStage = kTileSM + kTilePL + kTileRAW;
 constexpr int kOffPL = kTileSM, kOffRAW = kTileSM + kTilePL;
+
+// Huffman flavour
+constexpr int kSlots = 4;                        // stream slots (super-steps staged ahead)
+constexpr int kSlotBytes = 12 * 1024;            // stream bytes per slot (~85 B per chunk at 2.6 bits/weight)
+constexpr int kScratchStride = 36;               // bytes per decoder thread: 8 words + 1 of padding
+constexpr uint32_t kFromGlobal = 0x80000000u;    // table flag: the chunk's words are read from global memory
 
 struct SkArgs {
     int64_t m, n, k;
@@ -85,6 +115,12 @@ struct SkArgs {
     const uint8_t *rawexp;
     int64_t nflag;            // words of flagbits
     Palette16 pal;
+    // Huffman flavour
+    const uint32_t *stream;
+    const uint32_t *chunk_off;
+    const uint32_t *dlut;
+    uint64_t stream_bits;
+    uint64_t code_len;        // code length of palette index s in bits 4s..4s+3
     uint32_t *status;
 };
 
@@ -102,6 +138,16 @@ __device__ __forceinline__ void prefetch_l1(const void *p) {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+
 template <int BN>
 struct SkCfg {
     static constexpr int kX = BN * kBK * 2;
@@ -110,21 +156,120 @@ struct SkCfg {
     static_assert(2 * BN <= 512, "accumulators exceed TMEM");
 };
 
-// shared-memory bytes after the rings: raw masks, barriers, TMEM slot, flags
+// Huffman flavour: decode table, stream slots, their chunk tables and the
+// decoders' scratch lines, placed after the compressed ring
+constexpr int kHuffLut = kLutEntries * 4;
+constexpr int kHuffTable = kSlots * kBM * 16;    // per slot and row: uint4 {where, first word, start, end}
+constexpr int kHuffRaw4 = kSlots * kBM;          // per slot and row: the chunk's raw-group bits
+constexpr int kHuffScratch = kDecWarps * 32 * kScratchStride;
+constexpr int kHuffBytes = kHuffLut + kSlots * kSlotBytes + kHuffTable + kHuffRaw4 + kHuffScratch;
+static_assert(kHuffBytes % 16 == 0, "Huffman area keeps 16-byte alignment");
+
+// shared-memory bytes after the rings (and the Huffman area): raw masks,
+// barriers, TMEM slot, flags
 __host__ __device__ constexpr int sk_tail(int dc, int dw, int dx) {
-    return dc * 16 + (2 * dc + 2 * dw + 2 * dx + 4 + 2) * 8 + 16;
+    return dc * 16 + (2 * dc + 2 * dw + 2 * dx + 4 + 2 + 2 * kSlots + 1) * 8 + 16;
 }
 
-template <bool FUSED, int BN>
+// The CTA's super-steps: for each tile of its unit range and each 4-group
+// chunk index j touched there, the K-steps [ka, kb) of the tile that the CTA
+// owns.  Walked identically by the stream producer and the decoders.
+struct SuperSteps {
+    int64_t u0, u1, t, t_last;
+    int S, j, j_last, ka, kb;
+    __device__ __forceinline__ void start_tile() {
+        ka = t == u0 / S ? int(u0 - t * S) : 0;
+        kb = t == t_last ? int(u1 - t * S) : S;
+        j = ka >> 2;
+        j_last = (kb - 1) >> 2;
+    }
+    __device__ __forceinline__ SuperSteps(int64_t u0_, int64_t u1_, int S_) : u0(u0_), u1(u1_), S(S_) {
+        t = u0 / S;
+        t_last = (u1 - 1) / S;
+        start_tile();
+    }
+    __device__ __forceinline__ bool valid() const { return u1 > u0 && t <= t_last; }
+    __device__ __forceinline__ void next() {
+        if (++j > j_last) {
+            ++t;
+            if (t <= t_last) start_tile();
+        }
+    }
+};
+
+// Decode one group's 64 palette indices from bit p of a stream (words read
+// through `word(i)`), 8 per word into the scratch line at shared address
+// `line` (natural order: index i in bits 4(i%8).. of word i/8).  Never starts
+// a step past `end`; false if a window has no valid code or the group does
+// not complete.
+template <class Src>
+__device__ __forceinline__ bool decode_group(const Src &word, uint32_t &p, uint32_t end, uint32_t lut,
+                                             uint32_t line, uint64_t code_len) {
+    uint32_t lo = 0, na = 0, off = 0, rem4 = 256, err = 0;
+    auto push = [&](uint32_t s, uint32_t nbits) {
+        lo |= s << na;
+        const uint32_t carry = __funnelshift_l(s, 0u, na);
+        na += nbits;
+        if (na >= 32) {
+            sts32(line + off, lo);
+            off += 4u;
+            lo = carry;
+            na -= 32;
+        }
+    };
+    auto window = [&](uint32_t q) {
+        const uint32_t wi = q >> 5;
+        return __funnelshift_l(word(wi + 1), word(wi), q);
+    };
+    while (rem4 >= 40 && p <= end) {       // two whole table entries per window
+        const uint32_t top = window(p);
+        const uint32_t e1 = lds32(lut + ((top >> (32 - kLutBits)) << 2));
+        const uint32_t b1 = lut_bits(e1);
+        const uint32_t e2 = lds32(lut + (((top << b1) >> (32 - kLutBits)) << 2));
+        p += b1 + lut_bits(e2);
+        err |= e1 | e2;
+        const uint32_t n1 = lut_symbits(e1), n2 = lut_symbits(e2);
+        push(e1 & 0xFFFFFu, n1);
+        push(e2 & 0xFFFFFu, n2);
+        rem4 -= n1 + n2;
+    }
+    while (rem4 >= 20 && p <= end) {       // whole entries while at least 5 indices remain
+        const uint32_t e = lds32(lut + ((window(p) >> (32 - kLutBits)) << 2));
+        p += lut_bits(e);
+        err |= e;
+        const uint32_t n = lut_symbits(e);
+        push(e & 0xFFFFFu, n);
+        rem4 -= n;
+    }
+    while (rem4 > 0 && p <= end) {         // the last few one code at a time
+        const uint32_t e = lds32(lut + ((window(p) >> (32 - kLutBits)) << 2));
+        const uint32_t s = e & 15u;
+        p += uint32_t(code_len >> (4 * s)) & 15u;
+        err |= e;
+        push(s, 4);
+        rem4 -= 4;
+    }
+    return rem4 == 0 && !(err & kLutInvalid);
+}
+
+template <int MODE, int BN>
 __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMap *tmA, const CUtensorMap *tmB,
                                         const SkArgs &a) {
     using C = SkCfg<BN>;
+    constexpr bool FUSED = MODE != kModePlain;
+    constexpr bool HUFF = MODE == kModeHuff;
     extern __shared__ uint8_t smem_dyn[];
     const int dc = FUSED ? a.dc : 0, dw = a.dw, dx = a.dx;
     uint8_t *wring = align1024(smem_dyn);
     uint8_t *xring = wring + size_t(dw) * kTileW;
     uint8_t *cring = xring + size_t(dx) * C::kX;
-    uint32_t *masks = reinterpret_cast<uint32_t *>(cring + size_t(dc) * kCStage);   // [dc][4]
+    uint8_t *huff = cring + size_t(dc) * kCStage;                  // Huffman area
+    uint32_t *hlut = reinterpret_cast<uint32_t *>(huff);
+    uint8_t *hslots = huff + kHuffLut;
+    uint4 *htable = reinterpret_cast<uint4 *>(hslots + kSlots * kSlotBytes);   // [slot][128]
+    uint8_t *hraw4 = reinterpret_cast<uint8_t *>(htable + kSlots * kBM);       // [slot][128]
+    uint8_t *hscratch = hraw4 + kHuffRaw4;
+    uint32_t *masks = reinterpret_cast<uint32_t *>(huff + (HUFF ? kHuffBytes : 0));   // [dc][4]
     uint64_t *c_full = reinterpret_cast<uint64_t *>(masks + 4 * dc);
     uint64_t *c_empty = c_full + dc;
     uint64_t *w_full = c_empty + dc;
@@ -135,7 +280,10 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
     uint64_t *acc_empty = acc_full + 2;     // [2]
     uint64_t *never = acc_empty + 2;
     uint64_t *mma_done = never + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *s_full = mma_done + 1;        // [kSlots] (Huffman)
+    uint64_t *s_empty = s_full + kSlots;    // [kSlots]
+    uint64_t *lut_full = s_empty + kSlots;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(lut_full + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *last_flag = abort_flag + 1;
 
@@ -146,7 +294,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < dc; s++) {
-            mbar_init(&c_full[s], 1);
+            mbar_init(&c_full[s], HUFF ? 1 + 4 : 1);   // producer (+ the 4 decoder warps of a group)
             mbar_init(&c_empty[s], kRebuildWarps);
         }
         for (int s = 0; s < dw; s++) {
@@ -163,12 +311,19 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
         }
         mbar_init(never, 1);
         mbar_init(mma_done, 1);
+        if (HUFF) {
+            for (int s = 0; s < kSlots; s++) {
+                mbar_init(&s_full[s], 32);           // every stream-producer lane
+                mbar_init(&s_empty[s], 4);           // the 4 decoder warps of the group
+            }
+            mbar_init(lut_full, 1);
+        }
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(tmX);
         prefetch_tensormap(tmA);
-        if (FUSED) prefetch_tensormap(tmB);
+        if (MODE == kModePal) prefetch_tensormap(tmB);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -239,9 +394,10 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     masks[4 * s + 1] = m1;
                     masks[4 * s + 2] = m2;
                     masks[4 * s + 3] = m3;
-                    mbar_arrive_expect_tx(&c_full[s], uint32_t(kTileSM + kTilePL) + uint32_t(kGroup) * nraw);
+                    const uint32_t tile_bytes = HUFF ? uint32_t(kTileSM) : uint32_t(kTileSM + kTilePL);
+                    mbar_arrive_expect_tx(&c_full[s], tile_bytes + uint32_t(kGroup) * nraw);
                     tma_load_2d(st, tmA, ks * kBK, int32_t(n0), &c_full[s]);
-                    tma_load_2d(st + kOffPL, tmB, ks * (kBK / 2), int32_t(n0), &c_full[s]);
+                    if (!HUFF) tma_load_2d(st + kOffPL, tmB, ks * (kBK / 2), int32_t(n0), &c_full[s]);
                 }
                 __syncwarp();
 #pragma unroll
@@ -251,10 +407,11 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                                  kGroup, &c_full[s]);
                 issued = i + 1;
             }
-            // no copy may still be landing when the CTA exits
+            // no copy may still be landing when the CTA exits (after an abort a
+            // decoder's arrival may be missing: those waits run out, bounded)
             if (lane == 0)
                 for (int i = max(0, issued - dc); i < issued; i++)
-                    mbar_wait(&c_full[i % dc], uint32_t(i / dc) & 1u, T);
+                    mbar_wait(&c_full[i % dc], uint32_t(i / dc) & 1u, *abort_flag ? T / 64 + 1 : T);
         } else if (lane == 0) {
             for (int i = 0; i < nu; i++) {
                 const int64_t u = u0 + i;
@@ -431,7 +588,8 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 if (warp == kEpiWarp0 && lane == 0) a.counters[t] = 0u;
             }
         }
-    } else if constexpr (FUSED) {
+    } else if (warp < kStreamWarp) {
+        if constexpr (FUSED) {
         // ------------------------------------------------------------ rebuild
         const int tid = threadIdx.x - 32 * kFirstRebuildWarp;   // 0..255
         const int r = tid >> 1, h = tid & 1;
@@ -477,6 +635,155 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_full[ws]);
         }
+        }
+    } else if (warp == kStreamWarp) {
+        if constexpr (HUFF) {
+            // -------------------------------------------------------- stream producer
+            if (lane == 0) {   // the decode table, once
+                mbar_arrive_expect_tx(lut_full, uint32_t(kHuffLut));
+                bulk_g2s(hlut, a.dlut, kHuffLut, lut_full);
+            }
+            const int64_t G4 = a.k / (4 * kGroup);      // chunks per row
+            int sidx = 0;
+            for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
+                const int slot = sidx % kSlots;
+                int stop = 0;
+                if (lane == 0) {
+                    const bool ok = sidx < kSlots ||
+                                    mbar_wait_or_abort(&s_empty[slot], (uint32_t(sidx / kSlots) & 1u) ^ 1u, T,
+                                                       abort_flag);
+                    if (!ok) fail(!*abort_flag);
+                    stop = !ok || *abort_flag;
+                }
+                if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
+                const int64_t n0 = (ss.t / a.TB) * kBM;
+                uint32_t start[4], end[4], wfirst[4], bytes[4], raw4[4];
+#pragma unroll
+                for (int mm = 0; mm < 4; mm++) {
+                    const int64_t row = n0 + lane + 32 * mm;
+                    start[mm] = end[mm] = wfirst[mm] = bytes[mm] = raw4[mm] = 0u;
+                    if (row < a.n) {
+                        const int64_t c = row * G4 + ss.j;
+                        start[mm] = __ldg(a.chunk_off + c);
+                        end[mm] = __ldg(a.chunk_off + c + 1);
+                        const int64_t g = 4 * c;
+                        raw4[mm] = (__ldg(a.flagbits + (g >> 5)) >> (uint32_t(g) & 31u)) & 15u;
+                    }
+                }
+                // words [wfirst, wlast) hold bits [start, end) and the two words a
+                // window at `end` reads; whole 16-byte granules
+                uint32_t incl = 0;
+#pragma unroll
+                for (int mm = 0; mm < 4; mm++) {
+                    const bool sane = start[mm] <= end[mm] && uint64_t(end[mm]) <= a.stream_bits;
+                    if (sane && end[mm] > start[mm]) {
+                        wfirst[mm] = (start[mm] >> 5) & ~3u;
+                        const uint32_t wlast = ((end[mm] + 31u) >> 5) + 2u;
+                        bytes[mm] = ((wlast - wfirst[mm] + 3u) & ~3u) * 4u;
+                    }
+                    incl += bytes[mm];
+                }
+                // offsets: an exclusive prefix sum over the lanes, then the lane's rows in order
+                uint32_t scan = incl;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, scan, d);
+                    if (lane >= d) scan += v;
+                }
+                uint32_t off = scan - incl, staged = 0;
+                uint4 *tab = htable + slot * kBM;
+#pragma unroll
+                for (int mm = 0; mm < 4; mm++) {
+                    const int r = lane + 32 * mm;
+                    const bool fits = bytes[mm] > 0 && off + bytes[mm] <= uint32_t(kSlotBytes);
+                    tab[r] = make_uint4(fits ? off : kFromGlobal, wfirst[mm], start[mm], end[mm]);
+                    hraw4[slot * kBM + r] = uint8_t(raw4[mm]);
+                    if (fits) staged += bytes[mm];
+                    off += bytes[mm];
+                }
+                const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, staged);
+                if (lane == 0) mbar_arrive_expect_tx(&s_full[slot], total);
+                __syncwarp();
+                if (lane != 0) mbar_arrive(&s_full[slot]);
+                off = scan - incl;
+                uint8_t *sbase = hslots + slot * kSlotBytes;
+#pragma unroll
+                for (int mm = 0; mm < 4; mm++) {
+                    if (bytes[mm] > 0 && off + bytes[mm] <= uint32_t(kSlotBytes))
+                        bulk_g2s(sbase + off, a.stream + wfirst[mm], bytes[mm], &s_full[slot]);
+                    off += bytes[mm];
+                }
+            }
+            // no copy may still be landing when the CTA exits
+            if (lane == 0) {
+                for (int i = max(0, sidx - kSlots); i < sidx; i++)
+                    mbar_wait(&s_full[i % kSlots], uint32_t(i / kSlots) & 1u, T);
+                mbar_wait(lut_full, 0, T);
+            }
+            __syncwarp();
+        }
+    } else {
+        if constexpr (HUFF) {
+            // -------------------------------------------------------- decoders
+            const int dt = threadIdx.x - 32 * kFirstDecWarp;   // 0..255
+            const int grp = dt >> 7, r = dt & 127;
+            const uint32_t lut = smem_addr(hlut);
+            const uint32_t line = smem_addr(hscratch) + uint32_t(dt * kScratchStride);
+            const int sw32 = (r >> 2) & 1;
+            bool ok = mbar_wait_or_abort(lut_full, 0, T, abort_flag);
+            int sidx = 0;
+            for (SuperSteps ss(u0, u1, a.S); ss.valid() && ok; ss.next(), sidx++) {
+                if ((sidx & 1) != grp) continue;
+                const int slot = sidx % kSlots;
+                ok = mbar_wait_or_abort(&s_full[slot], uint32_t(sidx / kSlots) & 1u, T, abort_flag);
+                if (__any_sync(0xFFFFFFFFu, !ok)) {
+                    ok = false;
+                    break;
+                }
+                const uint4 e = htable[slot * kBM + r];
+                const uint32_t raw4 = hraw4[slot * kBM + r];
+                const int64_t row = (ss.t / a.TB) * kBM + r;
+                uint32_t p = e.z;
+                const uint32_t end = e.w;
+                bool good = e.z <= e.w && uint64_t(e.w) <= a.stream_bits;
+                const uint32_t sbase = smem_addr(hslots + slot * kSlotBytes) + (e.x & ~kFromGlobal);
+                const uint32_t wfirst = e.y;
+                const auto staged = [&](uint32_t wi) { return lds32(sbase + 4u * (wi - wfirst)); };
+                const auto global = [&](uint32_t wi) { return __ldg(a.stream + wi); };
+#pragma unroll 1
+                for (int q = 0; q < 4; q++) {
+                    const int ks = 4 * ss.j + q;
+                    const bool raw = (raw4 >> q) & 1u;
+                    if (row < a.n && !raw && good)
+                        good = (e.x & kFromGlobal) ? decode_group(global, p, end, lut, line, a.code_len)
+                                                   : decode_group(staged, p, end, lut, line, a.code_len);
+                    if (ks < ss.ka || ks >= ss.kb) continue;   // a K-step another CTA owns (uniform)
+                    const int i = int(ss.t * a.S + ks - u0);
+                    const int cs = i % dc;
+                    ok = i < dc || mbar_wait_or_abort(&c_empty[cs], (uint32_t(i / dc) & 1u) ^ 1u, T, abort_flag);
+                    if (__any_sync(0xFFFFFFFFu, !ok)) {
+                        ok = false;
+                        break;
+                    }
+                    if (row < a.n && !raw) {
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int w = 0; w < 8; w++) wv[w] = good ? natural_to_pal(lds32(line + 4u * w)) : 0u;
+                        uint8_t *pl = cring + size_t(cs) * kCStage + kOffPL + r * 32;
+                        *reinterpret_cast<uint4 *>(pl + (sw32 << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        *reinterpret_cast<uint4 *>(pl + ((1 ^ sw32) << 4)) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&c_full[cs]);
+                }
+                if (!ok) break;
+                // a chunk must decode cleanly and end exactly where the next starts
+                if (row < a.n && (!good || p != end)) flag_error(a.status, UW_DEVERR_CORRUPT);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[slot]);
+            }
+            if (!ok && lane == 0 && !*abort_flag) fail(true);
+        }
     }
 
     tc_fence_before();
@@ -488,17 +795,24 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kFusedThreads, 1)
+__global__ void __launch_bounds__(kPalThreads, 1)
     k_gemm_sk_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmSM,
                     const __grid_constant__ CUtensorMap tmPL, const SkArgs a) {
-    sk_body<true, BN>(&tmX, &tmSM, &tmPL, a);
+    sk_body<kModePal, BN>(&tmX, &tmSM, &tmPL, a);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kHuffThreads, 1)
+    k_gemm_sk_huff(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmSM,
+                   const SkArgs a) {
+    sk_body<kModeHuff, BN>(&tmX, &tmSM, &tmSM, a);
 }
 
 template <int BN>
 __global__ void __launch_bounds__(kPlainThreads, 1)
     k_gemm_sk_plain(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const SkArgs a) {
-    sk_body<false, BN>(&tmX, &tmW, &tmW, a);
+    sk_body<kModePlain, BN>(&tmX, &tmW, &tmW, a);
 }
 
 // ============================================================== host side
@@ -515,33 +829,40 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// ring depths per token tile (compressed depth for the fused flavour is the
+// ring depths per token tile (compressed depth for the fused flavours is the
 // largest that fits, at most 6, unless the plan asks for fewer)
 struct Depths {
     int dc, dw, dx;
 };
-Depths depths(bool fused, int bn, int stages) {
+Depths depths(int mode, int bn, int stages) {
     const int kx = bn * kBK * 2;
     Depths d{};
-    if (fused) {
+    if (mode == kModePal) {
         d.dw = bn <= 128 ? 3 : 2;
         d.dx = bn <= 64 ? 4 : (bn == 128 ? 3 : 2);
-        int room = kMaxSmem - 1024 - d.dw * kTileW - d.dx * kx - sk_tail(8, d.dw, d.dx);
+        const int room = kMaxSmem - 1024 - d.dw * kTileW - d.dx * kx - sk_tail(8, d.dw, d.dx);
+        d.dc = std::min(6, room / kCStage);
+        if (stages > 0) d.dc = std::min(d.dc, stages);
+    } else if (mode == kModeHuff) {
+        d.dw = 2;
+        d.dx = bn <= 64 ? 3 : 2;
+        const int room = kMaxSmem - 1024 - d.dw * kTileW - d.dx * kx - kHuffBytes - sk_tail(8, d.dw, d.dx);
         d.dc = std::min(6, room / kCStage);
         if (stages > 0) d.dc = std::min(d.dc, stages);
     } else {
         d.dc = 0;
         d.dx = bn <= 64 ? 6 : (bn == 128 ? 4 : 3);
-        int room = kMaxSmem - 1024 - d.dx * kx - sk_tail(0, 8, d.dx);
+        const int room = kMaxSmem - 1024 - d.dx * kx - sk_tail(0, 8, d.dx);
         d.dw = std::min(8, room / kTileW);
         if (stages > 0) d.dw = std::min(d.dw, std::max(2, stages));
     }
     return d;
 }
 
-size_t smem_bytes(bool fused, int bn, const Depths &d) {
-    return size_t(d.dw) * kTileW + size_t(d.dx) * bn * kBK * 2 + (fused ? size_t(d.dc) * kCStage : 0) + 1024 +
-           sk_tail(fused ? d.dc : 0, d.dw, d.dx);
+size_t smem_bytes(int mode, int bn, const Depths &d) {
+    const bool fused = mode != kModePlain;
+    return size_t(d.dw) * kTileW + size_t(d.dx) * bn * kBK * 2 + (fused ? size_t(d.dc) * kCStage : 0) +
+           (mode == kModeHuff ? size_t(kHuffBytes) : 0) + 1024 + sk_tail(fused ? d.dc : 0, d.dw, d.dx);
 }
 
 int device_sms() {
@@ -561,35 +882,37 @@ int device_sms() {
     return cache[dev];
 }
 
+// Once per (kernel, device): the shared-memory opt-in, and a check that one
+// CTA fits an SM and that co-resident CTAs would fit the 512 TMEM columns
+// (tcgen05.alloc would block).  Launches use at least half the SM's shared
+// memory, so the occupancy found for that size holds for every launch.
 template <class K>
-cudaError_t prepare(K kern, int threads, size_t smem, uint32_t tmem_cols, int (&ready)[64]) {
+cudaError_t prepare(K kern, int threads, uint32_t tmem_cols, int (&ready)[64]) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!ready[dev]) {
-        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-        if (err != cudaSuccess) return err;
-        ready[dev] = 1;
-    }
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (ready[dev]) return cudaSuccess;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (err != cudaSuccess) return err;
-    // a second CTA on the SM would block in tcgen05.alloc until the first ends
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, size_t(kMaxSmem / 2 + 1024));
+    if (err != cudaSuccess) return err;
     if (per_sm < 1 || per_sm * int(tmem_cols) > 512) return cudaErrorInvalidConfiguration;
+    ready[dev] = 1;
     return cudaSuccess;
 }
 
 template <int BN>
 cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
     using C = SkCfg<BN>;
-    const bool fused = p.w_bf16 == nullptr;
+    const int mode = p.w_bf16 ? kModePlain : (p.huffman ? kModeHuff : kModePal);
     const SkGeometry g = sk_geometry(p.m, p.n, p.k, BN);
     if (g.G <= 0) return cudaErrorInvalidValue;
     if (!p.sk_counters || !p.partial) return cudaErrorInvalidValue;
-    const Depths d = depths(fused, BN, p.stages);
-    if ((fused && d.dc < 2) || d.dw < 2 || d.dx < 2) return cudaErrorInvalidValue;
-    size_t smem = smem_bytes(fused, BN, d);
+    const Depths d = depths(mode, BN, p.stages);
+    if ((mode != kModePlain && d.dc < 2) || d.dw < 2 || d.dx < 2) return cudaErrorInvalidValue;
+    size_t smem = smem_bytes(mode, BN, d);
     smem = std::max(smem, size_t(kMaxSmem / 2 + 1024));   // one CTA per SM
     if (smem > size_t(kMaxSmem)) return cudaErrorInvalidValue;
 
@@ -616,27 +939,47 @@ cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
                   BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     cudaError_t err;
-    if (fused) {
+    if (mode != kModePlain) {
         a.flagbits = p.w->flagbits;
         a.rawbase = p.w->rawbase;
         a.rawexp = p.w->rawexp;
         a.nflag = (p.n * (p.k / kGroup) + 31) / 32;
         a.pal = make_palette16(p.w->palette);
         if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k), kBK,
-                      kBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-            !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n), uint64_t(p.k / 2),
+                      kBM, CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
+    }
+    if (mode == kModePal) {
+        if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n), uint64_t(p.k / 2),
                       kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
             return cudaErrorInvalidValue;
         static int ready[64] = {0};
-        err = prepare(k_gemm_sk_fused<BN>, kFusedThreads, smem, C::kTmemCols, ready);
+        err = prepare(k_gemm_sk_fused<BN>, kPalThreads, C::kTmemCols, ready);
         if (err != cudaSuccess) return err;
-        k_gemm_sk_fused<BN><<<unsigned(g.G), kFusedThreads, smem, stream>>>(mx, ma, mb, a);
+        k_gemm_sk_fused<BN><<<unsigned(g.G), kPalThreads, smem, stream>>>(mx, ma, mb, a);
+    } else if (mode == kModeHuff) {
+        // chunks of 4 groups must not straddle rows; the decoders' table
+        // needs the Huffman sections
+        if (BN > 128 || p.k % (4 * kGroup) || !p.w->stream || !p.w->chunk_off || !p.w->dlut)
+            return cudaErrorInvalidValue;
+        a.stream = p.w->stream;
+        a.chunk_off = p.w->chunk_off;
+        a.dlut = p.w->dlut;
+        a.stream_bits = p.w->stream_bits;
+        a.code_len = 0;
+        for (int i = 0; i < 16; i++) a.code_len |= uint64_t(p.w->code_len[i] & 15u) << (4 * i);
+        if constexpr (BN <= 128) {
+            static int ready[64] = {0};
+            err = prepare(k_gemm_sk_huff<BN>, kHuffThreads, C::kTmemCols, ready);
+            if (err != cudaSuccess) return err;
+            k_gemm_sk_huff<BN><<<unsigned(g.G), kHuffThreads, smem, stream>>>(mx, ma, a);
+        }
     } else {
         if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.w_bf16, uint64_t(p.k), uint64_t(p.n),
                       uint64_t(p.k) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         static int ready[64] = {0};
-        err = prepare(k_gemm_sk_plain<BN>, kPlainThreads, smem, C::kTmemCols, ready);
+        err = prepare(k_gemm_sk_plain<BN>, kPlainThreads, C::kTmemCols, ready);
         if (err != cudaSuccess) return err;
         k_gemm_sk_plain<BN><<<unsigned(g.G), kPlainThreads, smem, stream>>>(mx, ma, a);
     }

@@ -105,6 +105,7 @@ struct TcLaunch {
     float *y;                  // [m, n]
     float *partial;            // [split_k, m, n] when split_k > 1; stream-K: partial tiles
     uint32_t *sk_counters;     // stream-K: one counter per tile (zero between calls)
+    bool huffman;              // stream-K fused: decode the palette indices from the Huffman stream
     int bn, split_k, stages;
     uint32_t debug_flags;
     uint64_t timeout_ns;

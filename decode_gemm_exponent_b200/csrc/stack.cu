@@ -102,7 +102,7 @@ extern "C" uw_status uw_stack_run(const uw_stack_step *steps, int n_steps, void 
         if ((reinterpret_cast<uintptr_t>(s.x_dev) | reinterpret_cast<uintptr_t>(s.y_dev)) & 15u) return UW_ERR_INVALID_ARG;
         if (s.w->n <= 0 || s.w->k <= 0) return UW_ERR_INVALID_ARG;
         if (s.w->n % 64 || s.w->k % 64) return UW_ERR_UNSUPPORTED_SHAPE;
-        if (needs_prep(s.plan)) {
+        if (needs_prep(s.plan) || s.plan.pipeline == UW_PIPE_HUFFMAN_FUSED) {
             if (!(s.w->flags & UW_EMIT_HUFFMAN) || !s.w->stream) return UW_ERR_INVALID_ARG;
         } else {
             const uint8_t *pal = s.pal_dev ? s.pal_dev : s.w->pal;

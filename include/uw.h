@@ -196,7 +196,14 @@ typedef enum uw_pipeline {
                                      from the sign/mantissa and exponent bytes      */
     UW_PIPE_TRANSCODE_FUSED = 3,  /* transcode to the palette plane in the workspace, then
                                      the fused kernel                                    */
-    UW_PIPE_DIRECT_PALETTE = 4    /* fused kernel on the blob's (or a given) palette plane */
+    UW_PIPE_DIRECT_PALETTE = 4,   /* fused kernel on the blob's (or a given) palette plane */
+    UW_PIPE_HUFFMAN_FUSED = 5     /* the fused stream-K kernel decodes the Huffman stream to
+                                     palette indices in shared memory as it goes (pipeline 3's
+                                     transcode inside the matmul's producer): no preprocessing
+                                     pass and no workspace beyond the stream-K scratch.  Needs
+                                     UW_EMIT_HUFFMAN, kernel UW_KERNEL_TC_SK with bn <= 128 and
+                                     k a multiple of 256 (a 4-group stream chunk never
+                                     straddles two rows); UW_ERR_INVALID_ARG otherwise       */
 } uw_pipeline;
 
 typedef enum uw_kernel {

@@ -39,14 +39,19 @@ def check_bound(y_gpu, y_ref, a_ref):
         float((err / np.maximum(TOL * a_ref, 1e-30)).max()), np.argwhere(bad)[:5].tolist())
 
 
-def sk_case(uw, n, k, m, bn, seed=0, frac=0.002, pipelines=(1, 2, 3, 4), stages=0, oracle=True):
-    w = synth.weights_bf16(n, k, 0.02, frac, 1.0, seed=seed)
+def sk_case(uw, n, k, m, bn, seed=0, frac=0.002, pipelines=(1, 2, 3, 4, 5), stages=0, oracle=True, w=None):
+    """Plain BF16 twin vs every pipeline (pipeline 5, the in-kernel Huffman
+    decode, where the shape allows it) bit for bit, and the oracle bound."""
+    if w is None:
+        w = synth.weights_bf16(n, k, 0.02, frac, 1.0, seed=seed)
     x = synth.activations_bf16(m, k, seed=seed)
     mat = uw.Matrix(uw.encode(w))
     xd, wd = dev16(x), dev16(w)
     kw = dict(kernel=uw.KERNEL_TC_SK, bn=bn, split_k=1, stages=stages)
     y_plain = uw.matmul_bf16(xd, wd, uw.make_plan(pipeline=4, **kw)).cpu().numpy()
     for pipe in pipelines:
+        if pipe == uw.PIPE_HUFFMAN_FUSED and (bn > 128 or k % 256):
+            continue
         y = mat.matmul(xd, uw.make_plan(pipeline=pipe, **kw)).cpu().numpy()
         assert np.array_equal(y.view(np.uint32), y_plain.view(np.uint32)), "pipeline %d differs" % pipe
     assert mat.device_status() == 0
@@ -69,6 +74,56 @@ def test_sk_ragged_rows_and_unaligned_bitmap_words(uw):
     sk_case(uw, 320, 704, 40, 64, seed=3, frac=0.05)
     sk_case(uw, 320, 704, 3, 16, seed=4, frac=0.05)
     sk_case(uw, 192, 1344, 17, 32, seed=5, frac=0.002)
+    # k = 1280 (5 chunks per row) for the in-kernel Huffman decode: ragged rows, raw-heavy
+    sk_case(uw, 320, 1280, 24, 32, seed=13, frac=0.05)
+    sk_case(uw, 192, 1280, 5, 16, seed=14, frac=0.002)
+
+
+def test_sk_huffman_chunks_larger_than_a_stream_slot(uw):
+    """Exponents uniform over 16 values: every code is 4 bits, a chunk takes
+    1024 bits, and a super-step's 128 chunks (18 KB with their granules) do
+    not all fit the 12 KB stream slot, so some decoders read the stream from
+    global memory.  Results still equal the plain kernel bit for bit."""
+    rng = np.random.default_rng(21)
+    n, k = 256, 2048
+    e = rng.integers(110, 126, n * k).astype(np.uint16)
+    sm = rng.integers(0, 256, n * k).astype(np.uint16)
+    w = (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16).reshape(n, k)
+    sk_case(uw, n, k, 16, 16, seed=22, pipelines=(4, 5), w=w)
+    sk_case(uw, n, k, 100, 128, seed=23, pipelines=(5,), w=w)
+
+
+def test_sk_huffman_corrupt_stream_is_reported(uw):
+    w = synth.weights_bf16(256, 1024, 0.02, 0.001, 1.0, seed=24)
+    blob = uw.encode(w)
+    mat = uw.Matrix(blob)
+    off = mat.info.section_offset[uw.SEC_STREAM] + 256
+    mat.dev[off:off + 16] ^= 0x5A                      # the device copy only
+    xd = dev16(synth.activations_bf16(8, 1024, seed=24))
+    p = uw.make_plan(pipeline=uw.PIPE_HUFFMAN_FUSED, kernel=uw.KERNEL_TC_SK, bn=16, split_k=1)
+    mat.matmul(xd, p)
+    assert mat.device_status() == 3                   # UW_ERR_CORRUPT
+    clean = uw.Matrix(blob)                           # the context is still usable
+    y = clean.matmul(xd, p).cpu().numpy()
+    assert clean.device_status() == 0
+    y_ref, a_ref = O.gemm(synth.activations_bf16(8, 1024, seed=24), w)
+    check_bound(y, y_ref, a_ref)
+
+
+def test_sk_huffman_plan_checks(uw):
+    w = synth.weights_bf16(128, 704, 0.02, 0.0, 1.0, seed=25)
+    mat = uw.Matrix(uw.encode(w))
+    xd = dev16(synth.activations_bf16(4, 704, seed=25))
+    for kw in (dict(kernel=uw.KERNEL_TC_SK, bn=16),       # k = 704 is not a multiple of 256
+               dict(kernel=uw.KERNEL_TC, bn=16)):          # only the stream-K kernel decodes in place
+        with pytest.raises(uw.UwError) as e:
+            mat.matmul(xd, uw.make_plan(pipeline=uw.PIPE_HUFFMAN_FUSED, split_k=1, **kw))
+        assert e.value.status == 1
+    w2 = synth.weights_bf16(128, 1024, 0.02, 0.0, 1.0, seed=26)
+    mat2 = uw.Matrix(uw.encode(w2, flags=uw.EMIT_PALETTE))  # no Huffman stream in the blob
+    with pytest.raises(uw.UwError):
+        mat2.matmul(dev16(synth.activations_bf16(4, 1024, seed=26)),
+                    uw.make_plan(pipeline=uw.PIPE_HUFFMAN_FUSED, kernel=uw.KERNEL_TC_SK, bn=16, split_k=1))
 
 
 def test_sk_many_pieces_per_tile(uw):
@@ -157,8 +212,8 @@ def test_sk_stack_shares_scratch_with_split_k_steps(uw):
 @pytest.mark.parametrize("proj", [(14336, 4096), (4096, 14336)])
 def test_sk_full_size_8b_sampled(uw, m, bn, proj):
     """Llama-3.1-8B gate and down shapes at the bench's batch sizes: fused
-    (palette and exponent-plane pipelines) == plain bit for bit over the whole
-    output, and 512 sampled outputs within the oracle bound."""
+    (palette, exponent-plane and in-kernel Huffman pipelines) == plain bit for
+    bit over the whole output, and 512 sampled outputs within the oracle bound."""
     n, k = proj
     w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=1)
     x = synth.activations_bf16(m, k, seed=1)
@@ -166,7 +221,7 @@ def test_sk_full_size_8b_sampled(uw, m, bn, proj):
     xd, wd = dev16(x), dev16(w)
     kw = dict(kernel=uw.KERNEL_TC_SK, bn=bn, split_k=1)
     yp = uw.matmul_bf16(xd, wd, uw.make_plan(pipeline=4, **kw)).cpu().numpy()
-    for pipe in (4, 2):
+    for pipe in ((4, 2, 5) if bn <= 128 else (4, 2)):
         yf = mat.matmul(xd, uw.make_plan(pipeline=pipe, **kw)).cpu().numpy()
         assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32)), "pipeline %d" % pipe
     assert mat.device_status() == 0
