@@ -162,6 +162,20 @@ __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
                  : "memory");
 }
 
+// 16-byte cp.async that reads `src_bytes` (0 or 16) bytes and fills the rest
+// of the 16 with zeros (src must still be a valid address)
+__device__ __forceinline__ void cp_async16_zfill(void *dst_smem, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst_smem)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// Raise the transaction count of `bar`'s current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
 // Make `bar`'s current phase also wait for this thread's earlier cp.async
 // copies (the pending count is raised now and lowered when they land).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {

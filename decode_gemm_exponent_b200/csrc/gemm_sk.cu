@@ -25,37 +25,45 @@
 // CTA order (= K order) and writes Y, then zeroes the counter.  No CTA waits
 // for another, and the sum order is fixed by the schedule alone.
 //
+// Loads.  Measured on this GPU, a TMA copy costs the SM's copy engine about
+// the same time whether it moves 2 KB or 16 KB, so small copies cap the
+// bandwidth far below HBM.  Compressed W therefore arrives in super-steps of
+// four K-steps (one 4-group chunk of every row): two 16 KB sign/mantissa
+// boxes and one 16 KB palette box, all 128-byte swizzled.  Small or scattered
+// data -- X tiles of up to 64 tokens, the exponents of raw groups, Huffman
+// stream words -- go through the load/store path (cp.async, 16 bytes a lane).
+//
 // Roles (warps):
-//   0      producer: per K-step the sign/mantissa tile (TMA, 64-byte swizzle),
-//          the 4-bit palette tile (TMA, 32-byte swizzle; palette flavour), and
-//          for each raw (row, group) its 64 exponents by a 64-byte bulk copy,
-//          all counted on one barrier; the 32 lanes share the 128 rows' raw
-//          bits and write the step's 128-bit raw mask next to the stage.
-//          Plain flavour: the BF16 W tile (TMA, 128-byte swizzle).
+//   0      producer: per super-step the TMA boxes (W tiles for the plain
+//          flavour: one 16 KB box per K-step) and, in the fused flavours, the
+//          super-step's raw groups: the 32 lanes find the raw (row, group)
+//          pairs of the 128 rows, give each a slot in the stage (cp.async of
+//          its 64 exponents) and write a 128 x 4 table that tells the rebuild
+//          where each group's exponents are (palette plane, a slot, or, when
+//          the slots run out, the raw plane in global memory).
 //   1      MMA issuer and TMEM owner: 4 x tcgen05.mma (K = 16) per K-step into
 //          one of two accumulators (double-buffered, so the epilogue of one
 //          tile overlaps the MMAs of the next).
-//   2      X producer (TMA, 128-byte swizzle).
+//   2      X producer: cp.async into the 128-byte-swizzled K-major layout for
+//          up to 64 tokens, a TMA box per K-step for 128 and 256.
 //   3-6    epilogue: TMEM -> registers -> Y (or a partial tile + fix-up).
 //   7-14   rebuild (palette, Huffman): all 8 warps work on the same K-step;
-//          thread t rebuilds 32 weights (half h = t & 1) of tile row r = t >> 1
-//          into the 128-byte-swizzled K-major BF16 W tile.  The thread-to-data
-//          map keeps every 16-byte shared-memory access of a quarter warp on
-//          distinct bank groups (sign/mantissa, palette words and W stores).
-//   15     (Huffman) stream producer: per super-step (the K-steps of one
-//          4-group stream chunk in each of the tile's 128 rows) it reads the
-//          128 chunks' start bits, packs the chunks' stream words into one
-//          slot of a 4-slot shared-memory ring with bulk copies, and writes a
-//          table of where each chunk's words are (a chunk that does not fit
-//          the slot is read from global memory by its decoder instead).
+//          lane l of warp w rebuilds half h = (l >> 3) & 1 (32 weights) of
+//          tile row 16w + 8(l >> 4) + (l & 7) into the 128-byte-swizzled
+//          K-major BF16 W tile.  A quarter warp covers 8 consecutive rows, so
+//          under the 128-byte swizzle every 16-byte shared-memory access of
+//          it falls on its own bank group.
+//   15     (Huffman) stream producer: per super-step it reads the 128 chunks'
+//          start bits and copies each chunk's stream words (cp.async) into
+//          one slot of a shared-memory ring, with a table of where they are
+//          (a chunk that does not fit is read from global memory instead).
 //   16-23  (Huffman) decoders: two groups of 4 warps take alternate
-//          super-steps, one thread per tile row.  A thread decodes its row's
-//          chunk group by group with the 12-bit multi-symbol table, each
-//          group's 64 indices into a private scratch line, then copies them
-//          into the K-step's compressed stage in the stored 4-bit layout.
+//          super-steps, one thread per tile row; a thread decodes its row's
+//          chunk with the 12-bit multi-symbol table straight into the
+//          super-step's palette area, in the stored 4-bit layout.
 // Every wait is bounded; on time-out a role raises UW_DEVERR_TIMEOUT and sets
-// the CTA's abort flag, which ends every other wait of the CTA; TMA copies
-// and MMAs in flight are waited for (bounded) before TMEM is freed.
+// the CTA's abort flag, which ends every other wait of the CTA; copies and
+// MMAs in flight are waited for (bounded) before TMEM is freed.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -73,6 +81,7 @@ constexpr int kModePlain = 0, kModePal = 1, kModeHuff = 2;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
+constexpr int kSuper = 4;               // K-steps per super-step (one 4-group stream chunk)
 constexpr int kMaxSmem = 232448;        // 227 KB opt-in per CTA
 constexpr int kFixedWarps = 7;          // producer, MMA, X producer, 4 epilogue warps
 constexpr int kRebuildWarps = 8;
@@ -85,18 +94,31 @@ constexpr int kPlainThreads = kFixedWarps * 32;
 constexpr int kPalThreads = (kFixedWarps + kRebuildWarps) * 32;
 constexpr int kHuffThreads = (kFixedWarps + kRebuildWarps + 1 + kDecWarps) * 32;
 
-constexpr int kTileW = kBM * kBK * 2;            // BF16 W tile
-constexpr int kTileSM = kBM * kBK;               // sign/mantissa tile
-constexpr int kTilePL = kBM * kBK / 2;           // 4-bit palette tile
-constexpr int kTileRAW = kBM * kGroup;           // one 64-byte exponent slot per row
-constexpr int kCStage = kTileSM + kTilePL + kTileRAW;
-constexpr int kOffPL = kTileSM, kOffRAW = kTileSM + kTilePL;
+constexpr int kTileW = kBM * kBK * 2;   // BF16 W tile of one K-step (128 rows x 128 B)
+
+// compressed super-step stage (fused flavours)
+constexpr int kBox = kBM * 128;                  // one 128-row x 128-byte box
+constexpr int kOffSmA = 0;                       // sign/mantissa, K-steps 0-1 of the super-step
+constexpr int kOffSmB = kBox;                    //                K-steps 2-3
+constexpr int kOffNib = 2 * kBox;                // 4-bit palette indices, K-steps 0-3
+constexpr int kRawSlots = 128;                   // raw groups staged per super-step
+constexpr int kOffRaw = 3 * kBox;                // kRawSlots x 64 exponent bytes
+constexpr int kOffTab = kOffRaw + kRawSlots * kGroup;   // uint32 [128 rows][4 K-steps]
+constexpr int kCStage = kOffTab + kBM * kSuper * 4;
+static_assert(kCStage % 1024 == 0, "stages keep 1024-byte alignment");
+// raw table entry: 0 = palette; kTabSlot | slot = staged exponents;
+// kTabRank | rank = the raw plane at 64 * rank (no slot left)
+constexpr uint32_t kTabSlot = 0x80000000u, kTabRank = 0x40000000u;
 
 // Huffman flavour
-constexpr int kSlots = 4;                        // stream slots (super-steps staged ahead)
+constexpr int kSlots = 3;                        // stream slots (super-steps staged ahead)
 constexpr int kSlotBytes = 12 * 1024;            // stream bytes per slot (~85 B per chunk at 2.6 bits/weight)
-constexpr int kScratchStride = 36;               // bytes per decoder thread: 8 words + 1 of padding
-constexpr uint32_t kFromGlobal = 0x80000000u;    // table flag: the chunk's words are read from global memory
+constexpr uint32_t kFromGlobal = 0x80000000u;    // chunk table flag: read the words from global memory
+constexpr int kHuffLut = kLutEntries * 4;
+constexpr int kHuffTable = kSlots * kBM * 16;    // per slot and row: uint4 {where, first word, start, end}
+constexpr int kHuffRaw4 = kSlots * kBM;          // per slot and row: the chunk's raw-group bits
+constexpr int kHuffBytes = kHuffLut + kSlots * kSlotBytes + kHuffTable + kHuffRaw4;
+static_assert(kHuffBytes % 16 == 0, "Huffman area keeps 16-byte alignment");
 
 struct SkArgs {
     int64_t m, n, k;
@@ -104,9 +126,10 @@ struct SkArgs {
     int S;                    // K-steps per tile
     int TB;                   // token blocks
     int G;                    // CTAs
-    int dc, dw, dx;           // ring depths: compressed, W, X
+    int dc, dw, dx;           // ring depths: compressed super-steps, W tiles, X tiles
     uint32_t debug_flags;
     uint64_t timeout_ns;
+    const uint16_t *x;        // [m, k] BF16 (X by cp.async)
     float *y;
     uint32_t *counters;       // [tiles], zero between calls
     float *partial;           // [2G][BN][128]
@@ -120,6 +143,7 @@ struct SkArgs {
     const uint32_t *chunk_off;
     const uint32_t *dlut;
     uint64_t stream_bits;
+    uint64_t stream_words;    // words of the stream section (padded)
     uint64_t code_len;        // code length of palette index s in bits 4s..4s+3
     uint32_t *status;
 };
@@ -151,37 +175,29 @@ __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
 template <int BN>
 struct SkCfg {
     static constexpr int kX = BN * kBK * 2;
+    static constexpr bool kXByTma = BN >= 128;   // X boxes of 16 KB and more by TMA, smaller by cp.async
     static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32u : uint32_t(2 * BN);   // two accumulators
     static_assert(kX % 1024 == 0, "X stage keeps 1024-byte alignment");
     static_assert(2 * BN <= 512, "accumulators exceed TMEM");
 };
 
-// Huffman flavour: decode table, stream slots, their chunk tables and the
-// decoders' scratch lines, placed after the compressed ring
-constexpr int kHuffLut = kLutEntries * 4;
-constexpr int kHuffTable = kSlots * kBM * 16;    // per slot and row: uint4 {where, first word, start, end}
-constexpr int kHuffRaw4 = kSlots * kBM;          // per slot and row: the chunk's raw-group bits
-constexpr int kHuffScratch = kDecWarps * 32 * kScratchStride;
-constexpr int kHuffBytes = kHuffLut + kSlots * kSlotBytes + kHuffTable + kHuffRaw4 + kHuffScratch;
-static_assert(kHuffBytes % 16 == 0, "Huffman area keeps 16-byte alignment");
-
-// shared-memory bytes after the rings (and the Huffman area): raw masks,
-// barriers, TMEM slot, flags
+// shared-memory bytes after the rings (and the Huffman area): barriers,
+// TMEM slot, flags
 __host__ __device__ constexpr int sk_tail(int dc, int dw, int dx) {
-    return dc * 16 + (2 * dc + 2 * dw + 2 * dx + 4 + 2 + 2 * kSlots + 1) * 8 + 16;
+    return (2 * dc + 2 * dw + 2 * dx + 4 + 2 + 2 * kSlots + 1) * 8 + 16;
 }
 
-// The CTA's super-steps: for each tile of its unit range and each 4-group
-// chunk index j touched there, the K-steps [ka, kb) of the tile that the CTA
-// owns.  Walked identically by the stream producer and the decoders.
+// The CTA's super-steps: for each tile of its unit range and each chunk
+// index j (K-steps 4j..4j+3) touched there, the K-steps [lo, hi) the CTA
+// owns.  Walked the same way by every role that works per super-step.
 struct SuperSteps {
     int64_t u0, u1, t, t_last;
     int S, j, j_last, ka, kb;
     __device__ __forceinline__ void start_tile() {
         ka = t == u0 / S ? int(u0 - t * S) : 0;
         kb = t == t_last ? int(u1 - t * S) : S;
-        j = ka >> 2;
-        j_last = (kb - 1) >> 2;
+        j = ka / kSuper;
+        j_last = (kb - 1) / kSuper;
     }
     __device__ __forceinline__ SuperSteps(int64_t u0_, int64_t u1_, int S_) : u0(u0_), u1(u1_), S(S_) {
         t = u0 / S;
@@ -189,6 +205,8 @@ struct SuperSteps {
         start_tile();
     }
     __device__ __forceinline__ bool valid() const { return u1 > u0 && t <= t_last; }
+    __device__ __forceinline__ int lo() const { return max(ka, kSuper * j); }
+    __device__ __forceinline__ int hi() const { return min(kb, kSuper * j + kSuper); }
     __device__ __forceinline__ void next() {
         if (++j > j_last) {
             ++t;
@@ -198,21 +216,20 @@ struct SuperSteps {
 };
 
 // Decode one group's 64 palette indices from bit p of a stream (words read
-// through `word(i)`), 8 per word into the scratch line at shared address
-// `line` (natural order: index i in bits 4(i%8).. of word i/8).  Never starts
-// a step past `end`; false if a window has no valid code or the group does
-// not complete.
-template <class Src>
+// through `word(i)`), handing each full word of 8 indices (natural order:
+// index i in bits 4(i%8)..) to sink(w, word) for w = 0..7.  Never starts a
+// step past `end`; false if a window has no valid code or the group does not
+// complete.
+template <class Src, class Sink>
 __device__ __forceinline__ bool decode_group(const Src &word, uint32_t &p, uint32_t end, uint32_t lut,
-                                             uint32_t line, uint64_t code_len) {
-    uint32_t lo = 0, na = 0, off = 0, rem4 = 256, err = 0;
+                                             uint64_t code_len, const Sink &sink) {
+    uint32_t lo = 0, na = 0, w = 0, rem4 = 256, err = 0;
     auto push = [&](uint32_t s, uint32_t nbits) {
         lo |= s << na;
         const uint32_t carry = __funnelshift_l(s, 0u, na);
         na += nbits;
         if (na >= 32) {
-            sts32(line + off, lo);
-            off += 4u;
+            sink(w++, lo);
             lo = carry;
             na -= 32;
         }
@@ -268,9 +285,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
     uint8_t *hslots = huff + kHuffLut;
     uint4 *htable = reinterpret_cast<uint4 *>(hslots + kSlots * kSlotBytes);   // [slot][128]
     uint8_t *hraw4 = reinterpret_cast<uint8_t *>(htable + kSlots * kBM);       // [slot][128]
-    uint8_t *hscratch = hraw4 + kHuffRaw4;
-    uint32_t *masks = reinterpret_cast<uint32_t *>(huff + (HUFF ? kHuffBytes : 0));   // [dc][4]
-    uint64_t *c_full = reinterpret_cast<uint64_t *>(masks + 4 * dc);
+    uint64_t *c_full = reinterpret_cast<uint64_t *>(huff + (HUFF ? kHuffBytes : 0));
     uint64_t *c_empty = c_full + dc;
     uint64_t *w_full = c_empty + dc;
     uint64_t *w_empty = w_full + dw;
@@ -294,7 +309,9 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < dc; s++) {
-            mbar_init(&c_full[s], HUFF ? 1 + 4 : 1);   // producer (+ the 4 decoder warps of a group)
+            // 32 producer lanes once their table entries are written, 32 once
+            // their cp.async copies landed, + the 4 decoder warps of a group
+            mbar_init(&c_full[s], HUFF ? 64 + 4 : 64);
             mbar_init(&c_empty[s], kRebuildWarps);
         }
         for (int s = 0; s < dw; s++) {
@@ -302,7 +319,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             mbar_init(&w_empty[s], 1);
         }
         for (int s = 0; s < dx; s++) {
-            mbar_init(&x_full[s], 1);
+            mbar_init(&x_full[s], C::kXByTma ? 1 : 32);
             mbar_init(&x_empty[s], 1);
         }
         for (int b = 0; b < 2; b++) {
@@ -313,7 +330,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
         mbar_init(mma_done, 1);
         if (HUFF) {
             for (int s = 0; s < kSlots; s++) {
-                mbar_init(&s_full[s], 32);           // every stream-producer lane
+                mbar_init(&s_full[s], 64);           // stream-producer lanes: table written, words landed
                 mbar_init(&s_empty[s], 4);           // the 4 decoder warps of the group
             }
             mbar_init(lut_full, 1);
@@ -321,7 +338,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
-        prefetch_tensormap(tmX);
+        if (C::kXByTma) prefetch_tensormap(tmX);
         prefetch_tensormap(tmA);
         if (MODE == kModePal) prefetch_tensormap(tmB);
     }
@@ -341,78 +358,101 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        int issued = 0;
         if constexpr (FUSED) {
             const int64_t G64 = a.k / kGroup;     // groups per row
             int64_t wcur[4] = {-1, -1, -1, -1};
             uint32_t bm[4] = {0u, 0u, 0u, 0u}, rb[4] = {0u, 0u, 0u, 0u};
-            for (int i = 0; i < nu; i++) {
-                const int64_t u = u0 + i;
-                const int64_t t = u / a.S;
-                const int ks = int(u - t * a.S);
-                const int64_t n0 = (t / a.TB) * kBM;
-                const int s = i % dc;
-                // raw bits and ranks of this lane's rows r = lane + 32 j
-                uint32_t rawbits = 0u, rank[4] = {0u, 0u, 0u, 0u};
+            int sidx = 0;
+            for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
+                const int cs = sidx % dc;
+                const int64_t n0 = (ss.t / a.TB) * kBM;
+                const int q0 = ss.lo() - kSuper * ss.j, q1 = ss.hi() - kSuper * ss.j;
+                // raw (row, K-step) pairs of this lane's rows r = lane + 32 m
+                uint32_t rawbits = 0u, rank[16];
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const int64_t row = n0 + lane + 32 * j;
-                    if (row < a.n) {
-                        const int64_t g = row * G64 + ks;
-                        const int64_t w = g >> 5;
-                        if (w != wcur[j]) {
-                            bm[j] = __ldg(a.flagbits + w);
-                            rb[j] = __ldg(a.rawbase + w);
-                            wcur[j] = w;
-                            if (w + 1 < a.nflag) {   // the next word into L1 before it is needed
-                                prefetch_l1(a.flagbits + w + 1);
-                                prefetch_l1(a.rawbase + w + 1);
+                for (int mm = 0; mm < 4; mm++) {
+                    const int64_t row = n0 + lane + 32 * mm;
+#pragma unroll
+                    for (int q = 0; q < kSuper; q++) {
+                        rank[4 * mm + q] = 0u;
+                        if (row < a.n && q >= q0 && q < q1) {
+                            const int64_t g = row * G64 + kSuper * ss.j + q;
+                            const int64_t w = g >> 5;
+                            if (w != wcur[mm]) {
+                                bm[mm] = __ldg(a.flagbits + w);
+                                rb[mm] = __ldg(a.rawbase + w);
+                                wcur[mm] = w;
+                                if (w + 1 < a.nflag) {   // the next word into L1 before it is needed
+                                    prefetch_l1(a.flagbits + w + 1);
+                                    prefetch_l1(a.rawbase + w + 1);
+                                }
                             }
-                        }
-                        const uint32_t bit = uint32_t(g) & 31u;
-                        if ((bm[j] >> bit) & 1u) {
-                            rawbits |= 1u << j;
-                            rank[j] = rb[j] + __popc(bm[j] & ((1u << bit) - 1u));
+                            const uint32_t bit = uint32_t(g) & 31u;
+                            if ((bm[mm] >> bit) & 1u) {
+                                rawbits |= 1u << (4 * mm + q);
+                                rank[4 * mm + q] = rb[mm] + __popc(bm[mm] & ((1u << bit) - 1u));
+                            }
                         }
                     }
                 }
-                const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, rawbits & 1u);
-                const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, rawbits & 2u);
-                const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, rawbits & 4u);
-                const uint32_t m3 = __ballot_sync(0xFFFFFFFFu, rawbits & 8u);
-                const uint32_t nraw = __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
-                int ok = 1, stop = 0;
+                // slots: an exclusive prefix sum of the lanes' raw counts
+                const uint32_t cnt = __popc(rawbits);
+                uint32_t scan = cnt;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, scan, d);
+                    if (lane >= d) scan += v;
+                }
+                uint32_t slot = scan - cnt;
+                int stop = 0;
                 if (lane == 0) {
-                    if (i >= dc) ok = mbar_wait_or_abort(&c_empty[s], (uint32_t(i / dc) & 1u) ^ 1u, T, abort_flag);
+                    bool ok = true;
+                    if (sidx >= dc) ok = mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag);
                     if (!ok) fail(!*abort_flag);
                     stop = !ok || *abort_flag;
                 }
                 if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
-                uint8_t *st = cring + size_t(s) * kCStage;
+                uint8_t *st = cring + size_t(cs) * kCStage;
                 if (lane == 0) {
-                    masks[4 * s + 0] = m0;
-                    masks[4 * s + 1] = m1;
-                    masks[4 * s + 2] = m2;
-                    masks[4 * s + 3] = m3;
-                    const uint32_t tile_bytes = HUFF ? uint32_t(kTileSM) : uint32_t(kTileSM + kTilePL);
-                    mbar_arrive_expect_tx(&c_full[s], tile_bytes + uint32_t(kGroup) * nraw);
-                    tma_load_2d(st, tmA, ks * kBK, int32_t(n0), &c_full[s]);
-                    if (!HUFF) tma_load_2d(st + kOffPL, tmB, ks * (kBK / 2), int32_t(n0), &c_full[s]);
+                    mbar_expect_tx(&c_full[cs], HUFF ? uint32_t(2 * kBox) : uint32_t(3 * kBox));
+                    const int32_t xb = int32_t(kSuper * ss.j * kBK);   // first sign/mantissa byte of the chunk
+                    tma_load_2d(st + kOffSmA, tmA, xb, int32_t(n0), &c_full[cs]);
+                    tma_load_2d(st + kOffSmB, tmA, xb + 128, int32_t(n0), &c_full[cs]);
+                    if (!HUFF) tma_load_2d(st + kOffNib, tmB, xb / 2, int32_t(n0), &c_full[cs]);
                 }
-                __syncwarp();
+                uint32_t *tab = reinterpret_cast<uint32_t *>(st + kOffTab);
 #pragma unroll
-                for (int j = 0; j < 4; j++)
-                    if ((rawbits >> j) & 1u)
-                        bulk_g2s(st + kOffRAW + (lane + 32 * j) * kGroup, a.rawexp + uint64_t(rank[j]) * kGroup,
-                                 kGroup, &c_full[s]);
-                issued = i + 1;
+                for (int mm = 0; mm < 4; mm++) {
+                    const int r = lane + 32 * mm;
+#pragma unroll
+                    for (int q = 0; q < kSuper; q++) {
+                        uint32_t e = 0u;
+                        if ((rawbits >> (4 * mm + q)) & 1u) {
+                            if (slot < uint32_t(kRawSlots)) {
+                                const uint8_t *src = a.rawexp + uint64_t(rank[4 * mm + q]) * kGroup;
+                                uint8_t *dst = st + kOffRaw + slot * kGroup;
+#pragma unroll
+                                for (int c = 0; c < 4; c++) cp_async16(dst + 16 * c, src + 16 * c);
+                                e = kTabSlot | slot;
+                            } else {
+                                e = kTabRank | rank[4 * mm + q];
+                            }
+                            slot++;
+                        }
+                        tab[r * kSuper + q] = e;
+                    }
+                }
+                mbar_arrive(&c_full[cs]);                 // this lane's table entries are written
+                cp_async_mbar_arrive_noinc(&c_full[cs]);  // ... and, once landed, its raw copies
             }
+            cp_async_wait_all();
             // no copy may still be landing when the CTA exits (after an abort a
             // decoder's arrival may be missing: those waits run out, bounded)
             if (lane == 0)
-                for (int i = max(0, issued - dc); i < issued; i++)
+                for (int i = max(0, sidx - dc); i < sidx; i++)
                     mbar_wait(&c_full[i % dc], uint32_t(i / dc) & 1u, *abort_flag ? T / 64 + 1 : T);
         } else if (lane == 0) {
+            int issued = 0;
             for (int i = 0; i < nu; i++) {
                 const int64_t u = u0 + i;
                 const int64_t t = u / a.S;
@@ -458,6 +498,8 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 ok = mbar_wait_or_abort(&x_full[xs], uint32_t(i / dx) & 1u, T, abort_flag) &&
                      mbar_wait_or_abort(&w_full[ws], uint32_t(i / dw) & 1u, T, abort_flag);
                 if (!ok) break;
+                // X copied through the load/store path: make it visible to the tensor core
+                if (!C::kXByTma) fence_proxy_async_smem();
                 tc_fence_after();
                 const uint32_t sa = smem_addr(wring + size_t(ws) * kTileW);
                 const uint32_t sb = smem_addr(xring + size_t(xs) * C::kX);
@@ -482,26 +524,46 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
         __syncwarp();
     } else if (warp == 2) {
         // ------------------------------------------------------------ X producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < nu; i++) {
-                const int64_t u = u0 + i;
-                const int64_t t = u / a.S;
-                const int ks = int(u - t * a.S);
-                const int64_t m0 = (t % a.TB) * BN;
-                const int s = i % dx;
-                if (i >= dx && !mbar_wait_or_abort(&x_empty[s], (uint32_t(i / dx) & 1u) ^ 1u, T, abort_flag)) {
-                    fail(!*abort_flag);
-                    break;
-                }
-                if (*abort_flag) break;
-                mbar_arrive_expect_tx(&x_full[s], uint32_t(C::kX));   // rows past m read the zero fill
-                tma_load_2d(xring + size_t(s) * C::kX, tmX, ks * kBK, int32_t(m0), &x_full[s]);
-                issued = i + 1;
+        int issued = 0;
+        for (int i = 0; i < nu; i++) {
+            const int64_t u = u0 + i;
+            const int64_t t = u / a.S;
+            const int ks = int(u - t * a.S);
+            const int64_t m0 = (t % a.TB) * BN;
+            const int s = i % dx;
+            int stop = 0;
+            if (lane == 0) {
+                const bool ok =
+                    i < dx || mbar_wait_or_abort(&x_empty[s], (uint32_t(i / dx) & 1u) ^ 1u, T, abort_flag);
+                if (!ok) fail(!*abort_flag);
+                stop = !ok || *abort_flag;
             }
+            if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
+            uint8_t *xst = xring + size_t(s) * C::kX;
+            if constexpr (C::kXByTma) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&x_full[s], uint32_t(C::kX));   // rows past m read the zero fill
+                    tma_load_2d(xst, tmX, ks * kBK, int32_t(m0), &x_full[s]);
+                }
+            } else {
+                // the 128-byte-swizzled K-major tile: 16-byte chunk c of token
+                // row r at r * 128 + 16 * (c ^ (r & 7)); rows past m are zeros
+#pragma unroll
+                for (int idx = lane; idx < BN * 8; idx += 32) {
+                    const int r = idx >> 3, c = idx & 7;
+                    const int64_t tok = m0 + r;
+                    const bool live = tok < a.m;
+                    const uint16_t *src = a.x + (live ? tok * a.k + int64_t(ks) * kBK + c * 8 : 0);
+                    cp_async16_zfill(xst + r * 128 + ((c ^ (r & 7)) << 4), src, live ? 16u : 0u);
+                }
+                cp_async_mbar_arrive_noinc(&x_full[s]);
+            }
+            issued = i + 1;
+        }
+        if constexpr (!C::kXByTma) cp_async_wait_all();
+        if (lane == 0)
             for (int i = max(0, issued - dx); i < issued; i++)
                 mbar_wait(&x_full[i % dx], uint32_t(i / dx) & 1u, T);
-        }
         __syncwarp();
     } else if (warp < kFirstRebuildWarp) {
         // ------------------------------------------------------------ epilogue
@@ -590,51 +652,75 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
         }
     } else if (warp < kStreamWarp) {
         if constexpr (FUSED) {
-        // ------------------------------------------------------------ rebuild
-        const int tid = threadIdx.x - 32 * kFirstRebuildWarp;   // 0..255
-        const int r = tid >> 1, h = tid & 1;
-        const int sw64 = (r >> 1) & 3, sw32 = (r >> 2) & 1, sw128 = r & 7;
-        const Palette16 P = a.pal;
-        for (int i = 0; i < nu; i++) {
-            const int cs = i % dc, ws = i % dw;
-            bool ok = mbar_wait_or_abort(&c_full[cs], uint32_t(i / dc) & 1u, T, abort_flag);
-            if (ok && i >= dw) ok = mbar_wait_or_abort(&w_empty[ws], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag);
-            if (__any_sync(0xFFFFFFFFu, !ok)) {
-                if (lane == 0 && !*abort_flag) fail(true);
-                break;
+            // -------------------------------------------------------- rebuild
+            const int wi = warp - kFirstRebuildWarp;   // 0..7
+            const int R = 16 * wi + 8 * (lane >> 4) + (lane & 7);   // tile row
+            const int h = (lane >> 3) & 1;                          // half of the row's 64 weights
+            const int sw = R & 7;                                   // 128-byte swizzle phase of the row
+            const Palette16 P = a.pal;
+            int i = 0, sidx = 0;
+            bool ok = true;
+            for (SuperSteps ss(u0, u1, a.S); ss.valid() && ok; ss.next(), sidx++) {
+                const int cs = sidx % dc;
+                ok = mbar_wait_or_abort(&c_full[cs], uint32_t(sidx / dc) & 1u, T, abort_flag);
+                if (__any_sync(0xFFFFFFFFu, !ok)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *st = cring + size_t(cs) * kCStage;
+                const uint32_t *tab = reinterpret_cast<const uint32_t *>(st + kOffTab);
+                for (int ks = ss.lo(); ks < ss.hi(); ks++, i++) {
+                    const int q = ks - kSuper * ss.j;
+                    const int ws = i % dw;
+                    if (i >= dw) ok = mbar_wait_or_abort(&w_empty[ws], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag);
+                    if (__any_sync(0xFFFFFFFFu, !ok)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *smrow = st + (q >> 1) * kBox + R * 128;
+                    const int c0 = (q & 1) * 4 + 2 * h;
+                    const uint4 s0 = *reinterpret_cast<const uint4 *>(smrow + ((c0 ^ sw) << 4));
+                    const uint4 s1 = *reinterpret_cast<const uint4 *>(smrow + (((c0 + 1) ^ sw) << 4));
+                    const uint32_t e = tab[R * kSuper + q];
+                    uint32_t rv[8];
+                    if (e == 0u) {
+                        const uint4 p = *reinterpret_cast<const uint4 *>(st + kOffNib + R * 128 +
+                                                                         (((2 * q + h) ^ sw) << 4));
+                        pal_rot(p.x, P, rv[0], rv[1]);
+                        pal_rot(p.y, P, rv[2], rv[3]);
+                        pal_rot(p.z, P, rv[4], rv[5]);
+                        pal_rot(p.w, P, rv[6], rv[7]);
+                    } else {
+                        uint4 e0, e1;
+                        if (e & kTabSlot) {
+                            const uint8_t *rp = st + kOffRaw + (e & 0xFFFFu) * kGroup + h * 32;
+                            e0 = *reinterpret_cast<const uint4 *>(rp);
+                            e1 = *reinterpret_cast<const uint4 *>(rp + 16);
+                        } else {   // no slot was left: the raw plane itself
+                            const uint4 *rp = reinterpret_cast<const uint4 *>(
+                                a.rawexp + uint64_t(e & ~kTabRank) * kGroup + h * 32);
+                            e0 = __ldg(rp);
+                            e1 = __ldg(rp + 1);
+                        }
+                        rv[0] = rot4(e0.x); rv[1] = rot4(e0.y); rv[2] = rot4(e0.z); rv[3] = rot4(e0.w);
+                        rv[4] = rot4(e1.x); rv[5] = rot4(e1.y); rv[6] = rot4(e1.z); rv[7] = rot4(e1.w);
+                    }
+                    uint8_t *wrow = wring + size_t(ws) * kTileW + R * 128;
+                    const int w0 = 4 * h;
+                    *reinterpret_cast<uint4 *>(wrow + (((w0 + 0) ^ sw) << 4)) = join8(rv[0], rv[1], s0.x, s0.y);
+                    *reinterpret_cast<uint4 *>(wrow + (((w0 + 1) ^ sw) << 4)) = join8(rv[2], rv[3], s0.z, s0.w);
+                    *reinterpret_cast<uint4 *>(wrow + (((w0 + 2) ^ sw) << 4)) = join8(rv[4], rv[5], s1.x, s1.y);
+                    *reinterpret_cast<uint4 *>(wrow + (((w0 + 3) ^ sw) << 4)) = join8(rv[6], rv[7], s1.z, s1.w);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&w_full[ws]);
+                }
+                if (!ok) break;
+                // every K-step of the stage is rebuilt: hand it back to the producer
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[cs]);
             }
-            const uint8_t *st = cring + size_t(cs) * kCStage;
-            const bool raw = (masks[4 * cs + (r >> 5)] >> (r & 31)) & 1u;
-            const uint8_t *smrow = st + r * 64;
-            const uint4 s0 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h) ^ sw64) << 4));
-            const uint4 s1 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h + 1) ^ sw64) << 4));
-            uint32_t rv[8];
-            if (raw) {
-                const uint8_t *rp = st + kOffRAW + r * kGroup + h * 32;
-                const uint4 e0 = *reinterpret_cast<const uint4 *>(rp);
-                const uint4 e1 = *reinterpret_cast<const uint4 *>(rp + 16);
-                rv[0] = rot4(e0.x); rv[1] = rot4(e0.y); rv[2] = rot4(e0.z); rv[3] = rot4(e0.w);
-                rv[4] = rot4(e1.x); rv[5] = rot4(e1.y); rv[6] = rot4(e1.z); rv[7] = rot4(e1.w);
-            } else {
-                const uint4 p = *reinterpret_cast<const uint4 *>(st + kOffPL + r * 32 + ((h ^ sw32) << 4));
-                pal_rot(p.x, P, rv[0], rv[1]);
-                pal_rot(p.y, P, rv[2], rv[3]);
-                pal_rot(p.z, P, rv[4], rv[5]);
-                pal_rot(p.w, P, rv[6], rv[7]);
-            }
-            // the stage's bytes are all in registers: hand it back to the producer
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&c_empty[cs]);
-            uint8_t *wrow = wring + size_t(ws) * kTileW + r * 128;
-            const int c0 = 4 * h;
-            *reinterpret_cast<uint4 *>(wrow + (((c0 + 0) ^ sw128) << 4)) = join8(rv[0], rv[1], s0.x, s0.y);
-            *reinterpret_cast<uint4 *>(wrow + (((c0 + 1) ^ sw128) << 4)) = join8(rv[2], rv[3], s0.z, s0.w);
-            *reinterpret_cast<uint4 *>(wrow + (((c0 + 2) ^ sw128) << 4)) = join8(rv[4], rv[5], s1.x, s1.y);
-            *reinterpret_cast<uint4 *>(wrow + (((c0 + 3) ^ sw128) << 4)) = join8(rv[6], rv[7], s1.z, s1.w);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&w_full[ws]);
-        }
+            if (!ok && lane == 0 && !*abort_flag) fail(true);
         }
     } else if (warp == kStreamWarp) {
         if constexpr (HUFF) {
@@ -643,7 +729,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 mbar_arrive_expect_tx(lut_full, uint32_t(kHuffLut));
                 bulk_g2s(hlut, a.dlut, kHuffLut, lut_full);
             }
-            const int64_t G4 = a.k / (4 * kGroup);      // chunks per row
+            const int64_t G4 = a.k / (kSuper * kGroup);   // chunks per row
             int sidx = 0;
             for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
                 const int slot = sidx % kSlots;
@@ -666,7 +752,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                         const int64_t c = row * G4 + ss.j;
                         start[mm] = __ldg(a.chunk_off + c);
                         end[mm] = __ldg(a.chunk_off + c + 1);
-                        const int64_t g = 4 * c;
+                        const int64_t g = int64_t(kSuper) * c;
                         raw4[mm] = (__ldg(a.flagbits + (g >> 5)) >> (uint32_t(g) & 31u)) & 15u;
                     }
                 }
@@ -679,7 +765,9 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     if (sane && end[mm] > start[mm]) {
                         wfirst[mm] = (start[mm] >> 5) & ~3u;
                         const uint32_t wlast = ((end[mm] + 31u) >> 5) + 2u;
-                        bytes[mm] = ((wlast - wfirst[mm] + 3u) & ~3u) * 4u;
+                        const uint32_t nw = (wlast - wfirst[mm] + 3u) & ~3u;
+                        // words past the stream section are never staged (those chunks read global memory)
+                        bytes[mm] = uint64_t(wfirst[mm]) + nw <= a.stream_words ? nw * 4u : 0u;
                     }
                     incl += bytes[mm];
                 }
@@ -690,30 +778,24 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, scan, d);
                     if (lane >= d) scan += v;
                 }
-                uint32_t off = scan - incl, staged = 0;
+                uint32_t off = scan - incl;
                 uint4 *tab = htable + slot * kBM;
+                uint8_t *sbase = hslots + slot * kSlotBytes;
 #pragma unroll
                 for (int mm = 0; mm < 4; mm++) {
                     const int r = lane + 32 * mm;
                     const bool fits = bytes[mm] > 0 && off + bytes[mm] <= uint32_t(kSlotBytes);
                     tab[r] = make_uint4(fits ? off : kFromGlobal, wfirst[mm], start[mm], end[mm]);
                     hraw4[slot * kBM + r] = uint8_t(raw4[mm]);
-                    if (fits) staged += bytes[mm];
+                    if (fits)
+                        for (uint32_t b = 0; b < bytes[mm]; b += 16)
+                            cp_async16(sbase + off + b, reinterpret_cast<const uint8_t *>(a.stream + wfirst[mm]) + b);
                     off += bytes[mm];
                 }
-                const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, staged);
-                if (lane == 0) mbar_arrive_expect_tx(&s_full[slot], total);
-                __syncwarp();
-                if (lane != 0) mbar_arrive(&s_full[slot]);
-                off = scan - incl;
-                uint8_t *sbase = hslots + slot * kSlotBytes;
-#pragma unroll
-                for (int mm = 0; mm < 4; mm++) {
-                    if (bytes[mm] > 0 && off + bytes[mm] <= uint32_t(kSlotBytes))
-                        bulk_g2s(sbase + off, a.stream + wfirst[mm], bytes[mm], &s_full[slot]);
-                    off += bytes[mm];
-                }
+                mbar_arrive(&s_full[slot]);                 // this lane's table entries are written
+                cp_async_mbar_arrive_noinc(&s_full[slot]);  // ... and, once landed, its stream words
             }
+            cp_async_wait_all();
             // no copy may still be landing when the CTA exits
             if (lane == 0) {
                 for (int i = max(0, sidx - kSlots); i < sidx; i++)
@@ -728,14 +810,14 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             const int dt = threadIdx.x - 32 * kFirstDecWarp;   // 0..255
             const int grp = dt >> 7, r = dt & 127;
             const uint32_t lut = smem_addr(hlut);
-            const uint32_t line = smem_addr(hscratch) + uint32_t(dt * kScratchStride);
-            const int sw32 = (r >> 2) & 1;
+            const int sw = r & 7;
             bool ok = mbar_wait_or_abort(lut_full, 0, T, abort_flag);
             int sidx = 0;
             for (SuperSteps ss(u0, u1, a.S); ss.valid() && ok; ss.next(), sidx++) {
                 if ((sidx & 1) != grp) continue;
-                const int slot = sidx % kSlots;
-                ok = mbar_wait_or_abort(&s_full[slot], uint32_t(sidx / kSlots) & 1u, T, abort_flag);
+                const int slot = sidx % kSlots, cs = sidx % dc;
+                ok = mbar_wait_or_abort(&s_full[slot], uint32_t(sidx / kSlots) & 1u, T, abort_flag) &&
+                     (sidx < dc || mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag));
                 if (__any_sync(0xFFFFFFFFu, !ok)) {
                     ok = false;
                     break;
@@ -750,37 +832,28 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 const uint32_t wfirst = e.y;
                 const auto staged = [&](uint32_t wi) { return lds32(sbase + 4u * (wi - wfirst)); };
                 const auto global = [&](uint32_t wi) { return __ldg(a.stream + wi); };
+                const uint32_t nib = smem_addr(cring + size_t(cs) * kCStage + kOffNib) + uint32_t(r * 128);
+                if (row < a.n) {
 #pragma unroll 1
-                for (int q = 0; q < 4; q++) {
-                    const int ks = 4 * ss.j + q;
-                    const bool raw = (raw4 >> q) & 1u;
-                    if (row < a.n && !raw && good)
-                        good = (e.x & kFromGlobal) ? decode_group(global, p, end, lut, line, a.code_len)
-                                                   : decode_group(staged, p, end, lut, line, a.code_len);
-                    if (ks < ss.ka || ks >= ss.kb) continue;   // a K-step another CTA owns (uniform)
-                    const int i = int(ss.t * a.S + ks - u0);
-                    const int cs = i % dc;
-                    ok = i < dc || mbar_wait_or_abort(&c_empty[cs], (uint32_t(i / dc) & 1u) ^ 1u, T, abort_flag);
-                    if (__any_sync(0xFFFFFFFFu, !ok)) {
-                        ok = false;
-                        break;
+                    for (int q = 0; q < kSuper; q++) {
+                        if ((raw4 >> q) & 1u) continue;   // no codes in the stream for a raw group
+                        // word w of group q: weights 8w..8w+7 of K-step q, in the
+                        // stored 4-bit layout at the swizzled palette position
+                        const auto sink = [&](uint32_t w, uint32_t v) {
+                            sts32(nib + ((((2 * q) + (w >> 2)) ^ sw) << 4) + 4u * (w & 3u), natural_to_pal(v));
+                        };
+                        if (good)
+                            good = (e.x & kFromGlobal) ? decode_group(global, p, end, lut, a.code_len, sink)
+                                                       : decode_group(staged, p, end, lut, a.code_len, sink);
                     }
-                    if (row < a.n && !raw) {
-                        uint32_t wv[8];
-#pragma unroll
-                        for (int w = 0; w < 8; w++) wv[w] = good ? natural_to_pal(lds32(line + 4u * w)) : 0u;
-                        uint8_t *pl = cring + size_t(cs) * kCStage + kOffPL + r * 32;
-                        *reinterpret_cast<uint4 *>(pl + (sw32 << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                        *reinterpret_cast<uint4 *>(pl + ((1 ^ sw32) << 4)) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&c_full[cs]);
+                    // a chunk must decode cleanly and end exactly where the next starts
+                    if (!good || p != end) flag_error(a.status, UW_DEVERR_CORRUPT);
                 }
-                if (!ok) break;
-                // a chunk must decode cleanly and end exactly where the next starts
-                if (row < a.n && (!good || p != end)) flag_error(a.status, UW_DEVERR_CORRUPT);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[slot]);
+                if (lane == 0) {
+                    mbar_arrive(&c_full[cs]);
+                    mbar_arrive(&s_empty[slot]);
+                }
             }
             if (!ok && lane == 0 && !*abort_flag) fail(true);
         }
@@ -829,33 +902,36 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// ring depths per token tile (compressed depth for the fused flavours is the
-// largest that fits, at most 6, unless the plan asks for fewer)
+// ring depths: compressed super-steps (2 when it fits), W tiles and X tiles
+// per token tile; the plan's `stages` caps the compressed ring (fused) or the
+// W ring (plain)
 struct Depths {
     int dc, dw, dx;
 };
 Depths depths(int mode, int bn, int stages) {
     const int kx = bn * kBK * 2;
     Depths d{};
-    if (mode == kModePal) {
-        d.dw = bn <= 128 ? 3 : 2;
-        d.dx = bn <= 64 ? 4 : (bn == 128 ? 3 : 2);
-        const int room = kMaxSmem - 1024 - d.dw * kTileW - d.dx * kx - sk_tail(8, d.dw, d.dx);
-        d.dc = std::min(6, room / kCStage);
-        if (stages > 0) d.dc = std::min(d.dc, stages);
-    } else if (mode == kModeHuff) {
-        d.dw = 2;
-        d.dx = bn <= 64 ? 3 : 2;
-        const int room = kMaxSmem - 1024 - d.dw * kTileW - d.dx * kx - kHuffBytes - sk_tail(8, d.dw, d.dx);
-        d.dc = std::min(6, room / kCStage);
-        if (stages > 0) d.dc = std::min(d.dc, stages);
-    } else {
+    if (mode == kModePlain) {
         d.dc = 0;
-        d.dx = bn <= 64 ? 6 : (bn == 128 ? 4 : 3);
+        d.dx = bn <= 64 ? 8 : (bn == 128 ? 4 : 3);
         const int room = kMaxSmem - 1024 - d.dx * kx - sk_tail(0, 8, d.dx);
         d.dw = std::min(8, room / kTileW);
         if (stages > 0) d.dw = std::min(d.dw, std::max(2, stages));
+        return d;
     }
+    const int huff = mode == kModeHuff ? kHuffBytes : 0;
+    d.dc = 2;
+    d.dw = bn <= 64 && mode == kModePal ? 3 : 2;
+    int room = kMaxSmem - 1024 - d.dc * kCStage - huff - d.dw * kTileW - sk_tail(3, d.dw, 8);
+    d.dx = std::min(8, room / kx);
+    if (d.dx > 2) {   // a third compressed stage when X keeps at least 2 stages
+        room -= kCStage;
+        if (room / kx >= 2) {
+            d.dc = 3;
+            d.dx = std::min(8, room / kx);
+        }
+    }
+    if (stages > 0) d.dc = std::min(d.dc, std::max(2, stages));
     return d;
 }
 
@@ -929,14 +1005,16 @@ cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
     a.dx = d.dx;
     a.debug_flags = p.debug_flags;
     a.timeout_ns = p.timeout_ns;
+    a.x = p.x;
     a.y = p.y;
     a.counters = p.sk_counters;
     a.partial = p.partial;
     a.status = p.dev_status;
 
     CUtensorMap mx, ma, mb;
-    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2, kBK,
-                  BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    std::memset(&mx, 0, sizeof(mx));
+    if (C::kXByTma && !make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m),
+                                uint64_t(p.k) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     cudaError_t err;
     if (mode != kModePlain) {
@@ -945,13 +1023,15 @@ cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
         a.rawexp = p.w->rawexp;
         a.nflag = (p.n * (p.k / kGroup) + 31) / 32;
         a.pal = make_palette16(p.w->palette);
-        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k), kBK,
-                      kBM, CU_TENSOR_MAP_SWIZZLE_64B))
+        // sign/mantissa boxes of 128 bytes (two K-steps) x 128 rows
+        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k), 128,
+                      kBM, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
     if (mode == kModePal) {
+        // palette boxes of 128 bytes (four K-steps) x 128 rows
         if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n), uint64_t(p.k / 2),
-                      kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
+                      128, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         static int ready[64] = {0};
         err = prepare(k_gemm_sk_fused<BN>, kPalThreads, C::kTmemCols, ready);
@@ -960,20 +1040,18 @@ cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
     } else if (mode == kModeHuff) {
         // chunks of 4 groups must not straddle rows; the decoders' table
         // needs the Huffman sections
-        if (BN > 128 || p.k % (4 * kGroup) || !p.w->stream || !p.w->chunk_off || !p.w->dlut)
-            return cudaErrorInvalidValue;
+        if (p.k % (kSuper * kGroup) || !p.w->stream || !p.w->chunk_off || !p.w->dlut) return cudaErrorInvalidValue;
         a.stream = p.w->stream;
         a.chunk_off = p.w->chunk_off;
         a.dlut = p.w->dlut;
         a.stream_bits = p.w->stream_bits;
+        a.stream_words = p.w->stream_words;
         a.code_len = 0;
         for (int i = 0; i < 16; i++) a.code_len |= uint64_t(p.w->code_len[i] & 15u) << (4 * i);
-        if constexpr (BN <= 128) {
-            static int ready[64] = {0};
-            err = prepare(k_gemm_sk_huff<BN>, kHuffThreads, C::kTmemCols, ready);
-            if (err != cudaSuccess) return err;
-            k_gemm_sk_huff<BN><<<unsigned(g.G), kHuffThreads, smem, stream>>>(mx, ma, a);
-        }
+        static int ready[64] = {0};
+        err = prepare(k_gemm_sk_huff<BN>, kHuffThreads, C::kTmemCols, ready);
+        if (err != cudaSuccess) return err;
+        k_gemm_sk_huff<BN><<<unsigned(g.G), kHuffThreads, smem, stream>>>(mx, ma, a);
     } else {
         if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.w_bf16, uint64_t(p.k), uint64_t(p.n),
                       uint64_t(p.k) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -1002,7 +1080,17 @@ SkGeometry sk_geometry(int64_t m, int64_t n, int64_t k, int bn) {
     return g;
 }
 
+int sk_huffman_max_bn() {
+    // the largest token tile whose Huffman kernel fits shared memory
+    for (int bn : {256, 128, 64, 32, 16}) {
+        const Depths d = depths(kModeHuff, bn, 0);
+        if (d.dc >= 2 && d.dx >= 2 && smem_bytes(kModeHuff, bn, d) <= size_t(kMaxSmem)) return bn;
+    }
+    return 0;
+}
+
 cudaError_t launch_gemm_sk(const TcLaunch &p, cudaStream_t stream) {
+    if (p.huffman && p.bn > sk_huffman_max_bn()) return cudaErrorInvalidValue;
     switch (p.bn) {
         case 16: return launch_bn<16>(p, stream);
         case 32: return launch_bn<32>(p, stream);

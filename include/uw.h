@@ -11,7 +11,8 @@
  *        palette is stored raw, so the hot loop needs no per-element branch.
  *   §五  decompress next to the compute, never back to HBM, to save bandwidth.
  *   §六  four pipelines: full decode + GEMM, exponent-only decode, runtime
- *        Huffman -> 4-bit palette transcode, and pre-transcoded palette.
+ *        Huffman -> 4-bit palette transcode, and pre-transcoded palette; here
+ *        also a fifth, the runtime transcode done inside the matmul kernel.
  *   §七  reconstructive matmul: compressed tiles are staged into shared memory,
  *        rebuilt to BF16 there and fed straight to the tensor cores.
  *   §九  an autotuner measures the pipelines, the kernel variants and the
@@ -201,7 +202,7 @@ typedef enum uw_pipeline {
                                      palette indices in shared memory as it goes (pipeline 3's
                                      transcode inside the matmul's producer): no preprocessing
                                      pass and no workspace beyond the stream-K scratch.  Needs
-                                     UW_EMIT_HUFFMAN, kernel UW_KERNEL_TC_SK with bn <= 128 and
+                                     UW_EMIT_HUFFMAN, kernel UW_KERNEL_TC_SK with bn <= 64 and
                                      k a multiple of 256 (a 4-group stream chunk never
                                      straddles two rows); UW_ERR_INVALID_ARG otherwise       */
 } uw_pipeline;
