@@ -27,7 +27,7 @@ uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
         p->pipeline != UW_PIPE_TRANSCODE_FUSED && p->pipeline != UW_PIPE_DIRECT_PALETTE &&
         p->pipeline != UW_PIPE_HUFFMAN_FUSED)
         return UW_ERR_INVALID_ARG;
-    if (p->pipeline == UW_PIPE_HUFFMAN_FUSED && (p->kernel != UW_KERNEL_TC_SK || p->bn > 64 || k % 256))
+    if (p->pipeline == UW_PIPE_HUFFMAN_FUSED && (p->kernel != UW_KERNEL_TC_SK || p->bn > 32 || k % 256))
         return UW_ERR_INVALID_ARG;
     if (p->kernel == UW_KERNEL_FMA) {
         if (m > 8 || (p->bn != 1 && p->bn != 2) || p->split_k != 1) return UW_ERR_INVALID_ARG;

@@ -84,7 +84,7 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
             out.push_back(p);
             // the same kernel decoding the Huffman stream itself (pipeline 3's
             // transcode moved into the matmul)
-            if (pipe == UW_PIPE_TRANSCODE_FUSED && bn <= 64 && w.k % 256 == 0) {
+            if (pipe == UW_PIPE_TRANSCODE_FUSED && bn <= 32 && w.k % 256 == 0) {
                 p.pipeline = UW_PIPE_HUFFMAN_FUSED;
                 out.push_back(p);
             }

@@ -85,15 +85,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     return true;
 }
 
-// Potentially blocking test: the thread may be suspended in hardware until
-// the phase completes or a system-defined time slice ends, so waiting warps
-// take few issue slots from the working ones.
-__device__ __forceinline__ bool mbar_try_wait_susp(uint64_t *bar, uint32_t parity) {
+// Potentially blocking test: the thread is suspended in hardware until the
+// phase completes or about `hint_ns` pass, so a parked warp takes no issue
+// slots from the working ones (a spinning test loop of a dozen parked warps
+// measurably slows the producer, MMA and rebuild warps of the same SM).
+__device__ __forceinline__ bool mbar_try_wait_susp(uint64_t *bar, uint32_t parity, uint32_t hint_ns = 100000u) {
     uint32_t ok;
     asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }

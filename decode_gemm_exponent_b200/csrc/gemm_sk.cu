@@ -112,7 +112,8 @@ constexpr uint32_t kTabSlot = 0x80000000u, kTabRank = 0x40000000u;
 
 // Huffman flavour
 constexpr int kSlots = 3;                        // stream slots (super-steps staged ahead)
-constexpr int kSlotBytes = 12 * 1024;            // stream bytes per slot (~85 B per chunk at 2.6 bits/weight)
+constexpr int kSlotBytes = 15 * 1024;            // stream bytes per slot: 128 chunks of ~100 B (2.6 bits/weight
+                                                 // and the 16-byte granules around each chunk)
 constexpr uint32_t kFromGlobal = 0x80000000u;    // chunk table flag: read the words from global memory
 constexpr int kHuffLut = kLutEntries * 4;
 constexpr int kHuffTable = kSlots * kBM * 16;    // per slot and row: uint4 {where, first word, start, end}
@@ -211,6 +212,19 @@ struct SuperSteps {
         if (++j > j_last) {
             ++t;
             if (t <= t_last) start_tile();
+        }
+    }
+};
+
+// The CTA's units in order as (tile, K-step), advanced without divisions.
+struct UnitWalk {
+    int64_t t;
+    int ks, S;
+    __device__ __forceinline__ UnitWalk(int64_t u0, int S_) : t(u0 / S_), ks(int(u0 % S_)), S(S_) {}
+    __device__ __forceinline__ void next() {
+        if (++ks == S) {
+            ks = 0;
+            ++t;
         }
     }
 };
@@ -453,11 +467,14 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     mbar_wait(&c_full[i % dc], uint32_t(i / dc) & 1u, *abort_flag ? T / 64 + 1 : T);
         } else if (lane == 0) {
             int issued = 0;
-            for (int i = 0; i < nu; i++) {
-                const int64_t u = u0 + i;
-                const int64_t t = u / a.S;
-                const int ks = int(u - t * a.S);
-                const int64_t n0 = (t / a.TB) * kBM;
+            UnitWalk walk(u0, a.S);
+            int64_t tcur = -1, n0 = 0;
+            for (int i = 0; i < nu; i++, walk.next()) {
+                if (walk.t != tcur) {
+                    tcur = walk.t;
+                    n0 = (tcur / a.TB) * kBM;
+                }
+                const int ks = walk.ks;
                 const int s = i % dw;
                 if (i >= dw && !mbar_wait_or_abort(&w_empty[s], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag)) {
                     fail(!*abort_flag);
@@ -481,9 +498,9 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             int seg = -1;
             int64_t tprev = -1;
             bool first = true;
-            for (int i = 0; i < nu && ok; i++) {
-                const int64_t u = u0 + i;
-                const int64_t t = u / a.S;
+            UnitWalk walk(u0, a.S);
+            for (int i = 0; i < nu && ok; i++, walk.next()) {
+                const int64_t t = walk.t;
                 if (t != tprev) {   // a new tile: close the previous accumulator, claim the next
                     if (seg >= 0) tc_commit(&acc_full[seg & 1]);
                     seg++;
@@ -525,11 +542,14 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
     } else if (warp == 2) {
         // ------------------------------------------------------------ X producer
         int issued = 0;
-        for (int i = 0; i < nu; i++) {
-            const int64_t u = u0 + i;
-            const int64_t t = u / a.S;
-            const int ks = int(u - t * a.S);
-            const int64_t m0 = (t % a.TB) * BN;
+        UnitWalk walk(u0, a.S);
+        int64_t tcur = -1, m0 = 0;
+        for (int i = 0; i < nu; i++, walk.next()) {
+            if (walk.t != tcur) {
+                tcur = walk.t;
+                m0 = (tcur % a.TB) * BN;
+            }
+            const int ks = walk.ks;
             const int s = i % dx;
             int stop = 0;
             if (lane == 0) {
@@ -764,7 +784,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     const bool sane = start[mm] <= end[mm] && uint64_t(end[mm]) <= a.stream_bits;
                     if (sane && end[mm] > start[mm]) {
                         wfirst[mm] = (start[mm] >> 5) & ~3u;
-                        const uint32_t wlast = ((end[mm] + 31u) >> 5) + 2u;
+                        const uint32_t wlast = (end[mm] >> 5) + 2u;   // a window at bit p <= end reads words p/32, p/32 + 1
                         const uint32_t nw = (wlast - wfirst[mm] + 3u) & ~3u;
                         // words past the stream section are never staged (those chunks read global memory)
                         bytes[mm] = uint64_t(wfirst[mm]) + nw <= a.stream_words ? nw * 4u : 0u;

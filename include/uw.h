@@ -202,7 +202,7 @@ typedef enum uw_pipeline {
                                      palette indices in shared memory as it goes (pipeline 3's
                                      transcode inside the matmul's producer): no preprocessing
                                      pass and no workspace beyond the stream-K scratch.  Needs
-                                     UW_EMIT_HUFFMAN, kernel UW_KERNEL_TC_SK with bn <= 64 and
+                                     UW_EMIT_HUFFMAN, kernel UW_KERNEL_TC_SK with bn <= 32 and
                                      k a multiple of 256 (a 4-group stream chunk never
                                      straddles two rows); UW_ERR_INVALID_ARG otherwise       */
 } uw_pipeline;

@@ -50,7 +50,7 @@ def sk_case(uw, n, k, m, bn, seed=0, frac=0.002, pipelines=(1, 2, 3, 4, 5), stag
     kw = dict(kernel=uw.KERNEL_TC_SK, bn=bn, split_k=1, stages=stages)
     y_plain = uw.matmul_bf16(xd, wd, uw.make_plan(pipeline=4, **kw)).cpu().numpy()
     for pipe in pipelines:
-        if pipe == uw.PIPE_HUFFMAN_FUSED and (bn > 64 or k % 256):
+        if pipe == uw.PIPE_HUFFMAN_FUSED and (bn > 32 or k % 256):
             continue
         y = mat.matmul(xd, uw.make_plan(pipeline=pipe, **kw)).cpu().numpy()
         assert np.array_equal(y.view(np.uint32), y_plain.view(np.uint32)), "pipeline %d differs" % pipe
@@ -90,7 +90,7 @@ def test_sk_huffman_chunks_larger_than_a_stream_slot(uw):
     sm = rng.integers(0, 256, n * k).astype(np.uint16)
     w = (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16).reshape(n, k)
     sk_case(uw, n, k, 16, 16, seed=22, pipelines=(4, 5), w=w)
-    sk_case(uw, n, k, 100, 64, seed=23, pipelines=(5,), w=w)
+    sk_case(uw, n, k, 100, 32, seed=23, pipelines=(5,), w=w)
 
 
 def test_sk_huffman_corrupt_stream_is_reported(uw):
@@ -121,7 +121,7 @@ def test_sk_huffman_plan_checks(uw):
         assert e.value.status == 1
     w1 = synth.weights_bf16(128, 1024, 0.02, 0.0, 1.0, seed=27)
     mat1 = uw.Matrix(uw.encode(w1))
-    for kw in (dict(kernel=uw.KERNEL_TC_SK, bn=128),):     # the Huffman kernel's token tiles stop at 64
+    for kw in (dict(kernel=uw.KERNEL_TC_SK, bn=64),):      # the Huffman kernel's token tiles stop at 32
         with pytest.raises(uw.UwError) as e:
             mat1.matmul(dev16(synth.activations_bf16(4, 1024, seed=27)),
                         uw.make_plan(pipeline=uw.PIPE_HUFFMAN_FUSED, split_k=1, **kw))
@@ -228,7 +228,7 @@ def test_sk_full_size_8b_sampled(uw, m, bn, proj):
     xd, wd = dev16(x), dev16(w)
     kw = dict(kernel=uw.KERNEL_TC_SK, bn=bn, split_k=1)
     yp = uw.matmul_bf16(xd, wd, uw.make_plan(pipeline=4, **kw)).cpu().numpy()
-    for pipe in ((4, 2, 5) if bn <= 64 else (4, 2)):
+    for pipe in ((4, 2, 5) if bn <= 32 else (4, 2)):
         yf = mat.matmul(xd, uw.make_plan(pipeline=pipe, **kw)).cpu().numpy()
         assert np.array_equal(yf.view(np.uint32), yp.view(np.uint32)), "pipeline %d" % pipe
     assert mat.device_status() == 0
