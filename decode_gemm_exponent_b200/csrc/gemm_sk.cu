@@ -34,13 +34,8 @@
 // stream words -- go through the load/store path (cp.async, 16 bytes a lane).
 //
 // Roles (warps):
-//   0      producer: per super-step the TMA boxes (W tiles for the plain
-//          flavour: one 16 KB box per K-step) and, in the fused flavours, the
-//          super-step's raw groups: the 32 lanes find the raw (row, group)
-//          pairs of the 128 rows, give each a slot in the stage (cp.async of
-//          its 64 exponents) and write a 128 x 4 table that tells the rebuild
-//          where each group's exponents are (palette plane, a slot, or, when
-//          the slots run out, the raw plane in global memory).
+//   0      TMA producer: per super-step the compressed boxes (plain flavour:
+//          one 16 KB W box per K-step).
 //   1      MMA issuer and TMEM owner: 4 x tcgen05.mma (K = 16) per K-step into
 //          one of two accumulators (double-buffered, so the epilogue of one
 //          tile overlaps the MMAs of the next).
@@ -53,11 +48,16 @@
 //          K-major BF16 W tile.  A quarter warp covers 8 consecutive rows, so
 //          under the 128-byte swizzle every 16-byte shared-memory access of
 //          it falls on its own bank group.
-//   15     (Huffman) stream producer: per super-step it reads the 128 chunks'
+//   15     (fused) raw groups: per super-step the 32 lanes find the raw (row,
+//          group) pairs of the 128 rows, give each a slot in the stage
+//          (cp.async of its 64 exponents) and write a 128 x 4 table that tells
+//          the rebuild where each group's exponents are (palette plane, a
+//          slot, or, when the slots run out, the raw plane in global memory).
+//   16     (Huffman) stream producer: per super-step it reads the 128 chunks'
 //          start bits and copies each chunk's stream words (cp.async) into
 //          one slot of a shared-memory ring, with a table of where they are
 //          (a chunk that does not fit is read from global memory instead).
-//   16-23  (Huffman) decoders: two groups of 4 warps take alternate
+//   17-24  (Huffman) decoders: two groups of 4 warps take alternate
 //          super-steps, one thread per tile row; a thread decodes its row's
 //          chunk with the 12-bit multi-symbol table straight into the
 //          super-step's palette area, in the stored 4-bit layout.
@@ -87,12 +87,13 @@ constexpr int kFixedWarps = 7;          // producer, MMA, X producer, 4 epilogue
 constexpr int kRebuildWarps = 8;
 constexpr int kEpiWarp0 = 3;
 constexpr int kFirstRebuildWarp = kFixedWarps;
-constexpr int kStreamWarp = kFixedWarps + kRebuildWarps;   // Huffman flavour
+constexpr int kRawWarp = kFixedWarps + kRebuildWarps;      // fused flavours
+constexpr int kStreamWarp = kRawWarp + 1;                  // Huffman flavour
 constexpr int kFirstDecWarp = kStreamWarp + 1;
 constexpr int kDecWarps = 8;            // two groups of 4
 constexpr int kPlainThreads = kFixedWarps * 32;
-constexpr int kPalThreads = (kFixedWarps + kRebuildWarps) * 32;
-constexpr int kHuffThreads = (kFixedWarps + kRebuildWarps + 1 + kDecWarps) * 32;
+constexpr int kPalThreads = (kFixedWarps + kRebuildWarps + 1) * 32;
+constexpr int kHuffThreads = (kFixedWarps + kRebuildWarps + 2 + kDecWarps) * 32;
 
 constexpr int kTileW = kBM * kBK * 2;   // BF16 W tile of one K-step (128 rows x 128 B)
 
@@ -323,9 +324,10 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < dc; s++) {
-            // 32 producer lanes once their table entries are written, 32 once
-            // their cp.async copies landed, + the 4 decoder warps of a group
-            mbar_init(&c_full[s], HUFF ? 64 + 4 : 64);
+            // the TMA producer, the 32 raw-group lanes once their table entries
+            // are written and 32 once their copies landed, + the 4 decoder
+            // warps of a group
+            mbar_init(&c_full[s], HUFF ? 1 + 64 + 4 : 1 + 64);
             mbar_init(&c_empty[s], kRebuildWarps);
         }
         for (int s = 0; s < dw; s++) {
@@ -373,98 +375,30 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if constexpr (FUSED) {
-            const int64_t G64 = a.k / kGroup;     // groups per row
-            int64_t wcur[4] = {-1, -1, -1, -1};
-            uint32_t bm[4] = {0u, 0u, 0u, 0u}, rb[4] = {0u, 0u, 0u, 0u};
-            int sidx = 0;
-            for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
-                const int cs = sidx % dc;
-                const int64_t n0 = (ss.t / a.TB) * kBM;
-                const int q0 = ss.lo() - kSuper * ss.j, q1 = ss.hi() - kSuper * ss.j;
-                // raw (row, K-step) pairs of this lane's rows r = lane + 32 m
-                uint32_t rawbits = 0u, rank[16];
-#pragma unroll
-                for (int mm = 0; mm < 4; mm++) {
-                    const int64_t row = n0 + lane + 32 * mm;
-#pragma unroll
-                    for (int q = 0; q < kSuper; q++) {
-                        rank[4 * mm + q] = 0u;
-                        if (row < a.n && q >= q0 && q < q1) {
-                            const int64_t g = row * G64 + kSuper * ss.j + q;
-                            const int64_t w = g >> 5;
-                            if (w != wcur[mm]) {
-                                bm[mm] = __ldg(a.flagbits + w);
-                                rb[mm] = __ldg(a.rawbase + w);
-                                wcur[mm] = w;
-                                if (w + 1 < a.nflag) {   // the next word into L1 before it is needed
-                                    prefetch_l1(a.flagbits + w + 1);
-                                    prefetch_l1(a.rawbase + w + 1);
-                                }
-                            }
-                            const uint32_t bit = uint32_t(g) & 31u;
-                            if ((bm[mm] >> bit) & 1u) {
-                                rawbits |= 1u << (4 * mm + q);
-                                rank[4 * mm + q] = rb[mm] + __popc(bm[mm] & ((1u << bit) - 1u));
-                            }
-                        }
+            if (lane == 0) {
+                int sidx = 0;
+                for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
+                    const int cs = sidx % dc;
+                    if (sidx >= dc &&
+                        !mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag)) {
+                        fail(!*abort_flag);
+                        break;
                     }
+                    if (*abort_flag) break;
+                    uint8_t *st = cring + size_t(cs) * kCStage;
+                    const int32_t n0 = int32_t((ss.t / a.TB) * kBM);
+                    // 4-byte elements: the chunk's sign/mantissa bytes start at element 64 j
+                    // (two boxes of 128 bytes), its palette bytes at element 32 j
+                    mbar_arrive_expect_tx(&c_full[cs], HUFF ? uint32_t(2 * kBox) : uint32_t(3 * kBox));
+                    tma_load_2d(st + kOffSmA, tmA, 64 * ss.j, n0, &c_full[cs]);
+                    tma_load_2d(st + kOffSmB, tmA, 64 * ss.j + 32, n0, &c_full[cs]);
+                    if (!HUFF) tma_load_2d(st + kOffNib, tmB, 32 * ss.j, n0, &c_full[cs]);
                 }
-                // slots: an exclusive prefix sum of the lanes' raw counts
-                const uint32_t cnt = __popc(rawbits);
-                uint32_t scan = cnt;
-#pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, scan, d);
-                    if (lane >= d) scan += v;
-                }
-                uint32_t slot = scan - cnt;
-                int stop = 0;
-                if (lane == 0) {
-                    bool ok = true;
-                    if (sidx >= dc) ok = mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag);
-                    if (!ok) fail(!*abort_flag);
-                    stop = !ok || *abort_flag;
-                }
-                if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
-                uint8_t *st = cring + size_t(cs) * kCStage;
-                if (lane == 0) {
-                    mbar_expect_tx(&c_full[cs], HUFF ? uint32_t(2 * kBox) : uint32_t(3 * kBox));
-                    const int32_t xb = int32_t(kSuper * ss.j * kBK);   // first sign/mantissa byte of the chunk
-                    tma_load_2d(st + kOffSmA, tmA, xb, int32_t(n0), &c_full[cs]);
-                    tma_load_2d(st + kOffSmB, tmA, xb + 128, int32_t(n0), &c_full[cs]);
-                    if (!HUFF) tma_load_2d(st + kOffNib, tmB, xb / 2, int32_t(n0), &c_full[cs]);
-                }
-                uint32_t *tab = reinterpret_cast<uint32_t *>(st + kOffTab);
-#pragma unroll
-                for (int mm = 0; mm < 4; mm++) {
-                    const int r = lane + 32 * mm;
-#pragma unroll
-                    for (int q = 0; q < kSuper; q++) {
-                        uint32_t e = 0u;
-                        if ((rawbits >> (4 * mm + q)) & 1u) {
-                            if (slot < uint32_t(kRawSlots)) {
-                                const uint8_t *src = a.rawexp + uint64_t(rank[4 * mm + q]) * kGroup;
-                                uint8_t *dst = st + kOffRaw + slot * kGroup;
-#pragma unroll
-                                for (int c = 0; c < 4; c++) cp_async16(dst + 16 * c, src + 16 * c);
-                                e = kTabSlot | slot;
-                            } else {
-                                e = kTabRank | rank[4 * mm + q];
-                            }
-                            slot++;
-                        }
-                        tab[r * kSuper + q] = e;
-                    }
-                }
-                mbar_arrive(&c_full[cs]);                 // this lane's table entries are written
-                cp_async_mbar_arrive_noinc(&c_full[cs]);  // ... and, once landed, its raw copies
-            }
-            cp_async_wait_all();
-            // no copy may still be landing when the CTA exits (after an abort a
-            // decoder's arrival may be missing: those waits run out, bounded)
-            if (lane == 0)
+                // no copy may still be landing when the CTA exits (after an abort
+                // another role's arrival may be missing: those waits run out, bounded)
                 for (int i = max(0, sidx - dc); i < sidx; i++)
                     mbar_wait(&c_full[i % dc], uint32_t(i / dc) & 1u, *abort_flag ? T / 64 + 1 : T);
+            }
         } else if (lane == 0) {
             int issued = 0;
             UnitWalk walk(u0, a.S);
@@ -670,7 +604,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 if (warp == kEpiWarp0 && lane == 0) a.counters[t] = 0u;
             }
         }
-    } else if (warp < kStreamWarp) {
+    } else if (warp < kRawWarp) {
         if constexpr (FUSED) {
             // -------------------------------------------------------- rebuild
             const int wi = warp - kFirstRebuildWarp;   // 0..7
@@ -741,6 +675,104 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 if (lane == 0) mbar_arrive(&c_empty[cs]);
             }
             if (!ok && lane == 0 && !*abort_flag) fail(true);
+        }
+    } else if (warp == kRawWarp) {
+        if constexpr (FUSED) {
+            // -------------------------------------------------------- raw groups
+            // lane l handles rows r = l + 32 m; a row's 4 groups of the chunk are
+            // 4 consecutive bits of the raw bitmap (one funnel shift of the two
+            // words around them), so rows without raw groups cost a few
+            // instructions; a raw group's rank is the word's base plus the bits
+            // below it.  The entries are computed before the stage is free.
+            const int64_t G64 = a.k / kGroup;     // groups per row
+            int64_t wcur[4] = {-2, -2, -2, -2};
+            uint32_t blo[4], bhi[4], rlo[4], rhi[4];
+            int sidx = 0;
+            for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
+                const int cs = sidx % dc;
+                const int64_t n0 = (ss.t / a.TB) * kBM;
+                const int q0 = ss.lo() - kSuper * ss.j, q1 = ss.hi() - kSuper * ss.j;
+                const uint32_t qmask = ((1u << q1) - 1u) & ~((1u << q0) - 1u);
+                uint32_t rawbits = 0u, rank[16];
+#pragma unroll
+                for (int mm = 0; mm < 4; mm++) {
+#pragma unroll
+                    for (int q = 0; q < kSuper; q++) rank[4 * mm + q] = 0u;
+                    const int64_t row = n0 + lane + 32 * mm;
+                    if (row >= a.n) continue;
+                    const int64_t g0 = row * G64 + kSuper * ss.j;
+                    const int64_t w0 = g0 >> 5;
+                    if (w0 != wcur[mm]) {
+                        if (w0 == wcur[mm] + 1) {
+                            blo[mm] = bhi[mm];
+                            rlo[mm] = rhi[mm];
+                        } else {
+                            blo[mm] = __ldg(a.flagbits + w0);
+                            rlo[mm] = __ldg(a.rawbase + w0);
+                        }
+                        const bool more = w0 + 1 < a.nflag;
+                        bhi[mm] = more ? __ldg(a.flagbits + w0 + 1) : 0u;
+                        rhi[mm] = more ? __ldg(a.rawbase + w0 + 1) : 0u;
+                        wcur[mm] = w0;
+                    }
+                    const uint32_t b0 = uint32_t(g0) & 31u;
+                    const uint32_t bits = __funnelshift_r(blo[mm], bhi[mm], b0) & qmask;
+                    if (bits) {
+#pragma unroll
+                        for (int q = 0; q < kSuper; q++) {
+                            if (!((bits >> q) & 1u)) continue;
+                            const uint32_t b = b0 + uint32_t(q);
+                            rank[4 * mm + q] = b < 32u ? rlo[mm] + __popc(blo[mm] & ((1u << b) - 1u))
+                                                       : rhi[mm] + __popc(bhi[mm] & ((1u << (b - 32u)) - 1u));
+                        }
+                        rawbits |= bits << (4 * mm);
+                    }
+                }
+                // slots: an exclusive prefix sum of the lanes' raw counts
+                const uint32_t cnt = __popc(rawbits);
+                uint32_t scan = cnt;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, scan, d);
+                    if (lane >= d) scan += v;
+                }
+                uint32_t slot = scan - cnt;
+                int stop = 0;
+                if (lane == 0) {
+                    bool ok = true;
+                    if (sidx >= dc) ok = mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag);
+                    if (!ok) fail(!*abort_flag);
+                    stop = !ok || *abort_flag;
+                }
+                if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
+                uint8_t *st = cring + size_t(cs) * kCStage;
+                uint32_t *tab = reinterpret_cast<uint32_t *>(st + kOffTab);
+#pragma unroll
+                for (int mm = 0; mm < 4; mm++) {
+                    const int r = lane + 32 * mm;
+#pragma unroll
+                    for (int q = 0; q < kSuper; q++) {
+                        uint32_t e = 0u;
+                        if ((rawbits >> (4 * mm + q)) & 1u) {
+                            if (slot < uint32_t(kRawSlots)) {
+                                const uint8_t *src = a.rawexp + uint64_t(rank[4 * mm + q]) * kGroup;
+                                uint8_t *dst = st + kOffRaw + slot * kGroup;
+#pragma unroll
+                                for (int c = 0; c < 4; c++) cp_async16(dst + 16 * c, src + 16 * c);
+                                e = kTabSlot | slot;
+                            } else {
+                                e = kTabRank | rank[4 * mm + q];
+                            }
+                            slot++;
+                        }
+                        tab[r * kSuper + q] = e;
+                    }
+                }
+                mbar_arrive(&c_full[cs]);                 // this lane's table entries are written
+                cp_async_mbar_arrive_noinc(&c_full[cs]);  // ... and, once landed, its raw copies
+            }
+            cp_async_wait_all();
+            __syncwarp();
         }
     } else if (warp == kStreamWarp) {
         if constexpr (HUFF) {
@@ -1043,15 +1075,16 @@ cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
         a.rawexp = p.w->rawexp;
         a.nflag = (p.n * (p.k / kGroup) + 31) / 32;
         a.pal = make_palette16(p.w->palette);
-        // sign/mantissa boxes of 128 bytes (two K-steps) x 128 rows
-        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k), 128,
-                      kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+        // sign/mantissa boxes of 128 bytes (two K-steps) x 128 rows, as
+        // 4-byte elements (the copy engine moves the same bytes in fewer elements)
+        if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.w->sm, uint64_t(p.k / 4), uint64_t(p.n), uint64_t(p.k),
+                      32, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
     if (mode == kModePal) {
-        // palette boxes of 128 bytes (four K-steps) x 128 rows
-        if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n), uint64_t(p.k / 2),
-                      128, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+        // palette boxes of 128 bytes (four K-steps) x 128 rows, 4-byte elements
+        if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.pal, uint64_t(p.k / 8), uint64_t(p.n), uint64_t(p.k / 2),
+                      32, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         static int ready[64] = {0};
         err = prepare(k_gemm_sk_fused<BN>, kPalThreads, C::kTmemCols, ready);
