@@ -113,6 +113,23 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parit
     return true;
 }
 
+// mbar_wait_or_abort for roles that are not on the critical path (a warp
+// that waits a whole tile for its accumulator, a producer far ahead of its
+// consumer): between polls the warp sleeps, so that it leaves the issue
+// slots to the warps that do the work.  The time limit counts clock64 as
+// mbar_wait_or_abort does; sleeping only lengthens each poll.
+__device__ __forceinline__ bool mbar_wait_lazy(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                               const volatile int *abort, uint32_t sleep_ns = 256u) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long limit = (long long)(timeout_ns * 2);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort || clock64() - t0 > limit) return false;
+        __nanosleep(sleep_ns);
+    }
+    return true;
+}
+
 // Named barrier over `threads` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -41,23 +41,27 @@
 //          tile overlaps the MMAs of the next).
 //   2      X producer: cp.async into the 128-byte-swizzled K-major layout for
 //          up to 64 tokens, a TMA box per K-step for 128 and 256.
-//   3-6    epilogue: TMEM -> registers -> Y (or a partial tile + fix-up).
+//   3-6    epilogue: TMEM -> registers -> Y (or a partial tile + fix-up);
+//          it polls its accumulator barrier with sleeps in between, so that
+//          a warp waiting a whole tile leaves the issue slots to the rebuild.
 //   7-14   rebuild (palette, Huffman): all 8 warps work on the same K-step;
 //          lane l of warp w rebuilds half h = (l >> 3) & 1 (32 weights) of
 //          tile row 16w + 8(l >> 4) + (l & 7) into the 128-byte-swizzled
 //          K-major BF16 W tile.  A quarter warp covers 8 consecutive rows, so
 //          under the 128-byte swizzle every 16-byte shared-memory access of
 //          it falls on its own bank group.
-//   15     (fused) raw groups: per super-step the 32 lanes find the raw (row,
-//          group) pairs of the 128 rows, give each a slot in the stage
-//          (cp.async of its 64 exponents) and write a 128 x 4 table that tells
-//          the rebuild where each group's exponents are (palette plane, a
-//          slot, or, when the slots run out, the raw plane in global memory).
-//   16     (Huffman) stream producer: per super-step it reads the 128 chunks'
+//   15-18  (palette; 15-16 Huffman) raw groups: per super-step these warps
+//          find the raw (row, group) pairs of the 128 rows (each warp its
+//          share of the rows), give each a slot in the stage (cp.async of its
+//          64 exponents) and write a 128 x 4 table that tells the rebuild
+//          where each group's exponents are (palette plane, a slot, or, when
+//          the warp's slots run out, the raw plane in global memory).  One
+//          warp alone took longer per super-step than the rebuild.
+//   17     (Huffman) stream producer: per super-step it reads the 128 chunks'
 //          start bits and copies each chunk's stream words (cp.async) into
 //          one slot of a shared-memory ring, with a table of where they are
 //          (a chunk that does not fit is read from global memory instead).
-//   17-24  (Huffman) decoders: two groups of 4 warps take alternate
+//   18-25  (Huffman) decoders: two groups of 4 warps take alternate
 //          super-steps, one thread per tile row; a thread decodes its row's
 //          chunk with the 12-bit multi-symbol table straight into the
 //          super-step's palette area, in the stored 4-bit layout.
@@ -87,13 +91,14 @@ constexpr int kFixedWarps = 7;          // producer, MMA, X producer, 4 epilogue
 constexpr int kRebuildWarps = 8;
 constexpr int kEpiWarp0 = 3;
 constexpr int kFirstRebuildWarp = kFixedWarps;
-constexpr int kRawWarp = kFixedWarps + kRebuildWarps;      // fused flavours
-constexpr int kStreamWarp = kRawWarp + 1;                  // Huffman flavour
+constexpr int kRawWarp = kFixedWarps + kRebuildWarps;      // first raw-group warp (fused flavours)
+constexpr int kRawWarpsPal = 4, kRawWarpsHuff = 2;          // raw-group warps per flavour
+constexpr int kStreamWarp = kRawWarp + kRawWarpsHuff;      // Huffman flavour
 constexpr int kFirstDecWarp = kStreamWarp + 1;
 constexpr int kDecWarps = 8;            // two groups of 4
 constexpr int kPlainThreads = kFixedWarps * 32;
-constexpr int kPalThreads = (kFixedWarps + kRebuildWarps + 1) * 32;
-constexpr int kHuffThreads = (kFixedWarps + kRebuildWarps + 2 + kDecWarps) * 32;
+constexpr int kPalThreads = (kFixedWarps + kRebuildWarps + kRawWarpsPal) * 32;
+constexpr int kHuffThreads = (kFixedWarps + kRebuildWarps + kRawWarpsHuff + 1 + kDecWarps) * 32;
 
 constexpr int kTileW = kBM * kBK * 2;   // BF16 W tile of one K-step (128 rows x 128 B)
 
@@ -102,7 +107,7 @@ constexpr int kBox = kBM * 128;                  // one 128-row x 128-byte box
 constexpr int kOffSmA = 0;                       // sign/mantissa, K-steps 0-1 of the super-step
 constexpr int kOffSmB = kBox;                    //                K-steps 2-3
 constexpr int kOffNib = 2 * kBox;                // 4-bit palette indices, K-steps 0-3
-constexpr int kRawSlots = 128;                   // raw groups staged per super-step
+constexpr int kRawSlots = 64;                    // raw groups staged per super-step (16 per raw warp)
 constexpr int kOffRaw = 3 * kBox;                // kRawSlots x 64 exponent bytes
 constexpr int kOffTab = kOffRaw + kRawSlots * kGroup;   // uint32 [128 rows][4 K-steps]
 constexpr int kCStage = kOffTab + kBM * kSuper * 4;
@@ -157,11 +162,10 @@ __host__ __device__ __forceinline__ int sk_cta_of(int64_t u, int64_t units, int 
 }
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void prefetch_l1(const void *p) {
-    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+    // pointer arithmetic, not an integer round trip: the result stays
+    // recognisably a shared-memory pointer, so accesses through it compile
+    // to shared-memory loads and stores rather than generic ones
+    return p + ((1024u - (smem_addr(p) & 1023u)) & 1023u);
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -193,17 +197,20 @@ __host__ __device__ constexpr int sk_tail(int dc, int dw, int dx) {
 // index j (K-steps 4j..4j+3) touched there, the K-steps [lo, hi) the CTA
 // owns.  Walked the same way by every role that works per super-step.
 struct SuperSteps {
-    int64_t u0, u1, t, t_last;
-    int S, j, j_last, ka, kb;
+    int64_t u0, u1, t, t_last, rb;   // rb, tb: row block and token block of tile t
+    int S, TB, tb, j, j_last, ka, kb;
     __device__ __forceinline__ void start_tile() {
         ka = t == u0 / S ? int(u0 - t * S) : 0;
         kb = t == t_last ? int(u1 - t * S) : S;
         j = ka / kSuper;
         j_last = (kb - 1) / kSuper;
     }
-    __device__ __forceinline__ SuperSteps(int64_t u0_, int64_t u1_, int S_) : u0(u0_), u1(u1_), S(S_) {
+    __device__ __forceinline__ SuperSteps(int64_t u0_, int64_t u1_, int S_, int TB_)
+        : u0(u0_), u1(u1_), S(S_), TB(TB_) {
         t = u0 / S;
         t_last = (u1 - 1) / S;
+        rb = t / TB;
+        tb = int(t - rb * TB);
         start_tile();
     }
     __device__ __forceinline__ bool valid() const { return u1 > u0 && t <= t_last; }
@@ -212,20 +219,49 @@ struct SuperSteps {
     __device__ __forceinline__ void next() {
         if (++j > j_last) {
             ++t;
+            if (++tb == TB) {
+                tb = 0;
+                ++rb;
+            }
             if (t <= t_last) start_tile();
+        }
+    }
+};
+
+// Position in a ring of mbarrier-guarded stages: slot s, and the parity ph
+// of the pass over the ring (flips each time s wraps).  Advanced without
+// divisions; `wrapped` tells whether the slot was used before (its "empty"
+// barrier must then be waited for with parity ph ^ 1).
+struct Ring {
+    int s = 0;
+    uint32_t ph = 0;
+    bool wrapped = false;
+    __device__ __forceinline__ void next(int depth) {
+        if (++s == depth) {
+            s = 0;
+            ph ^= 1u;
+            wrapped = true;
         }
     }
 };
 
 // The CTA's units in order as (tile, K-step), advanced without divisions.
 struct UnitWalk {
-    int64_t t;
-    int ks, S;
-    __device__ __forceinline__ UnitWalk(int64_t u0, int S_) : t(u0 / S_), ks(int(u0 % S_)), S(S_) {}
+    int64_t t, rb;   // tile, its row block and token block
+    int ks, S, TB, tb;
+    __device__ __forceinline__ UnitWalk(int64_t u0, int S_, int TB_)
+        : t(u0 / S_), ks(int(u0 % S_)), S(S_), TB(TB_) {
+        rb = t / TB;
+        tb = int(t - rb * TB);
+    }
     __device__ __forceinline__ void next() {
         if (++ks == S) {
             ks = 0;
             ++t;
+            if (++tb == TB) {
+                tb = 0;
+                ++rb;
+            }
         }
     }
 };
@@ -327,7 +363,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             // the TMA producer, the 32 raw-group lanes once their table entries
             // are written and 32 once their copies landed, + the 4 decoder
             // warps of a group
-            mbar_init(&c_full[s], HUFF ? 1 + 64 + 4 : 1 + 64);
+            mbar_init(&c_full[s], HUFF ? 1 + 64 * kRawWarpsHuff + 4 : 1 + 64 * kRawWarpsPal);
             mbar_init(&c_empty[s], kRebuildWarps);
         }
         for (int s = 0; s < dw; s++) {
@@ -377,16 +413,16 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
         if constexpr (FUSED) {
             if (lane == 0) {
                 int sidx = 0;
-                for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
-                    const int cs = sidx % dc;
-                    if (sidx >= dc &&
-                        !mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag)) {
+                Ring rc;
+                for (SuperSteps ss(u0, u1, a.S, a.TB); ss.valid(); ss.next(), sidx++, rc.next(dc)) {
+                    const int cs = rc.s;
+                    if (rc.wrapped && !mbar_wait_or_abort(&c_empty[cs], rc.ph ^ 1u, T, abort_flag)) {
                         fail(!*abort_flag);
                         break;
                     }
                     if (*abort_flag) break;
                     uint8_t *st = cring + size_t(cs) * kCStage;
-                    const int32_t n0 = int32_t((ss.t / a.TB) * kBM);
+                    const int32_t n0 = int32_t(ss.rb * kBM);
                     // 4-byte elements: the chunk's sign/mantissa bytes start at element 64 j
                     // (two boxes of 128 bytes), its palette bytes at element 32 j
                     mbar_arrive_expect_tx(&c_full[cs], HUFF ? uint32_t(2 * kBox) : uint32_t(3 * kBox));
@@ -401,16 +437,13 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             }
         } else if (lane == 0) {
             int issued = 0;
-            UnitWalk walk(u0, a.S);
-            int64_t tcur = -1, n0 = 0;
-            for (int i = 0; i < nu; i++, walk.next()) {
-                if (walk.t != tcur) {
-                    tcur = walk.t;
-                    n0 = (tcur / a.TB) * kBM;
-                }
+            UnitWalk walk(u0, a.S, a.TB);
+            Ring rw;
+            for (int i = 0; i < nu; i++, walk.next(), rw.next(dw)) {
+                const int64_t n0 = walk.rb * kBM;
                 const int ks = walk.ks;
-                const int s = i % dw;
-                if (i >= dw && !mbar_wait_or_abort(&w_empty[s], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag)) {
+                const int s = rw.s;
+                if (rw.wrapped && !mbar_wait_or_abort(&w_empty[s], rw.ph ^ 1u, T, abort_flag)) {
                     fail(!*abort_flag);
                     break;
                 }
@@ -432,8 +465,9 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             int seg = -1;
             int64_t tprev = -1;
             bool first = true;
-            UnitWalk walk(u0, a.S);
-            for (int i = 0; i < nu && ok; i++, walk.next()) {
+            UnitWalk walk(u0, a.S, a.TB);
+            Ring rx, rw;
+            for (int i = 0; i < nu && ok; i++, walk.next(), rx.next(dx), rw.next(dw)) {
                 const int64_t t = walk.t;
                 if (t != tprev) {   // a new tile: close the previous accumulator, claim the next
                     if (seg >= 0) tc_commit(&acc_full[seg & 1]);
@@ -445,9 +479,9 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     tc_fence_after();
                     first = true;
                 }
-                const int xs = i % dx, ws = i % dw;
-                ok = mbar_wait_or_abort(&x_full[xs], uint32_t(i / dx) & 1u, T, abort_flag) &&
-                     mbar_wait_or_abort(&w_full[ws], uint32_t(i / dw) & 1u, T, abort_flag);
+                const int xs = rx.s, ws = rw.s;
+                ok = mbar_wait_or_abort(&x_full[xs], rx.ph, T, abort_flag) &&
+                     mbar_wait_or_abort(&w_full[ws], rw.ph, T, abort_flag);
                 if (!ok) break;
                 // X copied through the load/store path: make it visible to the tensor core
                 if (!C::kXByTma) fence_proxy_async_smem();
@@ -476,19 +510,15 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
     } else if (warp == 2) {
         // ------------------------------------------------------------ X producer
         int issued = 0;
-        UnitWalk walk(u0, a.S);
-        int64_t tcur = -1, m0 = 0;
-        for (int i = 0; i < nu; i++, walk.next()) {
-            if (walk.t != tcur) {
-                tcur = walk.t;
-                m0 = (tcur % a.TB) * BN;
-            }
+        UnitWalk walk(u0, a.S, a.TB);
+        Ring rx;
+        for (int i = 0; i < nu; i++, walk.next(), rx.next(dx)) {
+            const int64_t m0 = int64_t(walk.tb) * BN;
             const int ks = walk.ks;
-            const int s = i % dx;
+            const int s = rx.s;
             int stop = 0;
             if (lane == 0) {
-                const bool ok =
-                    i < dx || mbar_wait_or_abort(&x_empty[s], (uint32_t(i / dx) & 1u) ^ 1u, T, abort_flag);
+                const bool ok = !rx.wrapped || mbar_wait_lazy(&x_empty[s], rx.ph ^ 1u, T, abort_flag, 64u);
                 if (!ok) fail(!*abort_flag);
                 stop = !ok || *abort_flag;
             }
@@ -532,7 +562,7 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             const int64_t kb = t == t_last ? u1 - t * a.S : a.S;
             const bool split = ka != 0 || kb != a.S;
             const int slot = t == t_first ? 0 : 1;
-            const bool ok = mbar_wait_or_abort(&acc_full[b], uint32_t(seg >> 1) & 1u, T, abort_flag);
+            const bool ok = mbar_wait_lazy(&acc_full[b], uint32_t(seg >> 1) & 1u, T, abort_flag);
             // the four epilogue warps decide together, so that all of them
             // meet the same named barriers below
             if (named_bar_any(1, 128, !ok)) {
@@ -612,21 +642,21 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             const int h = (lane >> 3) & 1;                          // half of the row's 64 weights
             const int sw = R & 7;                                   // 128-byte swizzle phase of the row
             const Palette16 P = a.pal;
-            int i = 0, sidx = 0;
+            Ring rc, rw;
             bool ok = true;
-            for (SuperSteps ss(u0, u1, a.S); ss.valid() && ok; ss.next(), sidx++) {
-                const int cs = sidx % dc;
-                ok = mbar_wait_or_abort(&c_full[cs], uint32_t(sidx / dc) & 1u, T, abort_flag);
+            for (SuperSteps ss(u0, u1, a.S, a.TB); ss.valid() && ok; ss.next(), rc.next(dc)) {
+                const int cs = rc.s;
+                ok = mbar_wait_or_abort(&c_full[cs], rc.ph, T, abort_flag);
                 if (__any_sync(0xFFFFFFFFu, !ok)) {
                     ok = false;
                     break;
                 }
                 const uint8_t *st = cring + size_t(cs) * kCStage;
                 const uint32_t *tab = reinterpret_cast<const uint32_t *>(st + kOffTab);
-                for (int ks = ss.lo(); ks < ss.hi(); ks++, i++) {
+                for (int ks = ss.lo(); ks < ss.hi(); ks++, rw.next(dw)) {
                     const int q = ks - kSuper * ss.j;
-                    const int ws = i % dw;
-                    if (i >= dw) ok = mbar_wait_or_abort(&w_empty[ws], (uint32_t(i / dw) & 1u) ^ 1u, T, abort_flag);
+                    const int ws = rw.s;
+                    if (rw.wrapped) ok = mbar_wait_or_abort(&w_empty[ws], rw.ph ^ 1u, T, abort_flag);
                     if (__any_sync(0xFFFFFFFFu, !ok)) {
                         ok = false;
                         break;
@@ -676,29 +706,38 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             }
             if (!ok && lane == 0 && !*abort_flag) fail(true);
         }
-    } else if (warp == kRawWarp) {
+    } else if (warp < kRawWarp + (HUFF ? kRawWarpsHuff : kRawWarpsPal)) {
         if constexpr (FUSED) {
             // -------------------------------------------------------- raw groups
-            // lane l handles rows r = l + 32 m; a row's 4 groups of the chunk are
-            // 4 consecutive bits of the raw bitmap (one funnel shift of the two
-            // words around them), so rows without raw groups cost a few
+            // RAWW warps split the tile's rows: lane l of raw warp v handles
+            // rows r = 32 (MM v + m) + l, m < MM, and gives its raw groups
+            // slots of the warp's own range.  A row's 4 groups of the chunk
+            // are 4 consecutive bits of the raw bitmap (one funnel shift of the
+            // two words around them), so rows without raw groups cost a few
             // instructions; a raw group's rank is the word's base plus the bits
             // below it.  The entries are computed before the stage is free.
+            constexpr int RAWW = HUFF ? kRawWarpsHuff : kRawWarpsPal;
+            constexpr int MM = 4 / RAWW;                      // rows per lane
+            constexpr uint32_t kWarpSlots = kRawSlots / RAWW;
+            const int v = warp - kRawWarp;
+            const uint32_t slot_end = kWarpSlots * uint32_t(v + 1);
             const int64_t G64 = a.k / kGroup;     // groups per row
-            int64_t wcur[4] = {-2, -2, -2, -2};
-            uint32_t blo[4], bhi[4], rlo[4], rhi[4];
-            int sidx = 0;
-            for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
-                const int cs = sidx % dc;
-                const int64_t n0 = (ss.t / a.TB) * kBM;
+            int64_t wcur[MM];
+            uint32_t blo[MM], bhi[MM], rlo[MM], rhi[MM];
+#pragma unroll
+            for (int mm = 0; mm < MM; mm++) wcur[mm] = -2;
+            Ring rc;
+            for (SuperSteps ss(u0, u1, a.S, a.TB); ss.valid(); ss.next(), rc.next(dc)) {
+                const int cs = rc.s;
+                const int64_t n0 = ss.rb * kBM;
                 const int q0 = ss.lo() - kSuper * ss.j, q1 = ss.hi() - kSuper * ss.j;
                 const uint32_t qmask = ((1u << q1) - 1u) & ~((1u << q0) - 1u);
-                uint32_t rawbits = 0u, rank[16];
+                uint32_t rawbits = 0u, rank[4 * MM];
 #pragma unroll
-                for (int mm = 0; mm < 4; mm++) {
+                for (int mm = 0; mm < MM; mm++) {
 #pragma unroll
                     for (int q = 0; q < kSuper; q++) rank[4 * mm + q] = 0u;
-                    const int64_t row = n0 + lane + 32 * mm;
+                    const int64_t row = n0 + 32 * (MM * v + mm) + lane;
                     if (row >= a.n) continue;
                     const int64_t g0 = row * G64 + kSuper * ss.j;
                     const int64_t w0 = g0 >> 5;
@@ -736,11 +775,11 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                     const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, scan, d);
                     if (lane >= d) scan += v;
                 }
-                uint32_t slot = scan - cnt;
+                uint32_t slot = kWarpSlots * uint32_t(v) + scan - cnt;
                 int stop = 0;
                 if (lane == 0) {
                     bool ok = true;
-                    if (sidx >= dc) ok = mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag);
+                    if (rc.wrapped) ok = mbar_wait_or_abort(&c_empty[cs], rc.ph ^ 1u, T, abort_flag);
                     if (!ok) fail(!*abort_flag);
                     stop = !ok || *abort_flag;
                 }
@@ -748,13 +787,13 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
                 uint8_t *st = cring + size_t(cs) * kCStage;
                 uint32_t *tab = reinterpret_cast<uint32_t *>(st + kOffTab);
 #pragma unroll
-                for (int mm = 0; mm < 4; mm++) {
-                    const int r = lane + 32 * mm;
+                for (int mm = 0; mm < MM; mm++) {
+                    const int r = 32 * (MM * v + mm) + lane;
 #pragma unroll
                     for (int q = 0; q < kSuper; q++) {
                         uint32_t e = 0u;
                         if ((rawbits >> (4 * mm + q)) & 1u) {
-                            if (slot < uint32_t(kRawSlots)) {
+                            if (slot < slot_end) {
                                 const uint8_t *src = a.rawexp + uint64_t(rank[4 * mm + q]) * kGroup;
                                 uint8_t *dst = st + kOffRaw + slot * kGroup;
 #pragma unroll
@@ -783,18 +822,17 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             }
             const int64_t G4 = a.k / (kSuper * kGroup);   // chunks per row
             int sidx = 0;
-            for (SuperSteps ss(u0, u1, a.S); ss.valid(); ss.next(), sidx++) {
-                const int slot = sidx % kSlots;
+            Ring rs;
+            for (SuperSteps ss(u0, u1, a.S, a.TB); ss.valid(); ss.next(), sidx++, rs.next(kSlots)) {
+                const int slot = rs.s;
                 int stop = 0;
                 if (lane == 0) {
-                    const bool ok = sidx < kSlots ||
-                                    mbar_wait_or_abort(&s_empty[slot], (uint32_t(sidx / kSlots) & 1u) ^ 1u, T,
-                                                       abort_flag);
+                    const bool ok = !rs.wrapped || mbar_wait_or_abort(&s_empty[slot], rs.ph ^ 1u, T, abort_flag);
                     if (!ok) fail(!*abort_flag);
                     stop = !ok || *abort_flag;
                 }
                 if (__shfl_sync(0xFFFFFFFFu, stop, 0)) break;
-                const int64_t n0 = (ss.t / a.TB) * kBM;
+                const int64_t n0 = ss.rb * kBM;
                 uint32_t start[4], end[4], wfirst[4], bytes[4], raw4[4];
 #pragma unroll
                 for (int mm = 0; mm < 4; mm++) {
@@ -865,18 +903,20 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             const int sw = r & 7;
             bool ok = mbar_wait_or_abort(lut_full, 0, T, abort_flag);
             int sidx = 0;
-            for (SuperSteps ss(u0, u1, a.S); ss.valid() && ok; ss.next(), sidx++) {
+            Ring rs, rc;
+            for (SuperSteps ss(u0, u1, a.S, a.TB); ss.valid() && ok;
+                 ss.next(), sidx++, rs.next(kSlots), rc.next(dc)) {
                 if ((sidx & 1) != grp) continue;
-                const int slot = sidx % kSlots, cs = sidx % dc;
-                ok = mbar_wait_or_abort(&s_full[slot], uint32_t(sidx / kSlots) & 1u, T, abort_flag) &&
-                     (sidx < dc || mbar_wait_or_abort(&c_empty[cs], (uint32_t(sidx / dc) & 1u) ^ 1u, T, abort_flag));
+                const int slot = rs.s, cs = rc.s;
+                ok = mbar_wait_or_abort(&s_full[slot], rs.ph, T, abort_flag) &&
+                     (!rc.wrapped || mbar_wait_or_abort(&c_empty[cs], rc.ph ^ 1u, T, abort_flag));
                 if (__any_sync(0xFFFFFFFFu, !ok)) {
                     ok = false;
                     break;
                 }
                 const uint4 e = htable[slot * kBM + r];
                 const uint32_t raw4 = hraw4[slot * kBM + r];
-                const int64_t row = (ss.t / a.TB) * kBM + r;
+                const int64_t row = ss.rb * kBM + r;
                 uint32_t p = e.z;
                 const uint32_t end = e.w;
                 bool good = e.z <= e.w && uint64_t(e.w) <= a.stream_bits;

@@ -77,7 +77,10 @@ struct TcArgs {
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+    // pointer arithmetic, not an integer round trip: the result stays
+    // recognisably a shared-memory pointer, so accesses through it compile
+    // to shared-memory loads and stores rather than generic ones
+    return p + ((1024u - (smem_addr(p) & 1023u)) & 1023u);
 }
 
 // 4 x tcgen05.mma (K = 16 each) for one 64-wide K-step; A = W tile, B = X tile
