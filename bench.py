@@ -750,7 +750,8 @@ def case_kernel(argv):
                       "split": plan.split_k, "us": us, "alg_bytes": int(alg),
                       "gbs": alg / us / 1e3, "tflops": None if preprocessing else flops / us / 1e6,
                       "l2": "flushed before each call" if a.flush else
-                      "not flushed (a matrix under 126 MB stays in L2 between calls)"}))
+                      ("not flushed; the kernel's %.0f MB exceed the 126 MB L2" % (alg / 1e6) if alg > 126e6 else
+                       "not flushed: %.0f MB can stay in the 126 MB L2 between calls" % (alg / 1e6))}))
     return 0
 
 
@@ -967,7 +968,7 @@ def case_sweep70b(argv):
 
     for (job, blob) in zip(jobs, blobs):
         n, k, sigma, frac, seed = job
-        name = shapes[[s[1:] for s in shapes].index((n, k))][0]
+        name = shapes[(seed - 7000) % 10][0]   # gate and up share a shape: the seed tells them apart
         mat = uw.Matrix(blob)
         info = mat.info
         w = synth.weights_bf16(n, k, sigma, frac, 1.0, seed=seed)

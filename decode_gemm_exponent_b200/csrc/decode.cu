@@ -3,12 +3,10 @@
 // exponent bytes; pipeline 3 transcodes the Huffman stream to 4-bit palette
 // indices at run time).
 //
-// The grid is one wave of CTAs (three fit on an SM); each CTA of 256 threads
-// owns an equal contiguous share of the chunks and walks it in tiles of at
-// most 256 chunks (1024 groups, 65536 weights), so no SM idles in a partial
-// last wave.  Per tile:
-//   1. One thread TMA-bulk-copies the tile's slice of the bitstream (and,
-//      for the first tile, the 16 KB decode table) into shared memory (a slice larger than the buffer is
+// One CTA of 256 threads owns a tile of 256 chunks (1024 groups, 65536
+// weights); three CTAs fit on an SM.
+//   1. One thread TMA-bulk-copies the 16 KB decode table and the tile's slice
+//      of the bitstream into shared memory (a slice larger than the buffer is
 //      read from global memory instead).  Meanwhile every thread loads its
 //      chunk's bounds and, for BF16 output, the first sign/mantissa vectors
 //      it will write, so that their latency hides under the decode.
@@ -25,8 +23,6 @@
 //      the stored 4-bit layout (transcode), exponent bytes (exponent decode),
 //      or BF16 = palette exponent (or raw-plane exponent) joined with the
 //      sign/mantissa byte (decode).
-#include <algorithm>
-
 #include "device_common.cuh"
 #include "kernels.h"
 #include "uw_format.h"
@@ -200,26 +196,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(smem_raw);
     const int tid = threadIdx.x;
-    // This CTA's chunks: an equal share of the matrix's in runs of 8 chunks
-    // (32 groups, one raw-bitmap word), cut into equal tiles of at most 256.
-    const int64_t runs = (a.n_chunks + 7) / 8;
-    const int64_t cta_c0 = 8 * (runs * blockIdx.x / gridDim.x);
-    const int64_t cta_c1 = min(a.n_chunks, 8 * (runs * (blockIdx.x + 1) / gridDim.x));
-    const int64_t n_tiles = (cta_c1 - cta_c0 + kTileChunks - 1) / kTileChunks;
-    const int64_t tile_chunks = n_tiles ? 8 * ((cta_c1 - cta_c0 + 8 * n_tiles - 1) / (8 * n_tiles)) : 0;
-    if (tid == 0) {
-        mbar_init(&S.bar, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    // (rounding the tile size up to whole runs can leave the last tiles empty)
-    for (int64_t tile = 0; tile < n_tiles && cta_c0 + tile * tile_chunks < cta_c1; tile++) {
-    const int64_t c_begin = cta_c0 + tile * tile_chunks;
-    const int64_t c_end = min(cta_c1, c_begin + tile_chunks);
+    const int64_t c_begin = int64_t(blockIdx.x) * kTileChunks;
+    const int64_t c_end = min(a.n_chunks, c_begin + kTileChunks);
     const int64_t g_begin = c_begin * kChunkGroups;
     const int64_t g_end = min(a.n_groups, c_end * kChunkGroups);
     const uint32_t b_begin = a.chunk_off[c_begin], b_end = a.chunk_off[c_end];
-    const uint32_t parity = uint32_t(tile) & 1u;
 
     if (tid < kFlagWords) {
         const int64_t wi = g_begin / 32 + tid;
@@ -238,10 +219,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
         S.seg_word0 = use_global ? 0u : uint32_t(w0);
         S.use_global = use_global;
         if (bad) flag_error(a.status, UW_DEVERR_CORRUPT);
+        mbar_init(&S.bar, 1);
+        fence_mbar_init();
         const uint32_t seg_bytes = use_global ? 0u : uint32_t(w1 - w0) * 4u;
-        const uint32_t lut_bytes = tile == 0 ? uint32_t(kLutEntries * 4) : 0u;   // the table stays
-        mbar_arrive_expect_tx(&S.bar, lut_bytes + seg_bytes);
-        if (lut_bytes) bulk_g2s(S.lut, a.dlut, lut_bytes, &S.bar);
+        mbar_arrive_expect_tx(&S.bar, uint32_t(kLutEntries * 4) + seg_bytes);
+        bulk_g2s(S.lut, a.dlut, kLutEntries * 4, &S.bar);
         if (seg_bytes) bulk_g2s(S.seg, a.stream + w0, seg_bytes, &S.bar);
     }
 
@@ -261,11 +243,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
         }
     }
     __syncthreads();
-    const bool landed = mbar_wait(&S.bar, parity, kTimeoutNs);
+    const bool landed = mbar_wait(&S.bar, 0, kTimeoutNs);
     if (__syncthreads_or(!landed)) {
         if (tid == 0) {
             flag_error(a.status, UW_DEVERR_TIMEOUT);
-            mbar_wait(&S.bar, parity, kTimeoutNs);   // let any copy in flight land before exit
+            mbar_wait(&S.bar, 0, kTimeoutNs);   // let any copy in flight land before exit
         }
         return;
     }
@@ -398,8 +380,6 @@ __global__ void __launch_bounds__(kThreads, 3) k_huff_decode(const DecodeArgs a)
             }
         }
     }
-    __syncthreads();   // the tile's shared buffers are free for the next tile
-    }
 }
 
 }  // namespace
@@ -439,26 +419,17 @@ DecodeArgs decode_args(const uw_dmat &w) {
 
 template <int OUT>
 cudaError_t launch_mode(const DecodeArgs &a, cudaStream_t stream) {
+    const unsigned grid = unsigned((a.n_chunks + kTileChunks - 1) / kTileChunks);
     const size_t smem = sizeof(DecodeSmem);
-    // opt-in and the number of CTAs that fit the GPU at once, per device
-    static thread_local int ready_dev = -1, resident = 0;
+    static thread_local int ready_dev = -1;   // shared-memory opt-in done on this device
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (ready_dev != dev) {
         err = cudaFuncSetAttribute(k_huff_decode<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (err != cudaSuccess) return err;
-        int per_sm = 0, sms = 0;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_huff_decode<OUT>, kThreads, smem);
-        if (err != cudaSuccess) return err;
-        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (err != cudaSuccess) return err;
-        resident = std::max(1, per_sm * sms);
         ready_dev = dev;
     }
-    // one wave of CTAs, each an equal share of the chunks (no partial last wave)
-    const int64_t tiles = (a.n_chunks + kTileChunks - 1) / kTileChunks;
-    const unsigned grid = unsigned(std::max<int64_t>(1, std::min<int64_t>(tiles, resident)));
     k_huff_decode<OUT><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
