@@ -302,7 +302,23 @@ def run_reference(args, rank):
 # that launch, and a SHA-256 over the kernel's sources with comments and
 # whitespace removed (source_digest); a figure is reported (scaled to the
 # group's mean algorithmic bytes per launch) only while that code is unchanged.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    "fused/mma_gemv_s4_w2": {
+        "bytes": 92214784, "alg_bytes": 90053056,
+        "files": ("decode_gemm_exponent_b200/csrc/gemv_mma.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
+        "sha256": "575bde04e02e27b9e20c6421f3838dc51a43ce02e91afdfdf42155202f5a5fb3",
+    },
+    "fused/tcgen05_bn16": {
+        "bytes": 93618944, "alg_bytes": 91036096,
+        "files": ("decode_gemm_exponent_b200/csrc/gemm_tc.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
+        "sha256": "fda7251c9e7722428768fed0c161d8960c8678394b07b996cf7bb8641cbd8dec",
+    },
+    "fused/tcgen05_bn64": {
+        "bytes": 93693184, "alg_bytes": 94181824,
+        "files": ("decode_gemm_exponent_b200/csrc/gemm_tc.cu", "decode_gemm_exponent_b200/csrc/device_common.cuh"),
+        "sha256": "fda7251c9e7722428768fed0c161d8960c8678394b07b996cf7bb8641cbd8dec",
+    },
+}
 
 
 def source_digest(texts) -> str:
@@ -651,8 +667,10 @@ def run_gpu(args, rank, world):
 
 def case_kernel(argv):
     """One libuw kernel on one synthetic matrix, for timing or profiler capture:
-    one warm-up launch, then --reps timed launches (CUDA events); prints the
-    per-launch time and the algorithmic bytes / FLOPs per launch."""
+    one warm-up launch, then --reps timed launches (CUDA events) -- back to
+    back after one more untimed launch, or (--flush) each on its own after a
+    512 MB read; prints the per-launch time and the algorithmic bytes / FLOPs
+    per launch.  Under ncu, `-s 1 -c 1` captures the second launch."""
     ap = argparse.ArgumentParser(prog="bench.py --case kernel")
     ap.add_argument("--kernel", required=True,
                     choices=["decode", "exp_decode", "transcode", "fma", "tc", "mma", "sk",
@@ -740,6 +758,10 @@ def case_kernel(argv):
             total += e0.elapsed_time(e1)
         us = 1e3 * total / a.reps
     else:
+        # one untimed launch first, so that the GPU is busy while the host
+        # issues the start event and the timed launches: the host's issue
+        # time of the first timed launch does not count as GPU time
+        run()
         e0.record()
         for _ in range(a.reps):
             run()
