@@ -64,11 +64,12 @@ uint64_t prep_bytes(int64_t n, int64_t k, const uw_plan *p) { return prep_worksp
 uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const uw_dmat *w,
                      const uint8_t *pal, int64_t n, int64_t k, float *y, const uw_plan *plan,
                      float *partial, uint32_t *status, uint32_t *sk_counters, cudaStream_t stream,
-                     bool huffman = false) {
+                     bool huffman = false, bool w_stable = false) {
     if (plan->kernel == UW_KERNEL_FMA)
         return cuda_status(launch_gemv_fma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, status, stream));
     if (plan->kernel == UW_KERNEL_MMA)
-        return cuda_status(launch_gemv_mma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, plan->stages, stream));
+        return cuda_status(
+            launch_gemv_mma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, plan->stages, stream, w_stable));
     TcLaunch t{};
     t.x = x;
     t.m = m;
@@ -86,6 +87,7 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
     t.timeout_ns = plan->timeout_ns > 0 ? uint64_t(plan->timeout_ns) : kDefaultTimeoutNs;
     t.dev_status = status;
     t.huffman = huffman;
+    t.w_stable = w_stable;
     if (plan->kernel == UW_KERNEL_TC_SK) {
         uint8_t *base = reinterpret_cast<uint8_t *>(partial);
         if (!base) return UW_ERR_WORKSPACE;
@@ -289,7 +291,11 @@ uw_status fused_matmul_ex(const uint16_t *x_dev, int64_t m, const uw_dmat *w, co
         pal = pal_dev ? pal_dev : w->pal;
         if (!pal || !aligned(pal, 16)) return UW_ERR_INVALID_ARG;
     }
-    return run_kernel(x_dev, m, nullptr, w, pal, w->n, w->k, y_dev, plan, partial, w->dev_status, sk_counters, s);
+    // the blob's own 4-bit plane: no kernel writes it (a transcoded or
+    // caller-provided plane may still be being written by an earlier kernel)
+    const bool w_stable = plan->pipeline == UW_PIPE_DIRECT_PALETTE && pal == w->pal;
+    return run_kernel(x_dev, m, nullptr, w, pal, w->n, w->k, y_dev, plan, partial, w->dev_status, sk_counters, s,
+                      false, w_stable);
 }
 
 uw_status matmul_bf16_ex(const uint16_t *x_dev, int64_t m, const uint16_t *w_dev, int64_t n, int64_t k, float *y_dev,

@@ -130,6 +130,16 @@ __device__ __forceinline__ bool mbar_wait_lazy(uint64_t *bar, uint32_t parity, u
     return true;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel on its stream is still
+// running, once every CTA of that kernel has called pdl_trigger (or exited).
+// Before it reads anything an earlier kernel may have written, or writes
+// anything an earlier kernel may still read, a thread calls pdl_wait, which
+// returns when the earlier kernels have completed and their writes are
+// visible.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Named barrier over `threads` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -74,6 +74,7 @@ struct TcArgs {
     const uint8_t *rawexp;
     Palette16 pal;
     uint32_t *status;
+    int w_stable;              // fused: planes no kernel writes (loaded before pdl_wait)
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
@@ -145,6 +146,8 @@ __global__ void __launch_bounds__(kPlainThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();   // W may be the output of the kernel before (a decode)
     const int64_t n0 = int64_t(blockIdx.x) * kBM;
     const int64_t m0 = int64_t(blockIdx.y) * BN;
     const int split = blockIdx.z;
@@ -284,6 +287,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the next kernel on the stream may be scheduled now; with planes no
+    // kernel writes, the compressed tiles, the raw bitmap and the raw
+    // exponents are loaded before waiting for the previous kernel, X (and
+    // every write) only after it
+    pdl_trigger();
+    if (!a.w_stable) pdl_wait();
     const int64_t n0 = int64_t(blockIdx.x) * kBM;
     const int64_t m0 = int64_t(blockIdx.y) * BN * TT;
     const int split = blockIdx.z;
@@ -404,6 +413,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     } else if (warp == 2) {
         // ------------------------------------------------ X producer
         if (lane == 0) {
+            pdl_wait();
             int issued = 0;
             for (int ks = 0; ks < nks; ks++) {
                 const int s = ks % XS;
@@ -501,6 +511,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tc_fence_after();
         const bool skip = __any_sync(0xFFFFFFFFu, !ok || *abort_flag != 0 || nks == 0);
         if (!ok && lane == 0) flag_error(a.status, UW_DEVERR_TIMEOUT);
+        pdl_wait();   // (returns at once: X was read after it)
         if (!skip)
 #pragma unroll 1
             for (int t = 0; t < TT; t++)
@@ -520,6 +531,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
 __global__ void k_splitk_reduce(const float *__restrict__ partial, int split_k, int64_t count,
                                 float *__restrict__ y) {
+    pdl_trigger();
+    pdl_wait();   // the partials are the previous kernel's output
     const int64_t i4 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
     if (i4 >= count) return;
     if (i4 + 4 <= count && (count & 3) == 0) {
@@ -614,8 +627,8 @@ cudaError_t launch_plain(const TcLaunch &p, cudaStream_t stream) {
     cudaError_t err = prepare(k_gemm_tc_plain<BN>, kPlainThreads, smem, C::kTmemCols, stages, ready);
     if (err != cudaSuccess) return err;
     dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN - 1) / BN), unsigned(a.split_k));
-    k_gemm_tc_plain<BN><<<grid, kPlainThreads, smem, stream>>>(mx, mw, a);
-    err = cudaGetLastError();
+    err = launch_pdl(false, k_gemm_tc_plain<BN>, grid, dim3(kPlainThreads), smem, stream, mx, mw, a);
+    if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (a.split_k > 1) return launch_splitk_reduce(p.partial, a.split_k, p.m * p.n, p.y, stream);
     return cudaSuccess;
@@ -655,13 +668,15 @@ cudaError_t launch_fused(const TcLaunch &p, cudaStream_t stream) {
     a.rawbase = p.w->rawbase;
     a.rawexp = p.w->rawexp;
     a.pal = make_palette16(p.w->palette);
+    a.w_stable = p.w_stable ? 1 : 0;
     if (a.split_k > 1 && !p.partial) return cudaErrorInvalidValue;
     static thread_local int ready[16] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
     cudaError_t err = prepare(k_gemm_tc_fused<BN, TT>, kFusedThreads, smem, C::kTmemCols, cs, ready);
     if (err != cudaSuccess) return err;
     dim3 grid(unsigned((p.n + kBM - 1) / kBM), unsigned((p.m + BN * TT - 1) / (BN * TT)), unsigned(a.split_k));
-    k_gemm_tc_fused<BN, TT><<<grid, kFusedThreads, smem, stream>>>(mx, msm, mpl, a, bw);
-    err = cudaGetLastError();
+    err = launch_pdl(a.w_stable != 0, k_gemm_tc_fused<BN, TT>, grid, dim3(kFusedThreads), smem, stream, mx, msm, mpl,
+                     a, bw);
+    if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (a.split_k > 1) return launch_splitk_reduce(p.partial, a.split_k, p.m * p.n, p.y, stream);
     return cudaSuccess;
@@ -683,8 +698,9 @@ cudaError_t launch_splitk_reduce(const float *partial, int split_k, int64_t coun
                                  cudaStream_t stream) {
     const int threads = 256;
     const int64_t blocks = (count / 4 + 1 + threads - 1) / threads;
-    k_splitk_reduce<<<unsigned(blocks), threads, 0, stream>>>(partial, split_k, count, y);
-    return cudaGetLastError();
+    const cudaError_t err = launch_pdl(false, k_splitk_reduce, dim3(unsigned(blocks)), dim3(threads), 0, stream,
+                                       partial, split_k, count, y);
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const TcLaunch &p, cudaStream_t stream) {

@@ -63,6 +63,7 @@ struct MmaArgs {
     int64_t n, k;
     int m;
     int flag_words;            // fused: bitmap words staged per CTA (16 rows)
+    int w_stable;              // fused: planes no kernel writes (read before pdl_wait)
     float *y;                  // [m, n]
 };
 
@@ -178,6 +179,11 @@ __device__ __forceinline__ void gemv_mma_tile(const MmaArgs &a, int64_t tile) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slices = blockDim.x >> 5;
     const int g = lane >> 2, c = lane & 3;
+    // the next kernel on the stream may be scheduled now; with planes no
+    // kernel writes, the raw bitmap and the first loads of W are issued
+    // before waiting for the previous kernel (X, Y and everything else after)
+    pdl_trigger();
+    if (!a.w_stable) pdl_wait();
     const int64_t row0 = tile * kTileRows;
     const int64_t ra = row0 + g, rb = ra + 8;       // this lane's two rows
     const int64_t gpr = a.k / kChunk;               // groups per row
@@ -225,7 +231,7 @@ __device__ __forceinline__ void gemv_mma_tile(const MmaArgs &a, int64_t tile) {
 
     Half<Q> ha[kStages], hb[kStages];
     bool fa[kStages], fb[kStages];
-    auto issue = [&](int i, int s) {   // loads of chunk i into ring slot s
+    auto issue = [&](int i, int s, bool x_prefetch = true) {   // loads of chunk i into ring slot s
         const int bit = ((i * Q) & 63) + coff;
         fa[s] = PAL && ((rawa >> bit) & 1u);
         fb[s] = PAL && ((rawb >> bit) & 1u);
@@ -234,8 +240,10 @@ __device__ __forceinline__ void gemv_mma_tile(const MmaArgs &a, int64_t tile) {
         hb[s] = load_half<PAL, Q>(a, smb + int64_t(i) * kCh, palb + i * (kCh / 8), wb + int64_t(i) * kCh, fb[s],
                                   gb + i * Q + coff, goff, sflags, srb, wbase);
         // the chunk's X rows into L1 now, so that the MMA steps do not wait on L2
-        prefetch_l1(x0 + int64_t(i) * kCh);
-        if (NT == 2) prefetch_l1(x1 + int64_t(i) * kCh);
+        if (x_prefetch) {
+            prefetch_l1(x0 + int64_t(i) * kCh);
+            if (NT == 2) prefetch_l1(x1 + int64_t(i) * kCh);
+        }
     };
     auto mma_tile = [&](int t, const uint32_t (&wA)[8 * Q], const uint32_t (&wB)[8 * Q], const uint16_t *xrow) {
         uint32_t xw[8 * Q];
@@ -261,9 +269,12 @@ __device__ __forceinline__ void gemv_mma_tile(const MmaArgs &a, int64_t tile) {
         if (NT == 2) mma_tile(NT - 1, wA, wB, x1 + int64_t(i) * kCh);
     };
 
+    // the ring's first loads; X only after the previous kernel has ended (a
+    // prefetch before that could keep a stale line of X in L1)
 #pragma unroll
     for (int s = 0; s < kStages; s++)
-        if (s < nch) issue(s, s);
+        if (s < nch) issue(s, s, !a.w_stable);
+    if (a.w_stable) pdl_wait();
     int i0 = 0;
     for (; i0 + kStages <= nch; i0 += kStages) {
 #pragma unroll
@@ -349,7 +360,7 @@ __global__ void __launch_bounds__(kMaxSlices * 32) k_gemv_mma_batched(const __gr
 
 cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
                             const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices, int width,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool w_stable) {
     if (m < 1 || m > 16 || slices < 1 || slices > kMaxSlices || n % kTileRows || k % kChunk)
         return cudaErrorInvalidValue;
     const int q = width == 1 ? 1 : width == 2 ? 2 : (k % (2 * kChunk) == 0 ? 2 : 1);
@@ -371,13 +382,16 @@ cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, co
         a.rawbase = w->rawbase;
         a.rawexp = w->rawexp;
         a.palette = make_palette16(w->palette);
+        a.w_stable = w_stable ? 1 : 0;
     }
     const int nt = m > 8 ? 2 : 1;
     const unsigned grid = unsigned(n / kTileRows);
     const unsigned block = unsigned(slices * 32);
     const size_t smem = size_t(2 * a.flag_words) * 4 + (slices > 1 ? size_t(slices) * 32 * 4 * nt * 4 : 0);
     if (smem > size_t(kMaxSmem)) return cudaErrorInvalidValue;
-#define UW_MMA_LAUNCH(P_, N_, Q_) k_gemv_mma<P_, N_, Q_><<<grid, block, smem, stream>>>(a)
+    cudaError_t err = cudaSuccess;
+#define UW_MMA_LAUNCH(P_, N_, Q_) \
+    err = launch_pdl(a.w_stable != 0, k_gemv_mma<P_, N_, Q_>, dim3(grid), dim3(block), smem, stream, a)
     if (pal) {
         if (q == 2) { if (nt == 2) UW_MMA_LAUNCH(true, 2, 2); else UW_MMA_LAUNCH(true, 1, 2); }
         else { if (nt == 2) UW_MMA_LAUNCH(true, 2, 1); else UW_MMA_LAUNCH(true, 1, 1); }
@@ -386,7 +400,7 @@ cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, co
         else { if (nt == 2) UW_MMA_LAUNCH(false, 2, 1); else UW_MMA_LAUNCH(false, 1, 1); }
     }
 #undef UW_MMA_LAUNCH
-    return cudaGetLastError();
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_gemv_mma_batched(const MmaItem *items, int n_items, int slices, int width,

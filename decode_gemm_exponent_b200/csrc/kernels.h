@@ -1,5 +1,6 @@
 // kernels.h -- host-side launch interface of the libuw CUDA kernels (internal).
 #pragma once
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -79,7 +80,7 @@ cudaError_t launch_gemv_fma(const uint16_t *x, int m, const uint16_t *w_bf16, co
 // 2: 32, 0: 32 when k is a multiple of 128.  pal_plane == nullptr: plain BF16.
 cudaError_t launch_gemv_mma(const uint16_t *x, int m, const uint16_t *w_bf16, const uw_dmat *w,
                             const uint8_t *pal_plane, int64_t n, int64_t k, float *y, int slices, int width,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool w_stable = false);
 
 // The warp-MMA fused kernel over many matrices in as few launches as
 // possible (32 matrices per launch; items with m == 0 are skipped): item i
@@ -96,6 +97,31 @@ cudaError_t launch_gemv_mma_batched(const MmaItem *items, int n_items, int slice
                                     cudaStream_t stream);
 
 // tcgen05 GEMM (Unweight page §七, reconstructive matmul), token tile `bn`.
+// Launch, with programmatic stream serialization when `early` is set: the
+// kernel calls pdl_wait before touching data an earlier kernel on the stream
+// may own, so its CTAs can be scheduled, and start on what no kernel writes,
+// while that kernel drains.  Measured on a step of 12 matmuls (Llama-3.1-8B
+// MLP layer, M = 1, 4, 16, 64), early launches pay only for kernels that have
+// such work -- the fused kernels on the blob's own planes: +11% -- while
+// kernels that must wait at their first instruction ran slower launched early
+// (the BF16 twins: -11%; the split-K reduce: -4% on the step), so those are
+// launched as usual.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(bool early, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = early ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 struct TcLaunch {
     const uint16_t *x;         // [m, k] BF16
     int64_t m, n, k;
@@ -106,6 +132,8 @@ struct TcLaunch {
     float *partial;            // [split_k, m, n] when split_k > 1; stream-K: partial tiles
     uint32_t *sk_counters;     // stream-K: one counter per tile (zero between calls)
     bool huffman;              // stream-K fused: decode the palette indices from the Huffman stream
+    bool w_stable;             // fused: the compressed planes are the blob's (no kernel writes them),
+                               // so they may be read before the previous kernel on the stream ends
     int bn, split_k, stages;
     uint32_t debug_flags;
     uint64_t timeout_ns;

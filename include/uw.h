@@ -38,6 +38,14 @@
  *     allocates no device memory.  It owns only the host blobs that uw_encode
  *     returns; free them with uw_blob_free.
  *   - Calls are thread-safe as long as no two calls write the same buffers.
+ *   - Early start: a direct-palette matmul on the blob's own 4-bit plane
+ *     (pipeline 4, no separate palette plane) with the warp-MMA or tcgen05
+ *     kernel is launched with programmatic stream serialization.  Its CTAs
+ *     may be scheduled, and may read the blob's compressed planes, while the
+ *     previous libuw kernel on the stream is still draining; X is read, and
+ *     Y and the workspace are written, only after that kernel has completed.
+ *     Kernels of other libraries on the stream end before it starts, as
+ *     usual.  The library never writes a blob's device copy.
  */
 #ifndef UW_H
 #define UW_H
