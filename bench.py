@@ -18,7 +18,8 @@ value  = sum over the step's matmuls of 2*N*K (uncompressed BF16 weight bytes)
          / step time  [GB/s], inputs resident in HBM, CUDA events, max over ranks.
 e2e    = the same, with X copied from pinned host memory and Y read back to
          pinned host memory inside the timed region, through the C ABI (copies
-         on their own streams, ordered by events, overlapping the matmuls).
+         on their own streams, ordered by events; inputs and results double-
+         buffered, so a step's copies overlap the neighbouring steps' matmuls).
 plain_bf16: the same 12 calls with the same plans on uncompressed BF16 weights.
 large_m: the same layer at M = 256, 512 and 1024 (fused TFLOP/s against the
          dense BF16 tensor peak, next to decode + GEMM and uncompressed BF16).
@@ -570,43 +571,47 @@ def run_gpu(args, rank, world):
 
     # ---- end-to-end through the C ABI with pinned host buffers.  As a
     # serving loop would, the copies run on their own streams ordered by
-    # events: a step's inputs go up on one copy stream into one of two device
-    # input sets (so they can be sent while the previous step still reads the
-    # other set), every result comes down on another copy stream as soon as
-    # its matmul ends, and the step's matmuls wait only for their inputs.
+    # events, and inputs and results are double-buffered: a step's inputs go
+    # up on one copy stream into one of two device input sets (while the
+    # previous step still reads the other), its 12 matmuls run back to back
+    # into one of two result sets (so the early start of each matmul is not
+    # broken by event operations between them), and the step's results come
+    # down on another copy stream while the next step computes.
     hx = {(c["m"], c["mat"].k): c["x"].cpu().pin_memory() for c in calls}
     hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
     h2d = sum(t.numel() * 2 for t in hx.values())
     d2h = sum(t.numel() * 4 for t in hy)
     xsets = [{key: xs[key[0]][key[1]] for key in hx}, {key: xs[key[0]][key[1]].clone() for key in hx}]
+    ysets = [[c["y"] for c in calls], [torch.empty_like(c["y"]) for c in calls]]
     copy_in, copy_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     mk = lambda: torch.cuda.Event()
     x_ready = [mk() for _ in range(args.steps)]
     x_free = [mk() for _ in range(args.steps)]
-    y_ready = [[mk() for _ in calls] for _ in range(args.steps)]
-    y_free = [[mk() for _ in calls] for _ in range(args.steps)]
+    y_ready = [mk() for _ in range(args.steps)]
+    y_free = [mk() for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for s in range(args.steps):
-        xset = xsets[s & 1]
+        xset, yset = xsets[s & 1], ysets[s & 1]
         copy_in.wait_event(e0 if s < 2 else x_free[s - 2])     # matmuls of step s-2 read this set
         with torch.cuda.stream(copy_in):
             for key, t in hx.items():
                 xset[key].copy_(t, non_blocking=True)
         x_ready[s].record(copy_in)
         stream.wait_event(x_ready[s])
-        for i, (c, h) in enumerate(zip(calls, hy)):
-            if s > 0:
-                stream.wait_event(y_free[s - 1][i])              # last step's result is on the host
-            c["mat"].matmul(xset[(c["m"], c["mat"].k)], c["plan"], y=c["y"], ws=c["ws"])
-            y_ready[s][i].record(stream)
-            copy_out.wait_event(y_ready[s][i])
-            with torch.cuda.stream(copy_out):
-                h.copy_(c["y"], non_blocking=True)
-            y_free[s][i].record(copy_out)
+        if s >= 2:
+            stream.wait_event(y_free[s - 2])                    # step s-2's results (this set) are on the host
+        for c, y in zip(calls, yset):
+            c["mat"].matmul(xset[(c["m"], c["mat"].k)], c["plan"], y=y, ws=c["ws"])
         x_free[s].record(stream)
+        y_ready[s].record(stream)
+        copy_out.wait_event(y_ready[s])
+        with torch.cuda.stream(copy_out):
+            for h, y in zip(hy, yset):
+                h.copy_(y, non_blocking=True)
+        y_free[s].record(copy_out)
     stream.wait_stream(copy_out)                                # every result is on the host
     e1.record(stream)
     torch.cuda.synchronize()
