@@ -21,8 +21,13 @@
 //   compressed ring (CS stages): sign/mantissa tile (64-byte swizzle),
 //     palette tile (32-byte swizzle) and the exponents of the tile's raw rows
 //     (one 64-byte slot per row); freed as soon as the rebuild has read it;
-//   W ring (4 stages for BN <= 64, else 2): rebuilt BF16 W tiles (128-byte
-//     swizzle, K-major); freed by the MMA's commit;
+//   W ring (4 stages for BN <= 64, else 2): rebuilt BF16 W tiles, freed by
+//     the MMA's commit.  With one token tile per CTA the ring lives in tensor
+//     memory, 32 columns per K-step after the accumulator: each rebuild
+//     thread writes its row's 32 BF16 pairs to its lane (tcgen05.st), and
+//     the MMA takes A from there, so W never goes through shared memory;
+//     with two token tiles the accumulators fill TMEM and the ring is in
+//     shared memory (128-byte swizzle, K-major);
 //   X ring (8 / 4 / 2 stages): X tiles, freed by the MMA's commit.  With a
 //   256-token tile and more than 256 tokens, a CTA owns two token tiles: an
 //   X stage holds both, the MMA thread issues each K-step for both against
@@ -248,9 +253,20 @@ struct FusedCfg {
     static constexpr int kRAW = kBM * kGroup;           // raw exponents, one 64-byte slot per row
     static constexpr int kCStage = kSM + kPL + kRAW;    // compressed ring stage
     static constexpr int kOffPL = kSM, kOffRAW = kSM + kPL;
-    static constexpr uint32_t kTmemCols = uint32_t(TT) * (BN < 32 ? 32u : uint32_t(BN));
+    // one token tile per CTA: the rebuilt W ring lives in tensor memory (32
+    // columns per K-step after the accumulator) and the MMA takes A from
+    // there; with two token tiles the accumulators fill TMEM and W stays in
+    // shared memory
+    static constexpr bool kWInTmem = TT == 1;
+    static constexpr uint32_t kAccCols = BN < 32 ? 32u : uint32_t(BN);
+    static constexpr uint32_t kWCol0 = kAccCols;                      // first W column (TMEM ring)
+    static constexpr uint32_t kTmemUsed = kWInTmem ? kAccCols + uint32_t(kWS) * 32u : uint32_t(TT) * kAccCols;
+    static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                        : kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kWSmem = kWInTmem ? 0 : kWS * kW;              // W ring bytes in shared memory
     static_assert(kW % 1024 == 0 && kX % 1024 == 0 && kCStage % 1024 == 0, "1024-byte alignment");
-    static_assert(kTmemCols <= 512, "accumulators exceed TMEM");
+    static_assert(kTmemUsed <= 512, "accumulators and W ring exceed TMEM");
+    static_assert(kWCol0 >= uint32_t(BN), "the W ring starts after the accumulator");
 };
 
 constexpr int kRawProducers = 4;      // warps; lane l of warp j owns tile row 32 j + l
@@ -270,7 +286,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     constexpr int WS = C::kWS, XS = C::kXS;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *wring = align1024(smem_dyn);
-    uint8_t *xring = wring + WS * C::kW;
+    uint8_t *xring = wring + C::kWSmem;
     uint8_t *cring = xring + XS * C::kXT;
     const int CS = a.stages;                      // compressed stages (even)
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(cring + size_t(CS) * C::kCStage);   // [128][bw]
@@ -396,10 +412,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                      mbar_wait(&w_full[ws], uint32_t(ks / WS) & 1u, T);
                 if (!ok) break;
                 tc_fence_after();
+                if constexpr (C::kWInTmem) {
+                    constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+                    const uint32_t a0 = tmem + C::kWCol0 + uint32_t(ws) * 32u;
+                    const uint32_t sb = smem_addr(xring + size_t(xs) * C::kXT);
 #pragma unroll
-                for (int t = 0; t < TT; t++)
-                    mma_kstep<BN>(tmem + uint32_t(t * BN), smem_addr(wring + size_t(ws) * C::kW),
-                                  smem_addr(xring + size_t(xs) * C::kXT + size_t(t) * C::kX), ks == 0);
+                    for (int kk = 0; kk < kBK / 16; kk++)   // 8 columns = 16 K per MMA
+                        tc_mma_bf16_ta(tmem, a0 + 8u * kk, smem_desc_k128(sb + 32 * kk), idesc,
+                                       (ks != 0 || kk) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < TT; t++)
+                        mma_kstep<BN>(tmem + uint32_t(t * BN), smem_addr(wring + size_t(ws) * C::kW),
+                                      smem_addr(xring + size_t(xs) * C::kXT + size_t(t) * C::kX), ks == 0);
+                }
                 tc_commit(&w_empty[ws]);
                 tc_commit(&x_empty[xs]);
             }
@@ -479,6 +505,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const uint8_t *plrow = st + C::kOffPL + r * 32;
             uint8_t *wrow = wring + size_t(ws) * C::kW + r * 128;
             const bool raw = (bm[ks >> 5] >> (ks & 31)) & 1u;
+            uint32_t wv[32];                   // TMEM ring: BF16 pairs of the row in K order
+            if constexpr (C::kWInTmem) tc_fence_after();   // the slot's previous MMAs are done
 #pragma unroll
             for (int h = 0; h < 2; h++) {      // two halves of the row, 32 weights each
                 const uint4 s0 = *reinterpret_cast<const uint4 *>(smrow + (((2 * h) ^ sw64) << 4));
@@ -498,12 +526,33 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     pal_rot(p.w, a.pal, rv[6], rv[7]);
                 }
                 const int c0 = 4 * h;
-                *reinterpret_cast<uint4 *>(wrow + (((c0 + 0) ^ sw128) << 4)) = join8(rv[0], rv[1], s0.x, s0.y);
-                *reinterpret_cast<uint4 *>(wrow + (((c0 + 1) ^ sw128) << 4)) = join8(rv[2], rv[3], s0.z, s0.w);
-                *reinterpret_cast<uint4 *>(wrow + (((c0 + 2) ^ sw128) << 4)) = join8(rv[4], rv[5], s1.x, s1.y);
-                *reinterpret_cast<uint4 *>(wrow + (((c0 + 3) ^ sw128) << 4)) = join8(rv[6], rv[7], s1.z, s1.w);
+                const uint4 o0 = join8(rv[0], rv[1], s0.x, s0.y), o1 = join8(rv[2], rv[3], s0.z, s0.w);
+                const uint4 o2 = join8(rv[4], rv[5], s1.x, s1.y), o3 = join8(rv[6], rv[7], s1.z, s1.w);
+                if constexpr (C::kWInTmem) {
+                    const uint4 o[4] = {o0, o1, o2, o3};
+#pragma unroll
+                    for (int c = 0; c < 4; c++) {
+                        wv[16 * h + 4 * c + 0] = o[c].x;
+                        wv[16 * h + 4 * c + 1] = o[c].y;
+                        wv[16 * h + 4 * c + 2] = o[c].z;
+                        wv[16 * h + 4 * c + 3] = o[c].w;
+                    }
+                } else {
+                    *reinterpret_cast<uint4 *>(wrow + (((c0 + 0) ^ sw128) << 4)) = o0;
+                    *reinterpret_cast<uint4 *>(wrow + (((c0 + 1) ^ sw128) << 4)) = o1;
+                    *reinterpret_cast<uint4 *>(wrow + (((c0 + 2) ^ sw128) << 4)) = o2;
+                    *reinterpret_cast<uint4 *>(wrow + (((c0 + 3) ^ sw128) << 4)) = o3;
+                }
             }
-            fence_proxy_async_smem();
+            if constexpr (C::kWInTmem) {
+                // the warp writes its 32 rows (lanes 32 q ..) of the slot's 32 columns
+                __syncwarp();
+                tmem_st32(tmem + (uint32_t(q * 32) << 16) + C::kWCol0 + uint32_t(ws) * 32u, wv);
+                tmem_st_wait();
+                tc_fence_before();
+            } else {
+                fence_proxy_async_smem();
+            }
             mbar_arrive(&c_empty[cs]);
             mbar_arrive(&w_full[ws]);
         }
@@ -643,12 +692,12 @@ cudaError_t launch_fused(const TcLaunch &p, cudaStream_t stream) {
     a.k = p.k;
     split_k_slices(p, a);
     const int bw = (a.ks_per_split + 31) / 32;     // raw bitmap words per row
-    const int fixed = C::kWS * C::kW + C::kXS * C::kXT + 1024 + fused_tail(8, C::kWS, C::kXS, bw);
+    const int fixed = C::kWSmem + C::kXS * C::kXT + 1024 + fused_tail(8, C::kWS, C::kXS, bw);
     int max_cs = (kMaxSmem - fixed) / C::kCStage;
     max_cs = std::min(8, max_cs) & ~1;      // even: each rebuild group owns every other stage
     int cs = (p.stages <= 0 || p.stages > max_cs) ? max_cs : (p.stages & ~1);
     if (cs < 2) return cudaErrorInvalidValue;
-    const size_t smem = size_t(C::kWS) * C::kW + size_t(C::kXS) * C::kXT + size_t(cs) * C::kCStage + 1024 +
+    const size_t smem = size_t(C::kWSmem) + size_t(C::kXS) * C::kXT + size_t(cs) * C::kCStage + 1024 +
                         fused_tail(cs, C::kWS, C::kXS, bw);
     CUtensorMap mx, msm, mpl;
     if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2,
