@@ -410,7 +410,8 @@ def launches_per_call(plan):
 
 def kernel_name(plan):
     return {1: "fma_gemv", 3: "mma_gemv_s%d_w%d" % (plan.bn, plan.stages),
-            4: "tc_sk_bn%d" % plan.bn}.get(plan.kernel, "tcgen05_bn%d" % plan.bn)
+            4: "tc_sk_bn%d" % plan.bn, 5: "mma_sk_w%d_s%d" % (plan.bn, plan.stages)}.get(
+                plan.kernel, "tcgen05_bn%d" % plan.bn)
 
 
 def kernel_group(plan):
@@ -472,10 +473,14 @@ def run_gpu(args, rank, world):
             j = all_ms.index(m)
             for i, mat in enumerate(mats):
                 p = plans[i][j]
-                nb = max(mat.workspace_bytes(m, p), mat.workspace_bytes(m, same_plan(uw, p, 1)))
-                ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=dev)
+                ws = torch.zeros(max(mat.workspace_bytes(m, p), 256), dtype=torch.uint8, device=dev)
+                # the BF16 twin gets a workspace of its own: a stream-K plan keeps its tile
+                # counters where a preprocessing pipeline's output would lie in a shared one
+                ws_plain = torch.zeros(max(mat.workspace_bytes(m, same_plan(uw, p, 4)), 256), dtype=torch.uint8,
+                                       device=dev)
                 y = torch.empty(m, mat.n, dtype=torch.float32, device=dev)
-                calls.append(dict(mat=mat, m=m, plan=p, ws=ws, y=y, x=xs[m][mat.k], name=PROJ[i][0],
+                calls.append(dict(mat=mat, m=m, plan=p, ws=ws, ws_plain=ws_plain, y=y, x=xs[m][mat.k],
+                                  name=PROJ[i][0],
                                   w=plain_w[i]))
         return calls
 
@@ -486,7 +491,7 @@ def run_gpu(args, rank, world):
         c["mat"].matmul(c["x"], c["plan"], y=c["y"], ws=c["ws"])
 
     def issue_plain(c):
-        uw.matmul_bf16(c["x"], c["w"], c["plan"], y=c["y"], ws=c["ws"])
+        uw.matmul_bf16(c["x"], c["w"], c["plan"], y=c["y"], ws=c["ws_plain"])
 
     def barrier():
         if world > 1:
@@ -546,7 +551,11 @@ def run_gpu(args, rank, world):
     lsteps = max(3, args.steps // 4)
     for m in MS_LARGE:
         cs = [c for c in lcalls if c["m"] == m]
-        dec = [dict(c, plan=same_plan(uw, c["plan"], 1)) for c in cs]
+        dec = []
+        for c in cs:
+            p1 = same_plan(uw, c["plan"], 1)
+            dec.append(dict(c, plan=p1, ws=torch.zeros(max(c["mat"].workspace_bytes(m, p1), 256),
+                                                        dtype=torch.uint8, device=dev)))
         for c in cs + dec:
             issue(c)
         for c in cs:
@@ -678,12 +687,13 @@ def case_kernel(argv):
     per launch.  Under ncu, `-s 1 -c 1` captures the second launch."""
     ap = argparse.ArgumentParser(prog="bench.py --case kernel")
     ap.add_argument("--kernel", required=True,
-                    choices=["decode", "exp_decode", "transcode", "fma", "tc", "mma", "sk",
-                             "plain_fma", "plain_tc", "plain_mma", "plain_sk"])
+                    choices=["decode", "exp_decode", "transcode", "fma", "tc", "mma", "sk", "mma_sk",
+                             "plain_fma", "plain_tc", "plain_mma", "plain_sk", "plain_mma_sk"])
     ap.add_argument("--n", type=int, default=28672)
     ap.add_argument("--k", type=int, default=8192)
     ap.add_argument("--m", type=int, default=1)
-    ap.add_argument("--bn", type=int, default=0, help="TC token tile, FMA rows per warp or MMA K slices")
+    ap.add_argument("--bn", type=int, default=0,
+                    help="TC token tile, FMA rows per warp, MMA K slices or MMA_SK warps per SM")
     ap.add_argument("--split", type=int, default=1)
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--pipeline", type=int, default=4, help="fused kernels: 4 (palette plane) or 3 / 2")
@@ -723,6 +733,8 @@ def case_kernel(argv):
         plan = uw.make_plan(a.pipeline, uw.KERNEL_MMA, a.bn or 2, 1, a.stages)
     elif kind == "sk":
         plan = uw.make_plan(a.pipeline, uw.KERNEL_TC_SK, a.bn or 16, 1, a.stages)
+    elif kind == "mma_sk":
+        plan = uw.make_plan(a.pipeline, uw.KERNEL_MMA_SK, a.bn or 8, 1, a.stages)
     else:
         plan = uw.make_plan(a.pipeline, uw.KERNEL_TC, a.bn or 16, a.split, a.stages)
     preprocessing = a.kernel in ("decode", "exp_decode", "transcode")
@@ -1010,7 +1022,8 @@ def case_sweep70b(argv):
             yp = torch.empty_like(yf)
             us_f = timed(lambda: mat.matmul(x, p, y=yf, ws=ws))
             pp = same_plan(uw, p, 4)
-            us_p = timed(lambda: uw.matmul_bf16(x, wd, pp, y=yp, ws=ws))
+            ws_plain = torch.zeros(max(mat.workspace_bytes(m, pp), 256), dtype=torch.uint8, device="cuda")
+            us_p = timed(lambda: uw.matmul_bf16(x, wd, pp, y=yp, ws=ws_plain))
             same = torch.equal(yf.view(torch.int32), yp.view(torch.int32))
             if mat.device_status() != 0:
                 raise RuntimeError("kernel status")

@@ -39,6 +39,8 @@ uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
             return UW_ERR_INVALID_ARG;
     } else if (p->kernel == UW_KERNEL_TC_SK) {
         if (!valid_bn_tc(p->bn) || p->split_k != 1 || p->stages < 0 || p->stages > 8) return UW_ERR_INVALID_ARG;
+    } else if (p->kernel == UW_KERNEL_MMA_SK) {
+        if (m > 16 || k % 128 || p->split_k != 1 || gemv_sk_stages(p->bn, p->stages, m) == 0) return UW_ERR_INVALID_ARG;
     } else {
         return UW_ERR_INVALID_ARG;
     }
@@ -50,6 +52,10 @@ uw_status check_plan(const uw_plan *p, int64_t m, int64_t k) {
 // stream-K kernel its tile counters (unless the caller keeps them apart,
 // `own_counters`) followed by its partial tiles.
 uint64_t partial_bytes(int64_t m, int64_t n, int64_t k, const uw_plan *p, bool own_counters = false) {
+    if (p->kernel == UW_KERNEL_MMA_SK) {
+        const GemvSkGeometry g = gemv_sk_geometry(m, n, k, p->bn);
+        return (own_counters ? 0 : g.counter_bytes) + g.partial_bytes;
+    }
     if (p->kernel == UW_KERNEL_TC_SK) {
         const SkGeometry g = sk_geometry(m, n, k, p->bn);
         return (own_counters ? 0 : g.counter_bytes) + g.partial_bytes;
@@ -70,6 +76,30 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
     if (plan->kernel == UW_KERNEL_MMA)
         return cuda_status(
             launch_gemv_mma(x, int(m), w_bf16, w, pal, n, k, y, plan->bn, plan->stages, stream, w_stable));
+    if (plan->kernel == UW_KERNEL_MMA_SK) {
+        uint8_t *base = reinterpret_cast<uint8_t *>(partial);
+        if (!base) return UW_ERR_WORKSPACE;
+        GemvSkLaunch g{};
+        g.x = x;
+        g.m = m;
+        g.n = n;
+        g.k = k;
+        g.w_bf16 = w_bf16;
+        g.w = w;
+        g.pal = pal;
+        g.y = y;
+        g.warps = plan->bn;
+        g.stages = plan->stages;
+        g.w_stable = w_stable;
+        if (sk_counters) {
+            g.counters = sk_counters;
+            g.partial = partial;
+        } else {
+            g.counters = reinterpret_cast<uint32_t *>(base);
+            g.partial = reinterpret_cast<float *>(base + gemv_sk_geometry(m, n, k, plan->bn).counter_bytes);
+        }
+        return cuda_status(launch_gemv_sk(g, stream));
+    }
     TcLaunch t{};
     t.x = x;
     t.m = m;
@@ -239,7 +269,9 @@ extern "C" uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw
 namespace uw {
 
 uint64_t sk_counter_bytes(int64_t m, int64_t n, int64_t k, const uw_plan *plan) {
-    if (!plan || plan->kernel != UW_KERNEL_TC_SK || m <= 0) return 0;
+    if (!plan || m <= 0) return 0;
+    if (plan->kernel == UW_KERNEL_MMA_SK) return gemv_sk_geometry(m, n, k, plan->bn).counter_bytes;
+    if (plan->kernel != UW_KERNEL_TC_SK) return 0;
     return sk_geometry(m, n, k, plan->bn).counter_bytes;
 }
 

@@ -604,26 +604,33 @@ __device__ __forceinline__ void sk_body(const CUtensorMap *tmX, const CUtensorMa
             named_bar_sync(1, 128);
             if (*last_flag) {
                 __threadfence();
-                if (row < a.n) {
+                // every row of every piece is read and then zeroed (rows past
+                // n too, which the pieces hold as well), so that a completed
+                // call leaves its whole scratch zero: a later call whose tile
+                // counters lie where this call's partial tiles were finds them
+                // at zero
 #pragma unroll 1
-                    for (int c0 = 0; c0 < BN; c0 += 8) {
-                        float acc[8];
+                for (int c0 = 0; c0 < BN; c0 += 8) {
+                    float acc[8];
 #pragma unroll
-                        for (int j = 0; j < 8; j++) acc[j] = 0.f;
-                        for (int c = ca; c <= cb; c++) {
-                            const int sl = (t == sk_unit0(c, a.units, a.G) / a.S) ? 0 : 1;
-                            const float *pin = a.partial + (int64_t(2 * c + sl) * BN + c0) * kBM + r;
-                            float v[8];
+                    for (int j = 0; j < 8; j++) acc[j] = 0.f;
+                    for (int c = ca; c <= cb; c++) {
+                        const int sl = (t == sk_unit0(c, a.units, a.G) / a.S) ? 0 : 1;
+                        float *pin = a.partial + (int64_t(2 * c + sl) * BN + c0) * kBM + r;
+                        float v[8];
 #pragma unroll
-                            for (int j = 0; j < 8; j++) v[j] = __ldcg(pin + j * kBM);
-                            if (c == ca) {
+                        for (int j = 0; j < 8; j++) v[j] = __ldcg(pin + j * kBM);
 #pragma unroll
-                                for (int j = 0; j < 8; j++) acc[j] = v[j];
-                            } else {
+                        for (int j = 0; j < 8; j++) __stcg(pin + j * kBM, 0.f);
+                        if (c == ca) {
 #pragma unroll
-                                for (int j = 0; j < 8; j++) acc[j] += v[j];
-                            }
+                            for (int j = 0; j < 8; j++) acc[j] = v[j];
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 8; j++) acc[j] += v[j];
                         }
+                    }
+                    if (row < a.n) {
 #pragma unroll
                         for (int j = 0; j < 8; j++) {
                             const int64_t tok = m0 + c0 + j;
@@ -1158,6 +1165,8 @@ cudaError_t launch_bn(const TcLaunch &p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int sm_count() { return device_sms(); }
 
 SkGeometry sk_geometry(int64_t m, int64_t n, int64_t k, int bn) {
     SkGeometry g{};

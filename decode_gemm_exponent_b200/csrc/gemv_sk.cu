@@ -1,0 +1,525 @@
+// gemv_sk.cu -- persistent stream-K form of the warp-MMA skinny matmul
+// Y = X * W^T for m <= 16 tokens (Unweight page §七, the reconstructive
+// matmul, in the small-batch regime of §十 where the job is an HBM stream).
+//
+// Why a second form of the warp-MMA kernel.  The one-tile-per-CTA form
+// (gemv_mma.cu) keeps the next steps' loads in flight in a register ring,
+// about 3 KB per warp, so at the occupancy that ring allows an SM has a few
+// tens of KB of W requested at any time, which at HBM's loaded latency caps
+// the stream well below the HBM peak; and an 8B gate projection's 896 tiles
+// make two full waves of CTAs plus a nearly empty third one.  Here:
+//  - the warp copies each unit's compressed W and the chunk's X rows into
+//    shared memory with cp.async (16 bytes a copy, L1 bypassed), so a ring of
+//    several units per warp costs no registers, an SM keeps ~100 KB in
+//    flight, and the MMAs never wait on X from L2;
+//  - one CTA per SM of `S` warps, and every warp of the grid owns an equal
+//    contiguous run of units (16-row tile, 128-wide K chunk), in tile-major
+//    order, so every warp streams the same number of bytes: no tail wave;
+//  - a tile cut between warps is finished by the warp that completes its
+//    last piece: each piece's fp32 MMA fragments go to the workspace, an
+//    atomic counter per tile counts the pieces, and the warp that brings it
+//    to the number of pieces adds them in warp order (= K order), so the
+//    result does not depend on timing, and zeroes each piece after reading
+//    it, so that a completed call leaves its whole scratch (counters and
+//    pieces) zero.  No warp ever waits for another one: there are no
+//    barriers and no spin waits in this kernel.
+// Per unit, lane (g, c) = (lane / 4, lane % 4) handles rows g and g + 8 of
+// the tile and weights [32c, 32c + 32) of the chunk, with the same fragment
+// map as the one-tile kernel at 32 weights per lane (MMA K-step j, thread c,
+// K slots {2c, 2c+1, 2c+8, 2c+9} <- weights 32c + 4j + {0, 1, 2, 3}; X uses
+// the same map, so every product is formed once).  The copies are not made
+// by the lanes that use the data: each copy instruction of a warp reads whole
+// 128-byte lines (a row's 128 sign/mantissa bytes take 8 lanes, its 64
+// palette bytes 4), and after its copies have landed every lane passes a
+// warp barrier before reading the slot, whose rows are bank-swizzled.  A raw
+// group's quarter is copied from the raw plane instead of the palette plane
+// by the lane that would copy its palette bytes; the warp learns which
+// groups are raw from one bitmap lookup per lane and a ballot.  The fused
+// and plain kernels differ only in these copies and the rebuild, so their
+// outputs are bit-identical.
+#include <algorithm>
+#include <mutex>
+
+#include "device_common.cuh"
+#include "kernels.h"
+#include "uw_format.h"
+
+namespace uw {
+namespace {
+
+using namespace dev;
+
+constexpr int kRows = 16;                      // W rows per tile (the MMA's M)
+constexpr int kChunkK = 128;                   // weights along K per unit
+constexpr int kMaxWarps = 16;
+constexpr int kMaxStages = 8;
+constexpr int kMaxSmem = 227 * 1024;
+
+struct SkArgs {
+    const uint16_t *x;         // [m, k] BF16
+    const uint16_t *w_bf16;    // plain: [n, k] BF16
+    const uint8_t *sm;         // fused: sign/mantissa plane
+    const uint8_t *pal;        // fused: 4-bit plane
+    const uint32_t *flagbits;  // fused: raw-group bitmap
+    const uint32_t *rawbase;   // fused: raw groups before each bitmap word
+    const uint8_t *rawexp;     // fused: exponents of the raw groups
+    Palette16 palette;
+    int64_t n, k;
+    int64_t cpr;               // chunks per row (k / 128)
+    int64_t units;             // tiles * cpr
+    int64_t warps;             // warps of the grid that own units (<= units)
+    float *y;                  // [m, n]
+    float *partial;            // [2 * warps][NT][32 lanes][4] fp32 fragments
+    uint32_t *counters;        // [tiles], zero between calls
+    int m;
+    int stages;                // ring slots per warp (2..8)
+    int slot_bytes;            // bytes of one ring slot (W and the chunk's X rows)
+    int w_stable;              // fused: planes no kernel writes (read before pdl_wait)
+};
+
+// first unit of warp w
+__device__ __forceinline__ int64_t unit0(int64_t w, int64_t units, int64_t warps) { return w * units / warps; }
+// the warp whose run holds unit u (every run is non-empty: warps <= units)
+__device__ __forceinline__ int64_t owner(int64_t u, int64_t units, int64_t warps) {
+    return ((u + 1) * warps - 1) / units;
+}
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most n of this thread's copy groups are still in flight
+__device__ __forceinline__ void cp_wait(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    }
+}
+// 16-byte load from the ring (a plain load through a pointer into shared
+// memory: the compiler keeps it after the copy waits and warp barriers,
+// which clobber memory, and schedules it freely against the arithmetic and
+// MMAs around it)
+__device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t w4(const uint4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// Byte offsets inside a ring slot.
+//  - Fused: row r's 128 sign/mantissa bytes at r * 128, its 64 palette bytes
+//    at kPalOff + r * 64, and the exponents of its raw groups at kRawOff +
+//    r * 128 (one byte per weight; only raw groups' bytes are written).  The
+//    16-byte pieces of a 128-byte row sit at piece ^ (r & 1), so that rows g
+//    and g + 1, which a quarter warp reads together, fall on different banks.
+//  - Plain: row r's 256 BF16 bytes at row256(r, piece).
+//  - X (both): token row r's 256 bytes of the chunk at kXOff + row256(r, piece).
+//  row256 spaces rows 288 bytes apart and pieces 8-15 16 bytes further, so
+//  that the 8 lanes of a quarter warp, which read pieces 4c .. 4c + 3 of rows
+//  g and g + 1 (c = 0..3), hit 8 different bank groups, and every lane's 64
+//  bytes stay contiguous (its four loads differ by immediate offsets).
+constexpr int kPalOff = 16 * 128;
+constexpr int kRawOff = kPalOff + 16 * 64;
+constexpr int kXOff = kRawOff + 16 * 128;
+constexpr int kRow256 = 288;
+__host__ __device__ constexpr int slot_bytes(int xrows) { return kXOff + xrows * kRow256; }
+__device__ __forceinline__ uint32_t sw128(int r, int j) { return uint32_t(r * 128 + ((j ^ (r & 1)) << 4)); }
+__device__ __forceinline__ uint32_t row256(int r, int j) { return uint32_t(r * kRow256 + j * 16 + (j >= 8 ? 16 : 0)); }
+
+// One row's 32 weights (quarter c of the chunk) from a ring slot -> 16 BF16
+// pairs (weights 2i, 2i + 1 in pair i).  `sm0`, `sm1`: the row's two
+// sign/mantissa pieces of the quarter (the same offsets inside the raw
+// region hold its raw exponents); `pal`: its palette piece.
+__device__ __forceinline__ void rebuild_pal(const uint8_t *slot, uint32_t sm0, uint32_t sm1, uint32_t pal, bool raw,
+                                            const Palette16 &P, uint32_t (&w)[16]) {
+    const uint4 s0 = lds128(slot + sm0), s1 = lds128(slot + sm1);
+    uint32_t e[8];   // rotated exponent bytes, 4 weights per word
+    if (raw) {
+        const uint4 b0 = lds128(slot + kRawOff + sm0), b1 = lds128(slot + kRawOff + sm1);
+#pragma unroll
+        for (int i = 0; i < 4; i++) e[i] = rot4(w4(b0, i));
+#pragma unroll
+        for (int i = 0; i < 4; i++) e[4 + i] = rot4(w4(b1, i));
+    } else {
+        const uint4 b0 = lds128(slot + pal);
+#pragma unroll
+        for (int i = 0; i < 4; i++) pal_rot(w4(b0, i), P, e[2 * i], e[2 * i + 1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) join4(e[i], w4(s0, i), w[2 * i], w[2 * i + 1]);
+#pragma unroll
+    for (int i = 0; i < 4; i++) join4(e[4 + i], w4(s1, i), w[8 + 2 * i], w[8 + 2 * i + 1]);
+}
+
+// 16 consecutive words (64 contiguous bytes) from shared memory
+__device__ __forceinline__ void lds64b(const uint8_t *addr, uint32_t (&w)[16]) {
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        const uint4 v = lds128(addr + q * 16);
+        w[4 * q] = v.x;
+        w[4 * q + 1] = v.y;
+        w[4 * q + 2] = v.z;
+        w[4 * q + 3] = v.w;
+    }
+}
+
+template <bool PAL, int NT>   // NT: 8-token tiles (1: m <= 8, 2: m <= 16)
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int S = blockDim.x >> 5;
+    // the next kernel on the stream may be scheduled now
+    pdl_trigger();
+    const int64_t gw = int64_t(blockIdx.x) * S + warp;
+    if (gw >= a.warps) return;   // the last CTA's spare warps
+    const int64_t u_begin = unit0(gw, a.units, a.warps), u_end = unit0(gw + 1, a.units, a.warps);
+    const int nu = int(u_end - u_begin);
+    // with planes no kernel writes, W is requested before the previous
+    // kernel on the stream has ended, X only after it
+    const bool defer_x = a.w_stable != 0;
+    if (!defer_x) pdl_wait();
+
+    const int stages = a.stages, slot_b = a.slot_bytes, xrows = a.m;
+    const uint32_t ring = smem_addr(smem) + uint32_t(warp * stages * slot_b);
+    const uint32_t k = uint32_t(a.k), gpr = k / 64;
+    const int cpr = int(a.cpr);
+    const Palette16 P = a.palette;
+
+    // Element offsets below are 32-bit (n * k < 2^32 is checked at launch).
+    // Copy side (lane constants): fused sign/mantissa rows 4q + (lane >> 3),
+    // piece lane & 7; palette rows 8q + (lane >> 2), quarter lane & 3; raw
+    // flags of row lane >> 1, group lane & 1; plain BF16 rows 2q + (lane >> 4),
+    // piece lane & 15.
+    const uint32_t lc_sm = uint32_t(lane >> 3) * k + uint32_t(lane & 7) * 16;
+    const uint32_t lc_flag = uint32_t(lane >> 1) * gpr + uint32_t(lane & 1);
+    const int pr = lane >> 2, pj = lane & 3;
+    const uint32_t lc_bf = uint32_t(lane >> 4) * k + uint32_t(lane & 15) * 8;
+    const uint32_t d_sm = sw128(lane >> 3, lane & 7), d_bf = row256(lane >> 4, lane & 15);
+    // consumer side (lane constants): rows g and g + 8, quarter c
+    const int fbit_a = 2 * g + (c >> 1), fbit_b = 2 * (g + 8) + (c >> 1);
+    const uint32_t o_sm0 = sw128(g, 2 * c), o_sm1 = sw128(g, 2 * c + 1);
+    const uint32_t o_pal = uint32_t(kPalOff + g * 64 + c * 16);
+    const uint32_t o_bfa = row256(g, 4 * c), o_bfb = row256(g + 8, 4 * c);
+    // X token rows of this lane (clamped: columns >= m are not stored)
+    const uint32_t o_xa = uint32_t(kXOff) + row256(min(g, xrows - 1), 4 * c);
+    const uint32_t o_xb = uint32_t(kXOff) + row256(min(g + 8, xrows - 1), 4 * c);
+
+    // W copies of the unit whose first weight is element `uoff` into slot s;
+    // returns this lane's raw flags as a consumer (bit 0: row g, bit 1: row
+    // g + 8, of its quarter).  Each copy instruction of the warp reads whole
+    // 128-byte lines.
+    auto issue_w = [&](uint32_t uoff, int s) -> uint32_t {
+        const uint32_t dst = ring + uint32_t(s * slot_b);
+        if (!PAL) {
+            const uint16_t *src = a.w_bf16 + (uoff + lc_bf);
+#pragma unroll
+            for (int q = 0; q < 8; q++) cp16(dst + d_bf + q * 2 * kRow256, src + size_t(q) * 2 * k);
+            return 0u;
+        }
+        const uint8_t *src = a.sm + (uoff + lc_sm);
+#pragma unroll
+        for (int q = 0; q < 4; q++) cp16(dst + d_sm + q * 512, src + size_t(q) * 4 * k);
+        // raw flags of the unit's 32 (row, group) pairs, one lookup per lane
+        const uint32_t gl = (uoff >> 6) + lc_flag;
+        const uint32_t fw = __ldg(a.flagbits + (gl >> 5));
+        const uint32_t mask = __ballot_sync(0xFFFFFFFFu, (fw >> (gl & 31u)) & 1u);
+#pragma unroll
+        for (int q = 0; q < 2; q++) {
+            const int r = 8 * q + pr;
+            if ((mask >> (2 * r + (pj >> 1))) & 1u) {
+                // a raw group: the quarter's 32 exponents from the raw plane
+                const uint32_t gg = (uoff >> 6) + uint32_t(r) * gpr + uint32_t(pj >> 1);
+                const uint32_t fwg = __ldg(a.flagbits + (gg >> 5)), bg = gg & 31u;
+                const uint32_t rank = __ldg(a.rawbase + (gg >> 5)) + __popc(fwg & ((1u << bg) - 1u));
+                const uint8_t *e = a.rawexp + uint64_t(rank) * kGroup + (pj & 1) * 32;
+                cp16(dst + kRawOff + sw128(r, 2 * pj), e);
+                cp16(dst + kRawOff + sw128(r, 2 * pj + 1), e + 16);
+            } else {
+                cp16(dst + kPalOff + uint32_t(r * 64 + pj * 16), a.pal + ((uoff + uint32_t(r) * k) >> 1) + pj * 16);
+            }
+        }
+        return ((mask >> fbit_a) & 1u) | (((mask >> fbit_b) & 1u) << 1);
+    };
+    // X copies of chunk `kc` (K offset) into slot s: m rows of 256 bytes
+    auto issue_x = [&](uint32_t kc, int s) {
+        const uint32_t dst = ring + uint32_t(s * slot_b) + uint32_t(kXOff);
+        for (int p = lane; p < xrows * 16; p += 32) {
+            const int r = p >> 4, j = p & 15;
+            cp16(dst + row256(r, j), a.x + (uint32_t(r) * k + kc + uint32_t(j) * 8));
+        }
+    };
+
+    float d0[NT][4], d1[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int q = 0; q < 4; q++) d0[t][q] = d1[t][q] = 0.f;
+
+    auto consume = [&](int s, uint32_t flags) {
+        const uint8_t *slot = smem + (warp * stages + s) * slot_b;
+        uint32_t wA[16], wB[16];
+        if (PAL) {
+            rebuild_pal(slot, o_sm0, o_sm1, o_pal, flags & 1u, P, wA);
+            rebuild_pal(slot, o_sm0 + 8 * 128, o_sm1 + 8 * 128, o_pal + 8 * 64, (flags >> 1) & 1u, P, wB);
+        } else {
+            lds64b(slot + o_bfa, wA);
+            lds64b(slot + o_bfb, wB);
+        }
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+            uint32_t xw[16];
+            lds64b(slot + (t == 0 ? o_xa : o_xb), xw);
+            // K-step j: A = {row g pair 2j, row g+8 pair 2j, row g pair 2j+1, row g+8 pair 2j+1}
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                mma16816((j & 1) ? d1[t] : d0[t], wA[2 * j], wB[2 * j], wA[2 * j + 1], wB[2 * j + 1], xw[2 * j],
+                         xw[2 * j + 1]);
+        }
+    };
+
+    // end of a piece of tile t: write Y, or hand the piece to the fix-up
+    const int64_t t_first = u_begin / a.cpr;
+    auto finish = [&](int64_t t, bool whole) {
+        float v[NT][4];
+#pragma unroll
+        for (int tt = 0; tt < NT; tt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                v[tt][q] = d0[tt][q] + d1[tt][q];
+                d0[tt][q] = d1[tt][q] = 0.f;
+            }
+        if (!whole) {
+            // this warp's first piece goes to slot 2 gw, its last to 2 gw + 1
+            const int64_t slot = 2 * gw + (t == t_first ? 0 : 1);
+#pragma unroll
+            for (int tt = 0; tt < NT; tt++)
+                *reinterpret_cast<float4 *>(a.partial + ((slot * NT + tt) * 32 + lane) * 4) =
+                    make_float4(v[tt][0], v[tt][1], v[tt][2], v[tt][3]);
+            __threadfence();
+            __syncwarp();
+            uint32_t old = 0;
+            if (lane == 0) old = atomicAdd(a.counters + t, 1u);
+            old = __shfl_sync(0xFFFFFFFFu, old, 0);
+            const int64_t wf = owner(t * a.cpr, a.units, a.warps), wl = owner(t * a.cpr + a.cpr - 1, a.units, a.warps);
+            if (old != uint32_t(wl - wf)) return;   // another warp adds the pieces
+            __threadfence();
+            // the pieces in warp order: the first owner's piece is its last
+            // one unless its run starts with this tile
+            for (int64_t w = wf; w <= wl; w++) {
+                const int64_t sl = 2 * w + ((w == wf && unit0(wf, a.units, a.warps) < t * a.cpr) ? 1 : 0);
+#pragma unroll
+                for (int tt = 0; tt < NT; tt++) {
+                    float4 *pp = reinterpret_cast<float4 *>(a.partial + ((sl * NT + tt) * 32 + lane) * 4);
+                    const float4 p = __ldcg(pp);
+                    // read once, then zeroed: a completed call leaves its whole
+                    // scratch zero, so a later call whose tile counters lie
+                    // where these fragments were finds them at zero
+                    __stcg(pp, make_float4(0.f, 0.f, 0.f, 0.f));
+                    if (w == wf) {
+                        v[tt][0] = p.x;
+                        v[tt][1] = p.y;
+                        v[tt][2] = p.z;
+                        v[tt][3] = p.w;
+                    } else {
+                        v[tt][0] += p.x;
+                        v[tt][1] += p.y;
+                        v[tt][2] += p.z;
+                        v[tt][3] += p.w;
+                    }
+                }
+            }
+            if (lane == 0) a.counters[t] = 0u;
+        }
+        // d[t][0..1]: row g, tokens 8t + 2c, +1; d[t][2..3]: row g + 8, same tokens
+        const int64_t ra = t * kRows + g, rb = ra + 8;
+#pragma unroll
+        for (int tt = 0; tt < NT; tt++) {
+            const int tok = 8 * tt + 2 * c;
+            if (tok < a.m) {
+                a.y[int64_t(tok) * a.n + ra] = v[tt][0];
+                a.y[int64_t(tok) * a.n + rb] = v[tt][2];
+            }
+            if (tok + 1 < a.m) {
+                a.y[int64_t(tok + 1) * a.n + ra] = v[tt][1];
+                a.y[int64_t(tok + 1) * a.n + rb] = v[tt][3];
+            }
+        }
+    };
+    // issue side: the unit after the last one issued, at chunk ii of its
+    // tile, element offset uoff_i; ring slot is_
+    const int c_first = int(u_begin - t_first * cpr);
+    int ii = c_first;
+    uint32_t uoff_i = uint32_t(t_first) * 16u * k + uint32_t(ii) * 128u;
+    const uint32_t tile_jump = 16u * k - uint32_t(cpr) * 128u;   // past a tile's last chunk -> next tile
+    int is_ = 0;
+    uint32_t rawbits = 0;   // consumer raw flags, 2 bits per slot
+    auto advance = [&]() {
+        uoff_i += 128u;
+        if (++ii == cpr) {
+            ii = 0;
+            uoff_i += tile_jump;
+        }
+        ++is_;
+    };
+    const int npro = min(stages - 1, nu);
+    for (int s = 0; s < stages - 1; s++) {
+        if (s < nu) {
+            if (!defer_x) issue_x(uint32_t(ii) * 128u, s);
+            rawbits |= issue_w(uoff_i, s) << (2 * s);
+            advance();
+        }
+        cp_commit();
+    }
+    if (defer_x) {
+        // the previous kernel has ended: the prologue units' X, one more group
+        pdl_wait();
+        int cx = c_first;
+        for (int s = 0; s < npro; s++) {
+            issue_x(uint32_t(cx) * 128u, s);
+            if (++cx == cpr) cx = 0;
+        }
+        cp_commit();
+    }
+
+    int64_t ct = t_first;
+    int ci = c_first, piece0 = ci, cs = 0;
+    for (int j = 0; j < nu; j++) {
+        // this lane's copies of unit j have landed (with the deferred X group,
+        // the first unit waits for everything issued so far) ...
+        cp_wait(defer_x && j == 0 ? 0 : stages - 2);
+        // ... and every lane's: the slot is read across lanes.  The barrier
+        // also orders every lane's reads of the slot consumed last iteration
+        // before the copies that now refill it.
+        __syncwarp();
+        const uint32_t fl = (rawbits >> (2 * cs)) & 3u;
+        if (j + stages - 1 < nu) {
+            if (is_ == stages) is_ = 0;
+            issue_x(uint32_t(ii) * 128u, is_);
+            rawbits = (rawbits & ~(3u << (2 * is_))) | (issue_w(uoff_i, is_) << (2 * is_));
+            advance();
+        }
+        cp_commit();
+        consume(cs, fl);
+        if (++cs == stages) cs = 0;
+        if (++ci == cpr || j == nu - 1) {
+            finish(ct, piece0 == 0 && ci == cpr);
+            if (ci == cpr) {
+                ci = 0;
+                ++ct;
+            }
+            piece0 = ci;
+        }
+    }
+}
+
+
+std::mutex g_mu;
+
+template <class K>
+cudaError_t prepare(K kern, int (&ready)[64]) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ready[dev]) return cudaSuccess;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (err != cudaSuccess) return err;
+    ready[dev] = 1;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+int gemv_sk_stages(int warps, int stages, int64_t m) {
+    if (warps < 1 || warps > kMaxWarps || stages < 0 || stages > kMaxStages || m < 1 || m > 16) return 0;
+    const size_t slot = size_t(slot_bytes(int(m)));
+    if (stages == 0) {   // the deepest ring that fits, at most kMaxStages
+        stages = int(std::min<size_t>(kMaxStages, size_t(kMaxSmem) / (size_t(warps) * slot)));
+        return stages >= 2 ? stages : 0;
+    }
+    if (stages < 2 || size_t(warps) * stages * slot > size_t(kMaxSmem)) return 0;
+    return stages;
+}
+
+GemvSkGeometry gemv_sk_geometry(int64_t m, int64_t n, int64_t k, int warps) {
+    GemvSkGeometry g{};
+    if (m <= 0 || m > 16 || n <= 0 || k <= 0 || n % kRows || k % kChunkK || warps < 1 || warps > kMaxWarps)
+        return g;
+    g.S = warps;
+    g.NT = m > 8 ? 2 : 1;
+    g.tiles = n / kRows;
+    g.cpr = k / kChunkK;
+    g.units = g.tiles * g.cpr;
+    g.warps = std::min<int64_t>(int64_t(sm_count()) * warps, g.units);
+    g.G = int((g.warps + warps - 1) / warps);
+    g.counter_bytes = align_up(uint64_t(g.tiles) * 4, 256);
+    g.partial_bytes = align_up(uint64_t(2 * g.warps) * uint64_t(g.NT) * 32 * 4 * 4, 256);
+    return g;
+}
+
+cudaError_t launch_gemv_sk(const GemvSkLaunch &p, cudaStream_t stream) {
+    const GemvSkGeometry g = gemv_sk_geometry(p.m, p.n, p.k, p.warps);
+    const int stages = gemv_sk_stages(p.warps, p.stages, p.m);
+    if (g.G <= 0 || stages == 0 || !p.counters || !p.partial || !p.x || !p.y) return cudaErrorInvalidValue;
+    // element offsets inside the kernel are 32-bit
+    if (uint64_t(p.n) * uint64_t(p.k) > 0xFFFFFFFFull) return cudaErrorInvalidValue;
+    SkArgs a{};
+    a.x = p.x;
+    a.n = p.n;
+    a.k = p.k;
+    a.m = int(p.m);
+    a.cpr = g.cpr;
+    a.units = g.units;
+    a.warps = g.warps;
+    a.y = p.y;
+    a.partial = p.partial;
+    a.counters = p.counters;
+    a.stages = stages;
+    a.slot_bytes = slot_bytes(int(p.m));
+    const bool pal = p.pal != nullptr;
+    if (pal) {
+        if (!p.w) return cudaErrorInvalidValue;
+        a.sm = p.w->sm;
+        a.pal = p.pal;
+        a.flagbits = p.w->flagbits;
+        a.rawbase = p.w->rawbase;
+        a.rawexp = p.w->rawexp;
+        a.palette = make_palette16(p.w->palette);
+        a.w_stable = p.w_stable ? 1 : 0;
+    } else {
+        if (!p.w_bf16) return cudaErrorInvalidValue;
+        a.w_bf16 = p.w_bf16;
+    }
+    const size_t smem = size_t(p.warps) * stages * size_t(a.slot_bytes);
+    const dim3 grid(unsigned(g.G)), block(unsigned(p.warps * 32));
+    cudaError_t err = cudaSuccess;
+#define UW_SK_LAUNCH(P_, N_)                                                    \
+    do {                                                                        \
+        static int ready[64] = {0};                                             \
+        err = prepare(k_gemv_sk<P_, N_>, ready);                                \
+        if (err == cudaSuccess)                                                 \
+            err = launch_pdl(a.w_stable != 0, k_gemv_sk<P_, N_>, grid, block, smem, stream, a); \
+    } while (0)
+    if (pal) {
+        if (g.NT == 2) UW_SK_LAUNCH(true, 2); else UW_SK_LAUNCH(true, 1);
+    } else {
+        if (g.NT == 2) UW_SK_LAUNCH(false, 2); else UW_SK_LAUNCH(false, 1);
+    }
+#undef UW_SK_LAUNCH
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+}  // namespace uw

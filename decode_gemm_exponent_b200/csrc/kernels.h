@@ -96,6 +96,40 @@ struct MmaItem {
 cudaError_t launch_gemv_mma_batched(const MmaItem *items, int n_items, int slices, int width,
                                     cudaStream_t stream);
 
+// SMs of the current device (148 when no device answers, so that workspace
+// sizes can be computed on a host without a GPU).
+int sm_count();
+
+// Persistent stream-K form of the warp-MMA kernel, m <= 16, k a multiple of
+// 128 and n * k < 2^32 (gemv_sk.cu): one CTA of `warps` warps per SM, every
+// warp an equal contiguous run of (16-row tile, 128-wide K chunk) units, its
+// loads (W and the chunk's X rows) in a shared-memory ring of `stages` slots
+// of 5120 + 288 m bytes (0 = the deepest that fits) filled by cp.async; a
+// tile cut between warps is summed in warp order by the warp that finishes
+// its last piece.  Workspace: `counters` (one u32 per tile,
+// zero before the call and left zero by it) and `partial` (two fragment
+// sets of 32 x 4 x NT floats per warp).  pal == nullptr: plain BF16 `w_bf16`.
+struct GemvSkGeometry {
+    int G = 0, S = 0, NT = 0;
+    int64_t tiles = 0, cpr = 0, units = 0, warps = 0;
+    uint64_t counter_bytes = 0, partial_bytes = 0;
+};
+GemvSkGeometry gemv_sk_geometry(int64_t m, int64_t n, int64_t k, int warps);
+int gemv_sk_stages(int warps, int stages, int64_t m);   // the ring depth used, 0 if not valid for m tokens
+struct GemvSkLaunch {
+    const uint16_t *x;
+    int64_t m, n, k;
+    const uint16_t *w_bf16;    // plain path
+    const uw_dmat *w;          // fused path: sm/raw/flag planes
+    const uint8_t *pal;        // fused path: palette plane
+    float *y;
+    uint32_t *counters;
+    float *partial;
+    int warps, stages;
+    bool w_stable;             // fused: the planes are the blob's (read before the previous kernel ends)
+};
+cudaError_t launch_gemv_sk(const GemvSkLaunch &p, cudaStream_t stream);
+
 // tcgen05 GEMM (Unweight page §七, reconstructive matmul), token tile `bn`.
 // Launch, with programmatic stream serialization when `early` is set: the
 // kernel calls pdl_wait before touching data an earlier kernel on the stream

@@ -31,7 +31,7 @@ EMIT_PALETTE = 2
 SEC_SM, SEC_RAWEXP, SEC_FLAGS, SEC_RAWBASE, SEC_STREAM, SEC_CHUNKOFF, SEC_DLUT, SEC_PAL = range(8)
 NUM_SECTIONS = 8
 PIPE_DECODE_GEMM, PIPE_DECODE_EXP_FUSED, PIPE_TRANSCODE_FUSED, PIPE_DIRECT_PALETTE, PIPE_HUFFMAN_FUSED = 1, 2, 3, 4, 5
-KERNEL_FMA, KERNEL_TC, KERNEL_MMA, KERNEL_TC_SK = 1, 2, 3, 4
+KERNEL_FMA, KERNEL_TC, KERNEL_MMA, KERNEL_TC_SK, KERNEL_MMA_SK = 1, 2, 3, 4, 5
 DEBUG_NEVER_ARRIVE = 1
 
 # every symbol include/uw.h declares
@@ -446,7 +446,8 @@ def autotune(mats: Sequence[Matrix], ms: Sequence[int], reps: int = 5, stream=No
 PIPELINE_NAMES = {PIPE_DECODE_GEMM: "decode_gemm", PIPE_DECODE_EXP_FUSED: "decode_exp_fused",
                   PIPE_TRANSCODE_FUSED: "transcode_fused", PIPE_DIRECT_PALETTE: "direct_palette",
                   PIPE_HUFFMAN_FUSED: "huffman_fused"}
-KERNEL_NAMES = {KERNEL_FMA: "fma", KERNEL_TC: "tc", KERNEL_MMA: "mma", KERNEL_TC_SK: "tc_sk"}
+KERNEL_NAMES = {KERNEL_FMA: "fma", KERNEL_TC: "tc", KERNEL_MMA: "mma", KERNEL_TC_SK: "tc_sk",
+                KERNEL_MMA_SK: "mma_sk"}
 
 
 def plans_from_json(text: str, ms: Sequence[int]):

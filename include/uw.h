@@ -221,13 +221,23 @@ typedef enum uw_kernel {
     UW_KERNEL_MMA = 3,   /* m <= 16: W rebuilt in registers straight into warp-level
                             MMA fragments; one CTA per 16-row tile, whose `bn`
                             warps split K (summed in a fixed order)               */
-    UW_KERNEL_TC_SK = 4  /* any m: persistent stream-K tcgen05 kernel, token tile
+    UW_KERNEL_TC_SK = 4, /* any m: persistent stream-K tcgen05 kernel, token tile
                             `bn`, one CTA per SM, each owning an equal contiguous
                             run of (128-row x bn tile, 64-wide K-step) units; a
                             tile cut between CTAs is summed in CTA (= K) order by
                             the CTA that finishes its last piece.  Needs a
                             workspace whose tile counters are zero (see
                             uw_workspace_size); split_k must be 1             */
+    UW_KERNEL_MMA_SK = 5 /* m <= 16, k a multiple of 128, n*k < 2^32 (a larger matrix
+                            fails at launch, UW_ERR_CUDA): persistent stream-K form of
+                            UW_KERNEL_MMA, one CTA of `bn` (1..16) warps per SM;
+                            every warp owns an equal contiguous run of (16-row
+                            tile, 128-wide K chunk) units and stages its loads
+                            in a shared-memory ring filled by cp.async; a tile
+                            cut between warps is summed in warp (= K) order by
+                            the warp that finishes its last piece.  Needs a
+                            workspace whose tile counters are zero, as TC_SK;
+                            split_k must be 1                                 */
 } uw_kernel;
 
 #define UW_DEBUG_NEVER_ARRIVE 1u   /* TC kernel: wait on a barrier nobody signals, so
@@ -238,16 +248,20 @@ typedef struct uw_plan {
     int32_t kernel;       /* uw_kernel */
     int32_t bn;           /* TC: tokens per tile, one of 16,32,64,128,256;
                              FMA: weight rows per warp, 1 or 2;
-                             MMA: warps per CTA = K slices per 16-row tile, 1..8 */
+                             MMA: warps per CTA = K slices per 16-row tile, 1..8;
+                             MMA_SK: warps per CTA (one CTA per SM), 1..16 */
     int32_t split_k;      /* TC: K split into this many slices (>= 1), reduced in a
-                             fixed order; FMA, MMA, TC_SK: must be 1 */
+                             fixed order; FMA, MMA, TC_SK, MMA_SK: must be 1 */
     int32_t stages;       /* TC: shared-memory ring depth (0 = default: 4 for the plain
                              kernel, the largest that fits for the fused one);
                              TC_SK: compressed-tile ring depth of the fused kernel
                              (W-tile ring of the plain one), 0 = the largest that
                              fits (at most 6 / 8);
                              MMA: weights per lane and row per step, 1 = 16, 2 = 32
-                             (K a multiple of 128), 0 = 32 when K allows, else 16 */
+                             (K a multiple of 128), 0 = 32 when K allows, else 16;
+                             MMA_SK: ring slots per warp (2..8) of 5120 + 288 m
+                             bytes each, bn x stages slots within 227 KB; 0 = the
+                             deepest that fits, at most 8 */
     uint32_t debug_flags; /* UW_DEBUG_* (0 in production) */
     int64_t timeout_ns;   /* spin-wait limit inside kernels (0 = 2 s) */
 } uw_plan;
@@ -262,12 +276,21 @@ uw_status uw_plan_default(int64_t m, int64_t n, int64_t k, int32_t pipeline, uw_
  * pipeline 4: none), each part rounded up to 256 bytes, plus split_k*m*n
  * floats of partial sums for a TC plan with split_k > 1, or for a TC_SK plan
  * one uint32 counter per 128 x bn tile (256-byte rounded) followed by two
- * 128 x bn float tiles per CTA (one CTA per SM of the current device).
- * TC_SK: the counters must be zero when a call starts.  Zero the whole
- * workspace once after allocating it; every call that completes leaves the
- * counters zero again, so the same workspace serves any later TC_SK call
- * (any shape) without clearing.  After a call whose uw_device_status reports
- * an error, zero the workspace again before reusing it.                     */
+ * 128 x bn float tiles per CTA (one CTA per SM of the current device), or
+ * for an MMA_SK plan one uint32 counter per 16-row tile (256-byte rounded)
+ * followed by two sets of 128 (m <= 8) or 256 floats per warp of the grid
+ * (bn warps per SM of the current device, at most one per unit).
+ * TC_SK, MMA_SK: the counters must be zero when a call starts.  Zero the whole
+ * workspace once after allocating it; every call that completes leaves its
+ * counters and partial tiles zero again, so the same workspace serves any
+ * later direct-palette (pipeline 4) TC_SK or MMA_SK call, of any shape,
+ * without clearing.  A call
+ * of pipelines 1-3 writes its preprocessing output at the start of the
+ * workspace, where a pipeline-4 call keeps its counters: zero the workspace
+ * again after such a call before a stream-K call of another pipeline or
+ * shape uses it (uw_stack_run keeps its counters in a region of their own).
+ * After a call whose uw_device_status reports an error, zero the workspace
+ * again before reusing it.                                                  */
 uw_status uw_workspace_size(int64_t m, int64_t n, int64_t k, const uw_plan *plan,
                             size_t *bytes);
 
@@ -315,8 +338,8 @@ uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const
 /* Matmul without a caller workspace (no counterpart on the Unweight page).   */
 
 /* Bytes of the library-owned scratch array used by uw_fused_matmul_noalloc,
- * and how many of them (at its start) hold TC_SK tile counters, one uint32
- * per 128 x bn tile.                                                        */
+ * and how many of them (at its start) hold stream-K tile counters, one
+ * uint32 per 128 x bn tile (TC_SK) or per 16-row tile (MMA_SK).              */
 #define UW_NOALLOC_SCRATCH_BYTES (16u << 20)
 #define UW_NOALLOC_COUNTER_BYTES (64u << 10)
 
@@ -331,7 +354,7 @@ uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const
  *   - plan->pipeline must be UW_PIPE_DIRECT_PALETTE (INVALID_ARG otherwise);
  *     a plan whose scratch (uw_workspace_size) does not fit is rejected with
  *     UW_ERR_WORKSPACE before anything is launched: partial sums beyond
- *     UW_NOALLOC_SCRATCH_BYTES - UW_NOALLOC_COUNTER_BYTES, or (TC_SK) more
+ *     UW_NOALLOC_SCRATCH_BYTES - UW_NOALLOC_COUNTER_BYTES, or (TC_SK, MMA_SK) more
  *     tile counters than UW_NOALLOC_COUNTER_BYTES hold.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
@@ -343,7 +366,7 @@ uw_status uw_fused_matmul_batched(const uw_batch_item *items, int n_items, const
  *     the caller.  Partial sums do not carry over: in a call whose kernels
  *     complete, every partial sum read was written by that same call.  A
  *     call whose uw_device_status then reports an error may have left stale
- *     values in y, and (TC_SK) non-zero tile counters, after which the
+ *     values in y, and (TC_SK, MMA_SK) non-zero tile counters, after which the
  *     entry point should not be used again in the process.                 */
 uw_status uw_fused_matmul_noalloc(const uint16_t *x_dev, int64_t m, const uw_dmat *w,
                                   float *y_dev, const uw_plan *plan, void *stream);
@@ -386,8 +409,8 @@ typedef struct uw_stack_step {
 /* Workspace of uw_stack_run: two preprocessing slots, each the largest
  * preprocessing buffer of the stack (decode 2nk bytes, exponent decode a bit
  * over nk, transcode nk/2), plus the largest split-K scratch of any step,
- * plus (for TC_SK steps) a region of stream-K tile counters kept apart from
- * the partial sums.  Zero the workspace once after allocating it (the
+ * plus (for TC_SK and MMA_SK steps) a region of stream-K tile counters kept
+ * apart from the partial sums.  Zero the workspace once after allocating it (the
  * counters must start at zero; completed runs leave them zero).             */
 uw_status uw_stack_workspace_size(const uw_stack_step *steps, int n_steps, size_t *bytes);
 

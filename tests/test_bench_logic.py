@@ -150,6 +150,8 @@ def test_oracle_sample_is_the_step_on_a_row_sample():
 def test_kernel_names_of_every_plan_kind():
     from decode_gemm_exponent_b200 import uw
     assert bench.kernel_group(uw.make_plan(4, uw.KERNEL_TC_SK, 64, 1)) == "fused/tc_sk_bn64"
+    assert bench.kernel_group(uw.make_plan(4, uw.KERNEL_MMA_SK, 8, 1, 6)) == "fused/mma_sk_w8_s6"
+    assert bench.launches_per_call(uw.make_plan(4, uw.KERNEL_MMA_SK, 8, 1, 6)) == 1
     assert bench.plan_label(uw.make_plan(1, uw.KERNEL_TC, 64, 4)) == "decode+plain/tcgen05_bn64/split4"
     assert bench.launches_per_call(uw.make_plan(4, uw.KERNEL_TC_SK, 16, 1)) == 1
     assert bench.launches_per_call(uw.make_plan(3, uw.KERNEL_TC_SK, 16, 1)) == 2

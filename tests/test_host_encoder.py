@@ -262,6 +262,47 @@ def test_plans_and_workspace(uw):
         uw.workspace_size(4, n, 1600, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, stages=2))
 
 
+def test_stream_k_gemv_plans_and_workspace(uw):
+    """UW_KERNEL_MMA_SK: tile counters (one u32 per 16-row tile, 256-byte
+    rounded) then two fragment sets (32 lanes x 4 floats per 8-token tile) per
+    warp of the grid; with no GPU the library sizes the grid for 148 SMs.  A
+    ring slot holds 5120 + 288 m bytes and a CTA's slots must fit 227 KB."""
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    def fits(warps, stages, m):
+        return warps * stages * (5120 + 288 * m) <= 227 * 1024
+
+    n, k = 14336, 4096
+    tiles, units = n // 16, n // 16 * (k // 128)
+    for m, nt in ((1, 1), (4, 1), (8, 1), (9, 2), (16, 2)):
+        for warps, stages in ((8, 5), (16, 2), (12, 3), (11, 2), (8, 2), (1, 2), (16, 0), (12, 0), (4, 8)):
+            p = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA_SK, warps, 1, stages)
+            ok = fits(warps, stages, m) if stages else fits(warps, 2, m)
+            if ok:
+                w = min(148 * warps, units)
+                assert uw.workspace_size(m, n, k, p) == up(tiles * 4) + up(2 * w * nt * 32 * 4 * 4), (m, warps, stages)
+            else:
+                with pytest.raises(uw.UwError):
+                    uw.workspace_size(m, n, k, p)
+    # a small matrix: at most one warp per unit
+    p = uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA_SK, 16, 1, 2)
+    assert uw.workspace_size(1, 1024, 1024, p) == up(64 * 4) + up(2 * 512 * 32 * 4 * 4)
+    # the preprocessing output comes first
+    assert uw.workspace_size(1, 1024, 1024, uw.make_plan(uw.PIPE_DECODE_GEMM, uw.KERNEL_MMA_SK, 16, 1, 2)) == \
+        1024 * 1024 * 2 + up(64 * 4) + up(2 * 512 * 32 * 4 * 4)
+    for bad_m, bad_k, bad in ((17, k, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=8)),        # m <= 16
+                              (4, 1600, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=8)),      # k % 128
+                              (4, k, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=0)),
+                              (4, k, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=17)),
+                              (4, k, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=8, split_k=2)),
+                              (4, k, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=8, stages=1)),
+                              (4, k, uw.make_plan(kernel=uw.KERNEL_MMA_SK, bn=8, stages=9)),
+                              (4, k, uw.make_plan(pipeline=5, kernel=uw.KERNEL_MMA_SK, bn=8))):
+        with pytest.raises(uw.UwError):
+            uw.workspace_size(bad_m, n, bad_k, bad)
+
+
 def test_stack_workspace_and_argument_checks(uw):
     """uw_stack_workspace_size / uw_stack_run host logic.  The matrix is bound
     to a device address that is never dereferenced (binding reads only the
