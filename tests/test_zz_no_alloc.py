@@ -56,8 +56,9 @@ def test_noalloc_rejects_oversized_scratch(uw):
 def test_noalloc_alternating_plans_and_sizes(uw):
     """Calls of different sizes and kernels in a row share the one array: a
     large split-K call, then smaller ones that overwrite less of it, and
-    stream-K calls whose tile counters sit apart from the partial sums.  Each
-    result equals uw_fused_matmul with a fresh zero-filled workspace."""
+    stream-K calls (tcgen05 and warp-MMA) whose tile counters sit apart from
+    the partial sums.  Each result equals uw_fused_matmul with a fresh
+    zero-filled workspace."""
     n, k = 512, 1024
     mat = uw.Matrix(uw.encode(synth.weights_bf16(n, k, 0.02, 0.002, 1.0, seed=33)))
     calls = [(64, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 64, 8)),
@@ -66,7 +67,11 @@ def test_noalloc_alternating_plans_and_sizes(uw):
              (64, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 64, 8)),
              (100, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC_SK, 64, 1)),
              (3, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 16, 3)),
-             (16, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC_SK, 16, 1))]
+             (16, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC_SK, 16, 1)),
+             (1, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA_SK, 8, 1, 0)),
+             (64, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_TC, 64, 8)),
+             (16, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA_SK, 8, 1, 2)),
+             (5, uw.make_plan(uw.PIPE_DIRECT_PALETTE, uw.KERNEL_MMA_SK, 16, 1, 2))]
     for i, (m, plan) in enumerate(calls):
         x = torch.from_numpy(synth.activations_bf16(m, k, seed=50 + i).view(np.int16)).cuda()
         y_ref = mat.matmul(x, plan).cpu().numpy()
