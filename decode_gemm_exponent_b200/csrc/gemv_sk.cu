@@ -137,14 +137,16 @@ __host__ __device__ constexpr int slot_bytes(int xrows) { return kXOff + xrows *
 __device__ __forceinline__ uint32_t sw128(int r, int j) { return uint32_t(r * 128 + ((j ^ (r & 1)) << 4)); }
 __device__ __forceinline__ uint32_t row256(int r, int j) { return uint32_t(r * kRow256 + j * 16 + (j >= 8 ? 16 : 0)); }
 
-// One row's 32 weights (quarter c of the chunk) from a ring slot -> 16 BF16
-// pairs (weights 2i, 2i + 1 in pair i).  `sm0`, `sm1`: the row's two
-// sign/mantissa pieces of the quarter (the same offsets inside the raw
-// region hold its raw exponents); `pal`: its palette piece.
-__device__ __forceinline__ void rebuild_pal(const uint8_t *slot, uint32_t sm0, uint32_t sm1, uint32_t pal, bool raw,
-                                            const Palette16 &P, uint32_t (&w)[16]) {
+// One row's 32 weights (quarter c of the chunk) from a ring slot: its
+// sign/mantissa words sm[i] (weights 4i .. 4i + 3) and the rotated exponent
+// bytes of the same weights e[i].  `sm0`, `sm1`: the row's two sign/mantissa
+// pieces of the quarter (the same offsets inside the raw region hold its raw
+// exponents); `pal`: its palette piece.
+__device__ __forceinline__ void row_words(const uint8_t *slot, uint32_t sm0, uint32_t sm1, uint32_t pal, bool raw,
+                                          const Palette16 &P, uint32_t (&sm)[8], uint32_t (&e)[8]) {
     const uint4 s0 = lds128(slot + sm0), s1 = lds128(slot + sm1);
-    uint32_t e[8];   // rotated exponent bytes, 4 weights per word
+    sm[0] = s0.x; sm[1] = s0.y; sm[2] = s0.z; sm[3] = s0.w;
+    sm[4] = s1.x; sm[5] = s1.y; sm[6] = s1.z; sm[7] = s1.w;
     if (raw) {
         const uint4 b0 = lds128(slot + kRawOff + sm0), b1 = lds128(slot + kRawOff + sm1);
 #pragma unroll
@@ -155,22 +157,6 @@ __device__ __forceinline__ void rebuild_pal(const uint8_t *slot, uint32_t sm0, u
         const uint4 b0 = lds128(slot + pal);
 #pragma unroll
         for (int i = 0; i < 4; i++) pal_rot(w4(b0, i), P, e[2 * i], e[2 * i + 1]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; i++) join4(e[i], w4(s0, i), w[2 * i], w[2 * i + 1]);
-#pragma unroll
-    for (int i = 0; i < 4; i++) join4(e[4 + i], w4(s1, i), w[8 + 2 * i], w[8 + 2 * i + 1]);
-}
-
-// 16 consecutive words (64 contiguous bytes) from shared memory
-__device__ __forceinline__ void lds64b(const uint8_t *addr, uint32_t (&w)[16]) {
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-        const uint4 v = lds128(addr + q * 16);
-        w[4 * q] = v.x;
-        w[4 * q + 1] = v.y;
-        w[4 * q + 2] = v.z;
-        w[4 * q + 3] = v.w;
     }
 }
 
@@ -267,25 +253,38 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
 #pragma unroll
         for (int q = 0; q < 4; q++) d0[t][q] = d1[t][q] = 0.f;
 
+    // One unit, in four blocks of 8 weights per row: a block's BF16 pairs
+    // (4 per row) feed MMA K-steps 2b and 2b + 1 with 16 bytes of X per token
+    // tile, so only one block's pairs are live at a time.  Each accumulator
+    // receives its MMAs in K-step order, as if the unit's pairs were built
+    // first.
     auto consume = [&](int s, uint32_t flags) {
         const uint8_t *slot = smem + (warp * stages + s) * slot_b;
-        uint32_t wA[16], wB[16];
+        uint32_t smA[8], eA[8], smB[8], eB[8];
         if (PAL) {
-            rebuild_pal(slot, o_sm0, o_sm1, o_pal, flags & 1u, P, wA);
-            rebuild_pal(slot, o_sm0 + 8 * 128, o_sm1 + 8 * 128, o_pal + 8 * 64, (flags >> 1) & 1u, P, wB);
-        } else {
-            lds64b(slot + o_bfa, wA);
-            lds64b(slot + o_bfb, wB);
+            row_words(slot, o_sm0, o_sm1, o_pal, flags & 1u, P, smA, eA);
+            row_words(slot, o_sm0 + 8 * 128, o_sm1 + 8 * 128, o_pal + 8 * 64, (flags >> 1) & 1u, P, smB, eB);
         }
 #pragma unroll
-        for (int t = 0; t < NT; t++) {
-            uint32_t xw[16];
-            lds64b(slot + (t == 0 ? o_xa : o_xb), xw);
-            // K-step j: A = {row g pair 2j, row g+8 pair 2j, row g pair 2j+1, row g+8 pair 2j+1}
+        for (int b = 0; b < 4; b++) {
+            uint32_t wa[4], wb[4];   // pairs 4b .. 4b + 3 of rows g and g + 8
+            if (PAL) {
+                join4(eA[2 * b], smA[2 * b], wa[0], wa[1]);
+                join4(eA[2 * b + 1], smA[2 * b + 1], wa[2], wa[3]);
+                join4(eB[2 * b], smB[2 * b], wb[0], wb[1]);
+                join4(eB[2 * b + 1], smB[2 * b + 1], wb[2], wb[3]);
+            } else {
+                const uint4 va = lds128(slot + o_bfa + 16 * b), vb = lds128(slot + o_bfb + 16 * b);
+                wa[0] = va.x; wa[1] = va.y; wa[2] = va.z; wa[3] = va.w;
+                wb[0] = vb.x; wb[1] = vb.y; wb[2] = vb.z; wb[3] = vb.w;
+            }
 #pragma unroll
-            for (int j = 0; j < 8; j++)
-                mma16816((j & 1) ? d1[t] : d0[t], wA[2 * j], wB[2 * j], wA[2 * j + 1], wB[2 * j + 1], xw[2 * j],
-                         xw[2 * j + 1]);
+            for (int t = 0; t < NT; t++) {
+                const uint4 x = lds128(slot + (t == 0 ? o_xa : o_xb) + 16 * b);
+                // K-step j: A = {row g pair 2j, row g+8 pair 2j, row g pair 2j+1, row g+8 pair 2j+1}
+                mma16816(d0[t], wa[0], wb[0], wa[1], wb[1], x.x, x.y);   // j = 2b
+                mma16816(d1[t], wa[2], wb[2], wa[3], wb[3], x.z, x.w);   // j = 2b + 1
+            }
         }
     };
 
