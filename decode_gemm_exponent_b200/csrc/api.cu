@@ -91,6 +91,8 @@ uw_status run_kernel(const uint16_t *x, int64_t m, const uint16_t *w_bf16, const
         g.warps = plan->bn;
         g.stages = plan->stages;
         g.w_stable = w_stable;
+        g.status = status;
+        g.timeout_ns = plan->timeout_ns > 0 ? uint64_t(plan->timeout_ns) : kDefaultTimeoutNs;
         if (sk_counters) {
             g.counters = sk_counters;
             g.partial = partial;

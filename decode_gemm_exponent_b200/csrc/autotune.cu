@@ -7,8 +7,7 @@
 // runtime transcode + fused kernel, direct palette + fused kernel) crossed
 // with the kernel variants: the
 // warp-MMA kernel (m <= 16, 2-8 K slices per tile, 16 or 32 weights per lane
-// and step), its persistent stream-K form (m <= 16, 8-16 warps per SM with
-// 2-4 ring slots each, where they fit), the FMA GEMV (m <= 8, 1 or 2 rows per warp) and the tcgen05
+// and step), the FMA GEMV (m <= 8, 1 or 2 rows per warp) and the tcgen05
 // kernel with token tiles around m and split-K factors 1-8 (so that some
 // candidate fills the 148 SMs with close to whole waves).  Each candidate is
 // run once to warm up (its status is checked) and then `reps` times, each
@@ -16,7 +15,12 @@
 // space has pushed the matrix out of the 126 MB L2 (a read, so the evicted
 // lines are clean and no write-back lands in the timed call): the weights
 // stream from HBM as they do in a model's layer sequence.  The fastest
-// average wins.
+// average wins.  The persistent stream-K warp-MMA kernel (UW_KERNEL_MMA_SK)
+// is not a candidate: it wins such single calls on some shapes by a few
+// percent, but a step of calls run back to back is slower with it, since it
+// fills every SM's shared memory and registers and so cannot start while
+// the previous call drains, as the one-tile kernels do; it is used by
+// explicit plan.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -63,17 +67,6 @@ std::vector<uw_plan> candidates(const uw_dmat &w, int64_t m) {
                     p.stages = width;
                     out.push_back(p);
                 }
-            }
-        if (m <= 16 && w.k % 128 == 0)   // persistent stream-K warp-MMA kernel (ring sizes that fit)
-            for (const auto &ws : {std::pair<int, int>{16, 2}, {12, 3}, {12, 2}, {11, 2}, {8, 4}, {8, 2}}) {
-                if (uw::gemv_sk_stages(ws.first, ws.second, m) == 0) continue;
-                uw_plan p{};
-                p.pipeline = pipe;
-                p.kernel = UW_KERNEL_MMA_SK;
-                p.bn = ws.first;
-                p.split_k = 1;
-                p.stages = ws.second;
-                out.push_back(p);
             }
         if (m <= 8)
             for (int rows : {1, 2}) {

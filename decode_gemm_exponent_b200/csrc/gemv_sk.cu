@@ -8,10 +8,12 @@
 // tens of KB of W requested at any time, which at HBM's loaded latency caps
 // the stream well below the HBM peak; and an 8B gate projection's 896 tiles
 // make two full waves of CTAs plus a nearly empty third one.  Here:
-//  - the warp copies each unit's compressed W and the chunk's X rows into
-//    shared memory with cp.async (16 bytes a copy, L1 bypassed), so a ring of
-//    several units per warp costs no registers, an SM keeps ~100 KB in
-//    flight, and the MMAs never wait on X from L2;
+//  - one lane of the warp loads each unit's compressed W and the chunk's X
+//    rows into the warp's shared-memory ring with 2-D TMA boxes (16 rows x
+//    128 sign/mantissa bytes, 16 rows x 64 palette bytes, m rows x 128 X
+//    values), completing on one mbarrier per ring slot, so a ring of several
+//    units per warp costs no registers and next to no instructions, an SM
+//    keeps ~100 KB in flight, and the MMAs never wait on X from L2;
 //  - one CTA per SM of `S` warps, and every warp of the grid owns an equal
 //    contiguous run of units (16-row tile, 128-wide K chunk), in tile-major
 //    order, so every warp streams the same number of bytes: no tail wave;
@@ -27,16 +29,15 @@
 // the tile and weights [32c, 32c + 32) of the chunk, with the same fragment
 // map as the one-tile kernel at 32 weights per lane (MMA K-step j, thread c,
 // K slots {2c, 2c+1, 2c+8, 2c+9} <- weights 32c + 4j + {0, 1, 2, 3}; X uses
-// the same map, so every product is formed once).  The copies are not made
-// by the lanes that use the data: each copy instruction of a warp reads whole
-// 128-byte lines (a row's 128 sign/mantissa bytes take 8 lanes, its 64
-// palette bytes 4), and after its copies have landed every lane passes a
-// warp barrier before reading the slot, whose rows are bank-swizzled.  A raw
-// group's quarter is copied from the raw plane instead of the palette plane
-// by the lane that would copy its palette bytes; the warp learns which
-// groups are raw from one bitmap lookup per lane and a ballot.  The fused
-// and plain kernels differ only in these copies and the rebuild, so their
-// outputs are bit-identical.
+// the same map, so every product is formed once).  The boxes land densely
+// (row-major) in the slot.  A raw group's 32 exponents of a lane's quarter
+// are copied by that lane itself with cp.async from the raw plane (raw groups
+// are rare and scattered); the warp learns which groups are raw from one
+// bitmap lookup per lane and a ballot.  Every wait on a slot's barrier is
+// bounded: on time-out the kernel raises UW_DEVERR_TIMEOUT, stops issuing,
+// waits (bounded) for the boxes it has issued and returns.  The fused and
+// plain kernels differ only in the W boxes and the rebuild, so their outputs
+// are bit-identical.
 #include <algorithm>
 #include <mutex>
 
@@ -75,6 +76,8 @@ struct SkArgs {
     int stages;                // ring slots per warp (2..8)
     int slot_bytes;            // bytes of one ring slot (W and the chunk's X rows)
     int w_stable;              // fused: planes no kernel writes (read before pdl_wait)
+    uint32_t *status;          // device error word (UW_DEVERR_*), may be null
+    uint64_t timeout_ns;       // bound of every barrier wait
 };
 
 // first unit of warp w
@@ -117,25 +120,18 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ uint32_t w4(const uint4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
 
-// Byte offsets inside a ring slot.
-//  - Fused: row r's 128 sign/mantissa bytes at r * 128, its 64 palette bytes
-//    at kPalOff + r * 64, and the exponents of its raw groups at kRawOff +
-//    r * 128 (one byte per weight; only raw groups' bytes are written).  The
-//    16-byte pieces of a 128-byte row sit at piece ^ (r & 1), so that rows g
-//    and g + 1, which a quarter warp reads together, fall on different banks.
-//  - Plain: row r's 256 BF16 bytes at row256(r, piece).
-//  - X (both): token row r's 256 bytes of the chunk at kXOff + row256(r, piece).
-//  row256 spaces rows 288 bytes apart and pieces 8-15 16 bytes further, so
-//  that the 8 lanes of a quarter warp, which read pieces 4c .. 4c + 3 of rows
-//  g and g + 1 (c = 0..3), hit 8 different bank groups, and every lane's 64
-//  bytes stay contiguous (its four loads differ by immediate offsets).
+// Byte offsets inside a ring slot (every region 128-byte aligned, the TMA
+// boxes dense):
+//  - fused: the 16 rows' sign/mantissa bytes at r * 128 (one box), their
+//    palette bytes at kPalOff + r * 64 (one box), and the exponents of a
+//    lane's raw quarters at kRawOff + r * 128 + 32 c (copied by that lane);
+//  - plain: the 16 rows' BF16 weights at r * 256 (one box);
+//  - both: the chunk's m X rows at kXOff + r * 256 (one box).
+// A ring slot is followed, after all warps' rings, by one mbarrier per slot.
 constexpr int kPalOff = 16 * 128;
 constexpr int kRawOff = kPalOff + 16 * 64;
 constexpr int kXOff = kRawOff + 16 * 128;
-constexpr int kRow256 = 288;
-__host__ __device__ constexpr int slot_bytes(int xrows) { return kXOff + xrows * kRow256; }
-__device__ __forceinline__ uint32_t sw128(int r, int j) { return uint32_t(r * 128 + ((j ^ (r & 1)) << 4)); }
-__device__ __forceinline__ uint32_t row256(int r, int j) { return uint32_t(r * kRow256 + j * 16 + (j >= 8 ? 16 : 0)); }
+__host__ __device__ constexpr int slot_bytes(int xrows) { return kXOff + xrows * 256; }
 
 // One row's 32 weights (quarter c of the chunk) from a ring slot: its
 // sign/mantissa words sm[i] (weights 4i .. 4i + 3) and the rotated exponent
@@ -161,7 +157,10 @@ __device__ __forceinline__ void row_words(const uint8_t *slot, uint32_t sm0, uin
 }
 
 template <bool PAL, int NT>   // NT: 8-token tiles (1: m <= 8, 2: m <= 16)
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+    k_gemv_sk(const __grid_constant__ CUtensorMap tmW,   // fused: sign/mantissa plane; plain: BF16 W
+              const __grid_constant__ CUtensorMap tmP,   // fused: 4-bit plane (plain: unused)
+              const __grid_constant__ CUtensorMap tmX, const SkArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -178,73 +177,75 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
     if (!defer_x) pdl_wait();
 
     const int stages = a.stages, slot_b = a.slot_bytes, xrows = a.m;
-    const uint32_t ring = smem_addr(smem) + uint32_t(warp * stages * slot_b);
+    // the rings start 128-byte aligned (TMA destinations), the barriers follow
+    uint8_t *base = smem + ((128u - (smem_addr(smem) & 127u)) & 127u);
+    uint8_t *ring = base + warp * stages * slot_b;
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + S * stages * slot_b) + warp * stages;
     const uint32_t k = uint32_t(a.k), gpr = k / 64;
     const int cpr = int(a.cpr);
     const Palette16 P = a.palette;
+    const uint64_t T = a.timeout_ns;
+    if (lane == 0) {
+        for (int s = 0; s < stages; s++) mbar_init(&full[s], 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tmW);
+        if (PAL) prefetch_tensormap(&tmP);
+        prefetch_tensormap(&tmX);
+    }
+    __syncwarp();
 
     // Element offsets below are 32-bit (n * k < 2^32 is checked at launch).
-    // Copy side (lane constants): fused sign/mantissa rows 4q + (lane >> 3),
-    // piece lane & 7; palette rows 8q + (lane >> 2), quarter lane & 3; raw
-    // flags of row lane >> 1, group lane & 1; plain BF16 rows 2q + (lane >> 4),
-    // piece lane & 15.
-    const uint32_t lc_sm = uint32_t(lane >> 3) * k + uint32_t(lane & 7) * 16;
+    // Raw flags: lane l looks up row l / 2, group l % 2 of the unit's chunk.
     const uint32_t lc_flag = uint32_t(lane >> 1) * gpr + uint32_t(lane & 1);
-    const int pr = lane >> 2, pj = lane & 3;
-    const uint32_t lc_bf = uint32_t(lane >> 4) * k + uint32_t(lane & 15) * 8;
-    const uint32_t d_sm = sw128(lane >> 3, lane & 7), d_bf = row256(lane >> 4, lane & 15);
     // consumer side (lane constants): rows g and g + 8, quarter c
     const int fbit_a = 2 * g + (c >> 1), fbit_b = 2 * (g + 8) + (c >> 1);
-    const uint32_t o_sm0 = sw128(g, 2 * c), o_sm1 = sw128(g, 2 * c + 1);
+    const uint32_t o_sm0 = uint32_t(g * 128 + c * 32), o_sm1 = o_sm0 + 16;
     const uint32_t o_pal = uint32_t(kPalOff + g * 64 + c * 16);
-    const uint32_t o_bfa = row256(g, 4 * c), o_bfb = row256(g + 8, 4 * c);
+    const uint32_t o_bfa = uint32_t(g * 256 + c * 64), o_bfb = o_bfa + 8 * 256;
     // X token rows of this lane (clamped: columns >= m are not stored)
-    const uint32_t o_xa = uint32_t(kXOff) + row256(min(g, xrows - 1), 4 * c);
-    const uint32_t o_xb = uint32_t(kXOff) + row256(min(g + 8, xrows - 1), 4 * c);
+    const uint32_t o_xa = uint32_t(kXOff + min(g, xrows - 1) * 256 + c * 64);
+    const uint32_t o_xb = uint32_t(kXOff + min(g + 8, xrows - 1) * 256 + c * 64);
+    const uint32_t w_bytes = PAL ? 16 * 128 + 16 * 64 : 16 * 256, x_bytes = uint32_t(xrows) * 256;
 
-    // W copies of the unit whose first weight is element `uoff` into slot s;
-    // returns this lane's raw flags as a consumer (bit 0: row g, bit 1: row
-    // g + 8, of its quarter).  Each copy instruction of the warp reads whole
-    // 128-byte lines.
-    auto issue_w = [&](uint32_t uoff, int s) -> uint32_t {
-        const uint32_t dst = ring + uint32_t(s * slot_b);
-        if (!PAL) {
-            const uint16_t *src = a.w_bf16 + (uoff + lc_bf);
-#pragma unroll
-            for (int q = 0; q < 8; q++) cp16(dst + d_bf + q * 2 * kRow256, src + size_t(q) * 2 * k);
-            return 0u;
-        }
-        const uint8_t *src = a.sm + (uoff + lc_sm);
-#pragma unroll
-        for (int q = 0; q < 4; q++) cp16(dst + d_sm + q * 512, src + size_t(q) * 4 * k);
-        // raw flags of the unit's 32 (row, group) pairs, one lookup per lane
+    // TMA boxes of unit (tile t, chunk i) into slot s, issued by lane 0; the
+    // slot's barrier expects the X bytes too, so that it cannot complete
+    // before a deferred X box has landed
+    auto issue_w = [&](int64_t t, int i, int s, bool with_x) {
+        if (lane != 0) return;
+        uint8_t *dst = ring + s * slot_b;
+        fence_proxy_async_smem();   // earlier reads of the slot come before the boxes that refill it
+        mbar_arrive_expect_tx(&full[s], w_bytes + x_bytes);
+        tma_load_2d(dst, &tmW, i * kChunkK, int32_t(t * kRows), &full[s]);
+        if (PAL) tma_load_2d(dst + kPalOff, &tmP, i * (kChunkK / 2), int32_t(t * kRows), &full[s]);
+        if (with_x) tma_load_2d(dst + kXOff, &tmX, i * kChunkK, 0, &full[s]);
+    };
+    auto issue_x = [&](int i, int s) {
+        if (lane == 0) tma_load_2d(ring + s * slot_b + kXOff, &tmX, i * kChunkK, 0, &full[s]);
+    };
+    // raw flags of the unit whose first weight is element `uoff`, and this
+    // lane's raw quarters copied into slot s; returns the lane's flags as a
+    // consumer (bit 0: row g, bit 1: row g + 8, of its quarter)
+    auto issue_raw = [&](uint32_t uoff, int s) -> uint32_t {
+        if (!PAL) return 0u;
         const uint32_t gl = (uoff >> 6) + lc_flag;
         const uint32_t fw = __ldg(a.flagbits + (gl >> 5));
         const uint32_t mask = __ballot_sync(0xFFFFFFFFu, (fw >> (gl & 31u)) & 1u);
+        const uint32_t fl = ((mask >> fbit_a) & 1u) | (((mask >> fbit_b) & 1u) << 1);
+        if (fl) {
+            const uint32_t dst = smem_addr(ring + s * slot_b + kRawOff);
 #pragma unroll
-        for (int q = 0; q < 2; q++) {
-            const int r = 8 * q + pr;
-            if ((mask >> (2 * r + (pj >> 1))) & 1u) {
-                // a raw group: the quarter's 32 exponents from the raw plane
-                const uint32_t gg = (uoff >> 6) + uint32_t(r) * gpr + uint32_t(pj >> 1);
+            for (int h = 0; h < 2; h++) {
+                if (!((fl >> h) & 1u)) continue;
+                const int r = g + 8 * h;
+                const uint32_t gg = (uoff >> 6) + uint32_t(r) * gpr + uint32_t(c >> 1);
                 const uint32_t fwg = __ldg(a.flagbits + (gg >> 5)), bg = gg & 31u;
                 const uint32_t rank = __ldg(a.rawbase + (gg >> 5)) + __popc(fwg & ((1u << bg) - 1u));
-                const uint8_t *e = a.rawexp + uint64_t(rank) * kGroup + (pj & 1) * 32;
-                cp16(dst + kRawOff + sw128(r, 2 * pj), e);
-                cp16(dst + kRawOff + sw128(r, 2 * pj + 1), e + 16);
-            } else {
-                cp16(dst + kPalOff + uint32_t(r * 64 + pj * 16), a.pal + ((uoff + uint32_t(r) * k) >> 1) + pj * 16);
+                const uint8_t *e = a.rawexp + uint64_t(rank) * kGroup + (c & 1) * 32;
+                cp16(dst + uint32_t(r * 128 + c * 32), e);
+                cp16(dst + uint32_t(r * 128 + c * 32 + 16), e + 16);
             }
         }
-        return ((mask >> fbit_a) & 1u) | (((mask >> fbit_b) & 1u) << 1);
-    };
-    // X copies of chunk `kc` (K offset) into slot s: m rows of 256 bytes
-    auto issue_x = [&](uint32_t kc, int s) {
-        const uint32_t dst = ring + uint32_t(s * slot_b) + uint32_t(kXOff);
-        for (int p = lane; p < xrows * 16; p += 32) {
-            const int r = p >> 4, j = p & 15;
-            cp16(dst + row256(r, j), a.x + (uint32_t(r) * k + kc + uint32_t(j) * 8));
-        }
+        return fl;
     };
 
     float d0[NT][4], d1[NT][4];
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
     // receives its MMAs in K-step order, as if the unit's pairs were built
     // first.
     auto consume = [&](int s, uint32_t flags) {
-        const uint8_t *slot = smem + (warp * stages + s) * slot_b;
+        const uint8_t *slot = ring + s * slot_b;
         uint32_t smA[8], eA[8], smB[8], eB[8];
         if (PAL) {
             row_words(slot, o_sm0, o_sm1, o_pal, flags & 1u, P, smA, eA);
@@ -356,57 +357,64 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
             }
         }
     };
-    // issue side: the unit after the last one issued, at chunk ii of its
-    // tile, element offset uoff_i; ring slot is_
+    // issue side: the unit after the last one issued: tile it, chunk ii,
+    // element offset uoff_i of its first weight; ring slot is_
     const int c_first = int(u_begin - t_first * cpr);
+    int64_t it = t_first;
     int ii = c_first;
     uint32_t uoff_i = uint32_t(t_first) * 16u * k + uint32_t(ii) * 128u;
     const uint32_t tile_jump = 16u * k - uint32_t(cpr) * 128u;   // past a tile's last chunk -> next tile
-    int is_ = 0;
+    int is_ = 0, ni = 0;    // next slot, units issued
     uint32_t rawbits = 0;   // consumer raw flags, 2 bits per slot
     auto advance = [&]() {
         uoff_i += 128u;
         if (++ii == cpr) {
             ii = 0;
+            ++it;
             uoff_i += tile_jump;
         }
         ++is_;
+        ++ni;
     };
+    // the ring's first units (one copy group each, empty ones included, so
+    // that unit j's raw copies are always group j)
     const int npro = min(stages - 1, nu);
     for (int s = 0; s < stages - 1; s++) {
-        if (s < nu) {
-            if (!defer_x) issue_x(uint32_t(ii) * 128u, s);
-            rawbits |= issue_w(uoff_i, s) << (2 * s);
+        if (s < npro) {
+            issue_w(it, ii, s, !defer_x);
+            rawbits |= issue_raw(uoff_i, s) << (2 * s);
             advance();
         }
         cp_commit();
     }
     if (defer_x) {
-        // the previous kernel has ended: the prologue units' X, one more group
+        // the previous kernel has ended: the prologue units' X boxes
         pdl_wait();
         int cx = c_first;
         for (int s = 0; s < npro; s++) {
-            issue_x(uint32_t(cx) * 128u, s);
+            issue_x(cx, s);
             if (++cx == cpr) cx = 0;
         }
-        cp_commit();
     }
 
     int64_t ct = t_first;
-    int ci = c_first, piece0 = ci, cs = 0;
-    for (int j = 0; j < nu; j++) {
-        // this lane's copies of unit j have landed (with the deferred X group,
-        // the first unit waits for everything issued so far) ...
-        cp_wait(defer_x && j == 0 ? 0 : stages - 2);
-        // ... and every lane's: the slot is read across lanes.  The barrier
-        // also orders every lane's reads of the slot consumed last iteration
-        // before the copies that now refill it.
+    int ci = c_first, piece0 = ci, cs = 0, j = 0;
+    uint32_t phases = 0;   // bit s: parity of slot s's next barrier phase
+    bool dead = false;
+    for (; j < nu; j++) {
+        cp_wait(stages - 2);   // this lane's raw copies of unit j have landed
+        // ... and unit j's boxes (all lanes agree on a time-out)
+        dead = __any_sync(0xFFFFFFFFu, !mbar_wait(&full[cs], (phases >> cs) & 1u, T));
+        if (dead) break;
+        phases ^= 1u << cs;
+        // every lane has read the slot consumed last iteration, which is
+        // refilled now
         __syncwarp();
         const uint32_t fl = (rawbits >> (2 * cs)) & 3u;
         if (j + stages - 1 < nu) {
             if (is_ == stages) is_ = 0;
-            issue_x(uint32_t(ii) * 128u, is_);
-            rawbits = (rawbits & ~(3u << (2 * is_))) | (issue_w(uoff_i, is_) << (2 * is_));
+            issue_w(it, ii, is_, true);
+            rawbits = (rawbits & ~(3u << (2 * is_))) | (issue_raw(uoff_i, is_) << (2 * is_));
             advance();
         }
         cp_commit();
@@ -420,6 +428,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv_sk(const SkArgs a) {
             }
             piece0 = ci;
         }
+    }
+    if (dead) {
+        // time-out: no more work; wait (bounded) for the boxes and copies
+        // this warp has issued, so that none lands after the CTA has exited
+        if (lane == 0) flag_error(a.status, UW_DEVERR_TIMEOUT);
+        for (int u = j; u < ni; u++) mbar_wait(&full[u % stages], uint32_t(u / stages) & 1u, T);
+        cp_async_wait_all();
     }
 }
 
@@ -440,16 +455,34 @@ cudaError_t prepare(K kern, int (&ready)[64]) {
     return cudaSuccess;
 }
 
+// 2-D tensor map over a row-major [rows, inner] array (no swizzle, dense box)
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t rows,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// shared memory of one warp's ring slot and its barrier
+size_t slot_cost(int64_t m) { return size_t(slot_bytes(int(m))) + 8; }
+
 }  // namespace
 
 int gemv_sk_stages(int warps, int stages, int64_t m) {
     if (warps < 1 || warps > kMaxWarps || stages < 0 || stages > kMaxStages || m < 1 || m > 16) return 0;
-    const size_t slot = size_t(slot_bytes(int(m)));
+    const size_t slot = slot_cost(m);
+    const size_t room = size_t(kMaxSmem) - 128;   // less the alignment slack
     if (stages == 0) {   // the deepest ring that fits, at most kMaxStages
-        stages = int(std::min<size_t>(kMaxStages, size_t(kMaxSmem) / (size_t(warps) * slot)));
+        stages = int(std::min<size_t>(kMaxStages, room / (size_t(warps) * slot)));
         return stages >= 2 ? stages : 0;
     }
-    if (stages < 2 || size_t(warps) * stages * slot > size_t(kMaxSmem)) return 0;
+    if (stages < 2 || size_t(warps) * stages * slot > room) return 0;
     return stages;
 }
 
@@ -488,7 +521,13 @@ cudaError_t launch_gemv_sk(const GemvSkLaunch &p, cudaStream_t stream) {
     a.counters = p.counters;
     a.stages = stages;
     a.slot_bytes = slot_bytes(int(p.m));
+    a.status = p.status;
+    a.timeout_ns = p.timeout_ns;
     const bool pal = p.pal != nullptr;
+    CUtensorMap mw, mp, mx;
+    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, uint64_t(p.k), uint64_t(p.m), uint64_t(p.k) * 2,
+                  kChunkK, uint32_t(p.m)))
+        return cudaErrorInvalidValue;
     if (pal) {
         if (!p.w) return cudaErrorInvalidValue;
         a.sm = p.w->sm;
@@ -498,11 +537,20 @@ cudaError_t launch_gemv_sk(const GemvSkLaunch &p, cudaStream_t stream) {
         a.rawexp = p.w->rawexp;
         a.palette = make_palette16(p.w->palette);
         a.w_stable = p.w_stable ? 1 : 0;
+        if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w->sm, uint64_t(p.k), uint64_t(p.n), uint64_t(p.k),
+                      kChunkK, kRows) ||
+            !make_map(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.pal, uint64_t(p.k / 2), uint64_t(p.n), uint64_t(p.k / 2),
+                      kChunkK / 2, kRows))
+            return cudaErrorInvalidValue;
     } else {
         if (!p.w_bf16) return cudaErrorInvalidValue;
         a.w_bf16 = p.w_bf16;
+        if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.w_bf16, uint64_t(p.k), uint64_t(p.n),
+                      uint64_t(p.k) * 2, kChunkK, kRows))
+            return cudaErrorInvalidValue;
+        mp = mw;
     }
-    const size_t smem = size_t(p.warps) * stages * size_t(a.slot_bytes);
+    const size_t smem = size_t(p.warps) * stages * slot_cost(p.m) + 128;
     const dim3 grid(unsigned(g.G)), block(unsigned(p.warps * 32));
     cudaError_t err = cudaSuccess;
 #define UW_SK_LAUNCH(P_, N_)                                                    \
@@ -510,7 +558,7 @@ cudaError_t launch_gemv_sk(const GemvSkLaunch &p, cudaStream_t stream) {
         static int ready[64] = {0};                                             \
         err = prepare(k_gemv_sk<P_, N_>, ready);                                \
         if (err == cudaSuccess)                                                 \
-            err = launch_pdl(a.w_stable != 0, k_gemv_sk<P_, N_>, grid, block, smem, stream, a); \
+            err = launch_pdl(a.w_stable != 0, k_gemv_sk<P_, N_>, grid, block, smem, stream, mw, mp, mx, a); \
     } while (0)
     if (pal) {
         if (g.NT == 2) UW_SK_LAUNCH(true, 2); else UW_SK_LAUNCH(true, 1);

@@ -103,10 +103,10 @@ int sm_count();
 // Persistent stream-K form of the warp-MMA kernel, m <= 16, k a multiple of
 // 128 and n * k < 2^32 (gemv_sk.cu): one CTA of `warps` warps per SM, every
 // warp an equal contiguous run of (16-row tile, 128-wide K chunk) units, its
-// loads (W and the chunk's X rows) in a shared-memory ring of `stages` slots
-// of 5120 + 288 m bytes (0 = the deepest that fits) filled by cp.async; a
-// tile cut between warps is summed in warp order by the warp that finishes
-// its last piece.  Workspace: `counters` (one u32 per tile,
+// loads (W and the chunk's X rows, 2-D TMA boxes) in a shared-memory ring of
+// `stages` slots of 5120 + 256 m bytes plus an 8-byte barrier (0 = the
+// deepest that fits); a tile cut between warps is summed in warp order by
+// the warp that finishes its last piece.  Workspace: `counters` (one u32 per tile,
 // zero before the call and left zero by it) and `partial` (two fragment
 // sets of 32 x 4 x NT floats per warp).  pal == nullptr: plain BF16 `w_bf16`.
 struct GemvSkGeometry {
@@ -127,6 +127,8 @@ struct GemvSkLaunch {
     float *partial;
     int warps, stages;
     bool w_stable;             // fused: the planes are the blob's (read before the previous kernel ends)
+    uint32_t *status;          // device error word (time-out), may be null
+    uint64_t timeout_ns;       // bound of every wait in the kernel
 };
 cudaError_t launch_gemv_sk(const GemvSkLaunch &p, cudaStream_t stream);
 

@@ -233,7 +233,7 @@ typedef enum uw_kernel {
                             UW_KERNEL_MMA, one CTA of `bn` (1..16) warps per SM;
                             every warp owns an equal contiguous run of (16-row
                             tile, 128-wide K chunk) units and stages its loads
-                            in a shared-memory ring filled by cp.async; a tile
+                            in a shared-memory ring filled by 2-D TMA boxes; a tile
                             cut between warps is summed in warp (= K) order by
                             the warp that finishes its last piece.  Needs a
                             workspace whose tile counters are zero, as TC_SK;
@@ -259,9 +259,9 @@ typedef struct uw_plan {
                              fits (at most 6 / 8);
                              MMA: weights per lane and row per step, 1 = 16, 2 = 32
                              (K a multiple of 128), 0 = 32 when K allows, else 16;
-                             MMA_SK: ring slots per warp (2..8) of 5120 + 288 m
-                             bytes each, bn x stages slots within 227 KB; 0 = the
-                             deepest that fits, at most 8 */
+                             MMA_SK: ring slots per warp (2..8) of 5128 + 256 m
+                             bytes each, bn x stages slots within 227 KB less
+                             128 bytes; 0 = the deepest that fits, at most 8 */
     uint32_t debug_flags; /* UW_DEBUG_* (0 in production) */
     int64_t timeout_ns;   /* spin-wait limit inside kernels (0 = 2 s) */
 } uw_plan;

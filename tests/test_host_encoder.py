@@ -266,12 +266,13 @@ def test_stream_k_gemv_plans_and_workspace(uw):
     """UW_KERNEL_MMA_SK: tile counters (one u32 per 16-row tile, 256-byte
     rounded) then two fragment sets (32 lanes x 4 floats per 8-token tile) per
     warp of the grid; with no GPU the library sizes the grid for 148 SMs.  A
-    ring slot holds 5120 + 288 m bytes and a CTA's slots must fit 227 KB."""
+    ring slot and its barrier take 5128 + 256 m bytes, and a CTA's slots must
+    fit 227 KB less 128 bytes of alignment slack."""
     def up(x):
         return (x + 255) // 256 * 256
 
     def fits(warps, stages, m):
-        return warps * stages * (5120 + 288 * m) <= 227 * 1024
+        return warps * stages * (5128 + 256 * m) <= 227 * 1024 - 128
 
     n, k = 14336, 4096
     tiles, units = n // 16, n // 16 * (k // 128)
