@@ -585,13 +585,24 @@ def run_gpu(args, rank, world):
     # previous step still reads the other), its 12 matmuls run back to back
     # into one of two result sets (so the early start of each matmul is not
     # broken by event operations between them), and the step's results come
-    # down on another copy stream while the next step computes.
-    hx = {(c["m"], c["mat"].k): c["x"].cpu().pin_memory() for c in calls}
-    hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
-    h2d = sum(t.numel() * 2 for t in hx.values())
-    d2h = sum(t.numel() * 4 for t in hy)
-    xsets = [{key: xs[key[0]][key[1]] for key in hx}, {key: xs[key[0]][key[1]].clone() for key in hx}]
-    ysets = [[c["y"] for c in calls], [torch.empty_like(c["y"]) for c in calls]]
+    # down on another copy stream while the next step computes.  A step's
+    # inputs are one pinned host buffer (every (M, K) activation block back to
+    # back) and go up in one copy; its 12 results are views of one device
+    # buffer and come down in one copy: few large copies, not 20 small ones.
+    xkeys = sorted({(c["m"], c["mat"].k) for c in calls})
+    x_off = np.cumsum([0] + [m * k for m, k in xkeys])
+    y_off = np.cumsum([0] + [c["m"] * c["mat"].n for c in calls])
+    hx = torch.empty(int(x_off[-1]), dtype=torch.int16).pin_memory()
+    for i, (m, k) in enumerate(xkeys):
+        hx[int(x_off[i]):int(x_off[i + 1])].copy_(xs[m][k].reshape(-1).cpu())
+    hy = torch.empty(int(y_off[-1]), dtype=torch.float32).pin_memory()
+    h2d, d2h = hx.numel() * 2, hy.numel() * 4
+    dx = [torch.empty_like(hx, device=dev) for _ in range(2)]
+    dy = [torch.empty_like(hy, device=dev) for _ in range(2)]
+    xsets = [{key: dx[b][int(x_off[i]):int(x_off[i + 1])].view(key[0], key[1]) for i, key in enumerate(xkeys)}
+             for b in range(2)]
+    ysets = [[dy[b][int(y_off[i]):int(y_off[i + 1])].view(c["m"], c["mat"].n) for i, c in enumerate(calls)]
+             for b in range(2)]
     copy_in, copy_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     mk = lambda: torch.cuda.Event()
     x_ready = [mk() for _ in range(args.steps)]
@@ -606,8 +617,7 @@ def run_gpu(args, rank, world):
         xset, yset = xsets[s & 1], ysets[s & 1]
         copy_in.wait_event(e0 if s < 2 else x_free[s - 2])     # matmuls of step s-2 read this set
         with torch.cuda.stream(copy_in):
-            for key, t in hx.items():
-                xset[key].copy_(t, non_blocking=True)
+            dx[s & 1].copy_(hx, non_blocking=True)
         x_ready[s].record(copy_in)
         stream.wait_event(x_ready[s])
         if s >= 2:
@@ -618,8 +628,7 @@ def run_gpu(args, rank, world):
         y_ready[s].record(stream)
         copy_out.wait_event(y_ready[s])
         with torch.cuda.stream(copy_out):
-            for h, y in zip(hy, yset):
-                h.copy_(y, non_blocking=True)
+            hy.copy_(dy[s & 1], non_blocking=True)
         y_free[s].record(copy_out)
     stream.wait_stream(copy_out)                                # every result is on the host
     e1.record(stream)
