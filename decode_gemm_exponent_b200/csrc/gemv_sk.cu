@@ -23,8 +23,9 @@
 //    to the number of pieces adds them in warp order (= K order), so the
 //    result does not depend on timing, and zeroes each piece after reading
 //    it, so that a completed call leaves its whole scratch (counters and
-//    pieces) zero.  No warp ever waits for another one: there are no
-//    barriers and no spin waits in this kernel.
+//    pieces) zero.  No warp ever waits for another one: a warp waits only
+//    on its own ring slots' barriers (for the boxes its own lane issued)
+//    and on its lanes' own copies; there are no CTA-wide barriers.
 // Per unit, lane (g, c) = (lane / 4, lane % 4) handles rows g and g + 8 of
 // the tile and weights [32c, 32c + 32) of the chunk, with the same fragment
 // map as the one-tile kernel at 32 weights per lane (MMA K-step j, thread c,
