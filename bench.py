@@ -62,6 +62,7 @@ WORKLOAD = "llama-3.1-8b MLP layer (gate/up/down), M in {1,4,16,64}, autotuned p
 L2_NOTE = "no flush: each matrix is re-read after >= 160 MB of other matrices (inputs larger than L2)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ORACLE_ROW_FRACTION = 16      # the oracle sample keeps 1/16 of each matrix's rows
+ORACLE_PART_ROWS = 128        # ... in parts of 128 rows, one pool task each
 
 
 def rank_seed(proj_index: int, rank: int) -> int:
@@ -177,8 +178,10 @@ class ClockSampler:
 # The oracle runs the step's 12 calls (decode of the matrix + float64 matmul,
 # as pipeline 1 does per call) on a row sample of each matrix: the first
 # 1/ORACLE_ROW_FRACTION of its rows, encoded on its own by the oracle (same
-# recipe and seeds, so the same weight statistics).  Calls run in a spawn
-# process pool, one call per task; a step's wall time covers all 12.
+# recipe and seeds, so the same weight statistics).  Each call's sample is
+# cut into parts of ORACLE_PART_ROWS rows, each encoded on its own, so that a
+# step is many equal-sized tasks and a spawn process pool on every host core
+# stays busy; a step's wall time covers all 12 calls.
 
 _ORACLE = {}
 
@@ -187,29 +190,37 @@ def oracle_sample_rows(n: int) -> int:
     return max(64, n // ORACLE_ROW_FRACTION)
 
 
+def oracle_parts(n: int) -> int:
+    return max(1, oracle_sample_rows(n) // ORACLE_PART_ROWS)
+
+
 def _oracle_init(rank: int):
     from oracle import oracle as O
     from decode_gemm_exponent_b200 import synth
     for i, (_, n, k) in enumerate(PROJ):
         w = synth.weights_bf16(n, k, 0.02, 0.0005, 1.0, seed=rank_seed(i, rank))[:oracle_sample_rows(n)]
-        _ORACLE[i] = O.encode(w)                      # offline, untimed
+        rows = w.shape[0] // oracle_parts(n)
+        for p in range(oracle_parts(n)):              # offline, untimed
+            _ORACLE[("w", i, p)] = O.encode(w[p * rows:(p + 1) * rows])
     for m in MS:
         for k in {p[2] for p in PROJ}:
-            _ORACLE[(m, k)] = synth.activations_bf16(m, k, seed=m)
+            _ORACLE[("x", m, k)] = synth.activations_bf16(m, k, seed=m)
 
 
 def _oracle_call(task):
     from oracle import oracle as O
-    i, m = task
-    enc = _ORACLE[i]
+    i, m, p = task
+    enc = _ORACLE[("w", i, p)]
     t0 = time.perf_counter()
     wd = O.decode(enc)
-    O.gemm(_ORACLE[(m, enc.k)], wd)
+    O.gemm(_ORACLE[("x", m, enc.k)], wd)
     return time.perf_counter() - t0
 
 
 def oracle_tasks():
-    return [(i, m) for m in MS for i in range(len(PROJ))]
+    # the largest calls first, so that the pool ends on short tasks
+    tasks = [(i, m, p) for m in MS for i, (_, n, _) in enumerate(PROJ) for p in range(oracle_parts(n))]
+    return sorted(tasks, key=lambda t: -t[1] * PROJ[t[0]][2])
 
 
 def oracle_step_bytes() -> int:
@@ -219,7 +230,8 @@ def oracle_step_bytes() -> int:
 def oracle_sample_text(workers: int) -> str:
     rows = ", ".join("%s %d of %d rows" % (nm, oracle_sample_rows(n), n) for nm, n, _ in PROJ)
     return ("the step's 12 calls (M in %s x gate/up/down), each bit-by-bit Huffman decode + float64 matmul, "
-            "on a row sample (%s), %d worker process%s" % (list(MS), rows, workers, "" if workers == 1 else "es"))
+            "on a row sample (%s) in parts of %d rows, %d worker process%s"
+            % (list(MS), rows, ORACLE_PART_ROWS, workers, "" if workers == 1 else "es"))
 
 
 class OracleRunner:

@@ -139,9 +139,13 @@ def test_oracle_sample_is_the_step_on_a_row_sample():
     """The reference arm and the CPU baseline run the step's 12 calls on the
     first 1/16 of each matrix's rows; both arms print the same config."""
     tasks = bench.oracle_tasks()
-    assert sorted(tasks) == sorted((i, m) for m in bench.MS for i in range(len(bench.PROJ)))
     rows = [bench.oracle_sample_rows(n) for _, n, _ in bench.PROJ]
     assert rows == [896, 896, 256]
+    # every call's sample in 128-row parts: 7, 7 and 2 parts per M
+    assert [bench.oracle_parts(n) for _, n, _ in bench.PROJ] == [7, 7, 2]
+    assert sorted(tasks) == sorted((i, m, p) for m in bench.MS for i in range(len(bench.PROJ))
+                                   for p in range(bench.oracle_parts(bench.PROJ[i][1])))
+    assert all(r % bench.ORACLE_PART_ROWS == 0 for r in rows)
     assert bench.oracle_step_bytes() == sum(2 * r * k for r, (_, _, k) in zip(rows, bench.PROJ)) * len(bench.MS)
     assert bench.workload_config() == {"workload": bench.WORKLOAD, "l2": bench.L2_NOTE}
     assert "12 calls" in bench.oracle_sample_text(4) and "4 worker processes" in bench.oracle_sample_text(4)
