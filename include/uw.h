@@ -376,7 +376,11 @@ uw_status uw_fused_matmul_noalloc(const uint16_t *x_dev, int64_t m, const uw_dma
 
 /* For every matrix mats[i] and batch size ms[j], time the candidate
  * (pipeline, kernel, bn, split_k) plans with CUDA events on `stream` and
- * store the fastest in plans_out[i*n_ms + j].  Every timed call is preceded
+ * store the fastest in plans_out[i*n_ms + j].  The candidates cover every
+ * kernel but UW_KERNEL_MMA_SK, which occupies whole SMs and so cannot start
+ * while the previous call drains: it can win such isolated timings and still
+ * slow a sequence of calls down, so it is used by explicit plan only.  Every
+ * timed call is preceded
  * by a 192 MB read of the end of the workspace, so the weights come from HBM
  * (not from the 126 MB L2), as they do when a model's layers run in turn.
  * x_dev must hold at least max(ms) x max(k) BF16 values, y_dev max(ms) x
