@@ -262,6 +262,28 @@ def test_plans_and_workspace(uw):
         uw.workspace_size(4, n, 1600, uw.make_plan(kernel=uw.KERNEL_MMA, bn=2, stages=2))
 
 
+def test_binding_constants_match_the_header(uw):
+    """Every enum value and flag the binding passes across the ABI equals the
+    one include/uw.h declares (the binding restates them by hand)."""
+    with open(os.path.join(ROOT, "include", "uw.h"), encoding="utf-8") as f:
+        text = re.sub(r"/\*.*?\*/", " ", f.read(), flags=re.S)
+    decl = {name: int(val) for name, val in re.findall(r"\b(UW_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+    decl.update({name: int(val) for name, val in re.findall(r"#define\s+(UW_[A-Z0-9_]+)\s+(\d+)u?\b", text)})
+    pairs = {"UW_OK": uw.UW_OK, "UW_EMIT_HUFFMAN": uw.EMIT_HUFFMAN, "UW_EMIT_PALETTE": uw.EMIT_PALETTE}
+    for name in ("INVALID_ARG", "UNSUPPORTED_SHAPE", "CORRUPT", "CUDA", "NOMEM", "TIMEOUT", "WORKSPACE"):
+        pairs["UW_ERR_" + name] = getattr(uw, "ERR_" + name)
+    for name in ("SM", "RAWEXP", "FLAGS", "RAWBASE", "STREAM", "CHUNKOFF", "DLUT", "PAL"):
+        pairs["UW_SEC_" + name] = getattr(uw, "SEC_" + name)
+    for name in ("DECODE_GEMM", "DECODE_EXP_FUSED", "TRANSCODE_FUSED", "DIRECT_PALETTE", "HUFFMAN_FUSED"):
+        pairs["UW_PIPE_" + name] = getattr(uw, "PIPE_" + name)
+    for name in ("FMA", "TC", "MMA", "TC_SK", "MMA_SK"):
+        pairs["UW_KERNEL_" + name] = getattr(uw, "KERNEL_" + name)
+    for name, value in pairs.items():
+        assert decl.get(name) == value, (name, decl.get(name), value)
+    # and every kernel the header declares has a name in the binding's plan files
+    assert sorted(uw.KERNEL_NAMES) == sorted(v for n, v in decl.items() if n.startswith("UW_KERNEL_"))
+
+
 def test_stream_k_gemv_plans_and_workspace(uw):
     """UW_KERNEL_MMA_SK: tile counters (one u32 per 16-row tile, 256-byte
     rounded) then two fragment sets (32 lanes x 4 floats per 8-token tile) per
